@@ -1,0 +1,589 @@
+"""Benchmark of the B200 BitLinear (W1.58A8) path.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+
+One step is one pass of the hot path over one batch of synthetic input: the
+prefill workload of the 2B model's projection shapes, M = 4096 tokens through
+(K, N) = (2560, 6912) and (6912, 2560), each as RMSNorm prelude + per-token
+int8 quant (bitnet_quant_act) followed by the int8 x ternary contraction with
+its bf16 dequant epilogue (bitnet_linear).  The packed weights are prepared
+once (the pages' packed checkpoint stores them ternary, "offline").
+
+Prints ONE JSON line (rank 0).  `value` is int8 TOPS (2*M*N*K per projection,
+zero weights not skipped) over all ranks; `roofline` is the tcgen05 GEMM's
+achieved fraction of the int8 tensor peak; `e2e` is the same step through the
+C ABI with host buffers (pinned H2D of the activations, D2H of the outputs);
+`cpu_baseline` is the CPU oracle on a bounded sample of the same step;
+`workloads` adds the decode GEMV streaming bandwidth and the FFN / H-FFN /
+tiny configurations.
+
+Under torchrun (N > 1) every rank runs the same step on its own GPU (the
+projection is independent per token, so tokens shard with no data-path
+collective: weak scaling); the elapsed time is the max over ranks.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "BitLinear W1.58A8 int8 TOPS (prefill) & GB/s (decode), % of roofline on 1 B200"
+PREFILL_M = 4096
+PREFILL_KN = ((2560, 6912), (6912, 2560))
+DECODE_M = (1, 4, 16)
+DECODE_KN = ((2560, 2560), (2560, 6912), (6912, 2560))
+GEMM_KERNEL_SRC = os.path.join(ROOT, "ternary_weight_token_b200", "csrc", "gemm_tc.cuh")
+GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_tc_prefill_4096x2560x6912.md")
+
+
+def prefill_ops():
+    return sum(2 * PREFILL_M * N * K for K, N in PREFILL_KN)
+
+
+def decode_bytes(M, K, N):
+    """Algorithmic bytes of one decode call: packed weights + codes + scales +
+    bf16 outputs + gamma."""
+    return N * K // 4 + M * K + 4 * M + 2 * M * N + 4
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value, dist, device=None):
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="bench_clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "50"], stdout=self.out,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        self.t0 = time.time()
+
+    def stop(self, window):
+        if self.proc is None:
+            return None
+        time.sleep(0.06)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[5:]))
+                except (ValueError, IndexError):
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        t_start, t_end = window
+        inside = [r for r in rows if t_start - 0.05 <= r[0] <= t_end + 0.05]
+        note = "samples inside the timed region"
+        if not inside:
+            inside = rows
+            note = "timed region shorter than the 50 ms sample period: samples around it"
+        names = ["active", "hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        reasons = set()
+        for r in inside:
+            for name, val in zip(names[1:], r[3][1:]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r[1] for r in inside),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": sorted(reasons),
+                "samples": len(inside), "note": note}
+
+
+# ------------------------------------------------------------- references
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per GEMM launch from the committed ncu summary, or None when
+    the summary is missing or the kernel source changed since the capture."""
+    if not os.path.exists(GEMM_PROFILE):
+        return None
+    txt = open(GEMM_PROFILE).read()
+    m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", txt)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", txt)
+    if not m_sha or not m_b or m_sha.group(1) != file_sha(GEMM_KERNEL_SRC):
+        return None
+    return int(m_b.group(1))
+
+
+# ---------------------------------------------------------- CPU reference
+
+def oracle_prefill_sample(target_s=12.0, max_tokens=PREFILL_M):
+    """Time the oracle on a bounded token sample of the prefill step."""
+    import oracle
+    threads = oracle.num_threads()
+    prepared = []
+    for i, (K, N) in enumerate(PREFILL_KN):
+        inp = synthetic.linear_inputs(PREFILL_M, K, N, seed=i)
+        g, T, _ = oracle.quantize_weights(inp["W"])
+        prepared.append((K, N, inp["X"], T, g))
+
+    def run(tokens):
+        t0 = time.perf_counter()
+        for K, N, X, T, g in prepared:
+            y = oracle.bitlinear(X[:tokens], T, g, oracle.PRELUDE_RMSNORM, eps=1e-5)
+            oracle.round_bf16(y)
+        return time.perf_counter() - t0
+
+    tokens = 8
+    dt = run(tokens)
+    if dt < target_s:
+        tokens = int(min(max_tokens, max(8, tokens * target_s / max(dt, 1e-3) * 0.8)))
+        dt = run(tokens)
+    ops = sum(2 * tokens * N * K for K, N in PREFILL_KN)
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",
+            "sample": f"{tokens} of the {PREFILL_M} tokens of one prefill step (both "
+                      f"projections: RMSNorm + int8 quant + int64 contraction + fp64 dequant + "
+                      f"bf16 round), {dt:.1f} s on {threads} OpenMP threads"}
+
+
+def run_reference(args, world, rank):
+    """Reference arm: the CPU oracle as it stands, on this host's cores."""
+    if rank != 0:
+        return 0
+    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    import oracle
+    threads = oracle.num_threads()
+    prepared = []
+    for i, (K, N) in enumerate(PREFILL_KN):
+        inp = synthetic.linear_inputs(PREFILL_M, K, N, seed=i)
+        g, T, _ = oracle.quantize_weights(inp["W"])
+        prepared.append((K, N, inp["X"], T, g))
+
+    def step(tokens, off):
+        for K, N, X, T, g in prepared:
+            rows = X[off:off + tokens]
+            oracle.round_bf16(oracle.bitlinear(rows, T, g, oracle.PRELUDE_RMSNORM, eps=1e-5))
+
+    t0 = time.perf_counter()
+    step(2, 0)
+    dt = time.perf_counter() - t0
+    tokens = int(max(1, min(PREFILL_M, 2 * per_step / max(dt, 1e-4))))
+    for i in range(args.warmup):
+        step(tokens, (i * tokens) % (PREFILL_M - tokens + 1))
+    times = []
+    for i in range(args.steps):
+        t0 = time.perf_counter()
+        step(tokens, (i * tokens) % (PREFILL_M - tokens + 1))
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    ops = sum(2 * tokens * N * K for K, N in PREFILL_KN) * args.steps
+    value = ops / total / 1e12
+    sample = (f"{tokens} tokens of the {PREFILL_M}-token prefill step per step (both projections,"
+              f" RMSNorm + quant + contraction + dequant + bf16 round)")
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"prefill BitLinear M={PREFILL_M}, (K,N)=(2560,6912)+(6912,2560)"
+                                   ", RMSNorm prelude, bf16 out", "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------ GPU timing
+
+class Prefill:
+    """Device buffers and the launch sequence of one prefill step."""
+
+    def __init__(self, torch, bn, device):
+        self.torch, self.bn = torch, bn
+        self.shapes = []
+        for i, (K, N) in enumerate(PREFILL_KN):
+            inp = synthetic.linear_inputs(PREFILL_M, K, N, seed=i)
+            W = torch.from_numpy(inp["W"]).to(device)
+            P, g, ws = bn.alloc_packed(N, K, device)
+            bn.bitnet_pack_weights(W, P, g, ws)
+            del W
+            X = torch.from_numpy(inp["X"]).to(device)
+            q, s, rs = bn.alloc_quant(PREFILL_M, K, device)
+            Y = torch.empty((PREFILL_M, N), dtype=torch.bfloat16, device=device)
+            self.shapes.append({"K": K, "N": N, "X": X, "P": P, "g": g, "q": q, "s": s,
+                                "rs": rs, "Y": Y, "X_host": None, "Y_host": None})
+        torch.cuda.synchronize()
+        self.launches_per_step = 2 * len(self.shapes)
+
+    def step(self, gemm_events=None):
+        bn = self.bn
+        for i, sh in enumerate(self.shapes):
+            bn.bitnet_quant_act(sh["X"], sh["q"], sh["s"], sh["rs"],
+                                prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
+            if gemm_events is not None:
+                gemm_events[i][0].record()
+            bn.bitnet_linear(sh["q"], sh["s"], sh["rs"], sh["P"], sh["g"], sh["K"], sh["Y"])
+            if gemm_events is not None:
+                gemm_events[i][1].record()
+
+    def e2e_buffers(self):
+        torch = self.torch
+        for sh in self.shapes:
+            if sh["X_host"] is None:
+                sh["X_host"] = sh["X"].cpu().pin_memory()
+                sh["Y_host"] = torch.empty(sh["Y"].shape, dtype=sh["Y"].dtype).pin_memory()
+
+    def e2e_step(self):
+        bn = self.bn
+        for sh in self.shapes:
+            sh["X"].copy_(sh["X_host"], non_blocking=True)
+            bn.bitnet_quant_act(sh["X"], sh["q"], sh["s"], sh["rs"],
+                                prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
+            bn.bitnet_linear(sh["q"], sh["s"], sh["rs"], sh["P"], sh["g"], sh["K"], sh["Y"])
+            sh["Y_host"].copy_(sh["Y"], non_blocking=True)
+
+    def h2d_bytes(self):
+        return sum(sh["X"].numel() * sh["X"].element_size() for sh in self.shapes)
+
+    def d2h_bytes(self):
+        return sum(sh["Y"].numel() * sh["Y"].element_size() for sh in self.shapes)
+
+
+def time_loop(torch, fn, steps):
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        fn()
+    end.record()
+    end.synchronize()
+    return start.elapsed_time(end) / 1e3
+
+
+def bench_decode(torch, bn, device, reps=3):
+    """Steady-state decode GEMV streaming: a CUDA graph of back-to-back calls
+    over a pool of distinct packed-weight copies larger than twice the L2."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    out = []
+    for (K, N) in DECODE_KN:
+        inp = synthetic.linear_inputs(max(DECODE_M), K, N, seed=K + N)
+        W = torch.from_numpy(inp["W"]).to(device)
+        P0, g, ws = bn.alloc_packed(N, K, device)
+        bn.bitnet_pack_weights(W, P0, g, ws)
+        del W
+        wbytes = P0.numel()
+        pool = max(8, int(2 * l2 // wbytes) + 2)
+        pool_bufs = [P0.clone() for _ in range(pool)]
+        X = torch.from_numpy(inp["X"]).to(device)
+        for M in DECODE_M:
+            q, s, rs = bn.alloc_quant(M, K, device)
+            bn.bitnet_quant_act(X[:M].contiguous(), q, s, rs)
+            Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            for Pb in pool_bufs[:2]:
+                bn.bitnet_linear(q, s, rs, Pb, g, K, Y)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            stream = torch.cuda.Stream(device)
+            with torch.cuda.stream(stream):
+                graph.capture_begin(capture_error_mode="thread_local")
+                for Pb in pool_bufs:
+                    bn.bitnet_linear(q, s, rs, Pb, g, K, Y, stream=stream)
+                graph.capture_end()
+            torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            best = None
+            for _ in range(reps):
+                dt = time_loop(torch, graph.replay, 4)
+                best = dt if best is None else min(best, dt)
+            calls = 4 * pool
+            gbs = decode_bytes(M, K, N) * calls / best / 1e9
+            out.append({"M": M, "K": K, "N": N, "us_per_call": best / calls * 1e6,
+                        "GB_s": gbs, "weights_in_pool": pool})
+            del graph
+        del pool_bufs
+        torch.cuda.empty_cache()
+    return out
+
+
+def bench_ffn(torch, bn, device, iters=20):
+    cfg = synthetic.WORKLOADS["ffn"].dims
+    M, H, I = cfg["M"], cfg["H"], cfg["I"]
+    inp = synthetic.ffn_inputs(M, H, I, seed=0)
+    packs = []
+    for k in ("Wg", "Wu", "Wd"):
+        W = torch.from_numpy(inp[k]).to(device)
+        P, g, ws = bn.alloc_packed(*W.shape, device)
+        bn.bitnet_pack_weights(W, P, g, ws)
+        packs.append((P, g))
+    X = torch.from_numpy(inp["x_bf16"].view(np.int16)).to(device).view(torch.bfloat16)
+    Y = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+    ws = bn.alloc_ffn_workspace(M, H, I, device=device)
+
+    def run():
+        bn.bitnet_ffn(X, packs[0][0], packs[0][1], packs[1][0], packs[1][1], packs[2][0],
+                      packs[2][1], Y, ws, variant=bn.BITNET_FFN_RELU2_GLU, eps=1e-5)
+    for _ in range(3):
+        run()
+    dt = time_loop(torch, run, iters) / iters
+    ops = 2 * 2 * M * H * I + 2 * M * I * H
+    return {"M": M, "H": H, "I": I, "us": dt * 1e6, "TOPS": ops / dt / 1e12}
+
+
+def bench_hffn(torch, bn, device, iters=50):
+    cfg = synthetic.WORKLOADS["hffn"].dims
+    M, D, F = cfg["M"], cfg["D"], cfg["F"]
+    inp = synthetic.hffn_inputs(M, D, F, seed=0)
+    packs = []
+    for k in ("W1", "W2"):
+        W = torch.from_numpy(inp[k]).to(device)
+        P, g, ws = bn.alloc_packed(*W.shape, device)
+        bn.bitnet_pack_weights(W, P, g, ws)
+        packs.append((P, g))
+    X = torch.from_numpy(inp["X"]).to(device)
+    Y = torch.empty((M, D), device=device)
+    ws = bn.alloc_ffn_workspace(M, D, F, bn.BITNET_FFN_HADAMARD_SILU, device=device)
+
+    def run():
+        bn.bitnet_ffn(X, packs[0][0], packs[0][1], None, None, packs[1][0], packs[1][1], Y, ws,
+                      variant=bn.BITNET_FFN_HADAMARD_SILU)
+    for _ in range(3):
+        run()
+    dt = time_loop(torch, run, iters) / iters
+    ops = 2 * 2 * M * D * F
+    return {"M": M, "D": D, "F": F, "us": dt * 1e6, "TOPS": ops / dt / 1e12}
+
+
+def bench_tiny(torch, bn, device, iters=200):
+    d = synthetic.WORKLOADS["tiny"].dims
+    M, K, N = d["M"], d["K"], d["N"]
+    inp = synthetic.linear_inputs(M, K, N, seed=0)
+    W = torch.from_numpy(inp["W"]).to(device)
+    P, g, ws = bn.alloc_packed(N, K, device)
+    bn.bitnet_pack_weights(W, P, g, ws)
+    X = torch.from_numpy(inp["X"]).to(device)
+    q, s, rs = bn.alloc_quant(M, K, device)
+    Y = torch.empty((M, N), device=device)
+
+    def run():
+        bn.bitnet_quant_act(X, q, s, rs)
+        bn.bitnet_linear(q, s, rs, P, g, K, Y)
+    for _ in range(5):
+        run()
+    dt = time_loop(torch, run, iters) / iters
+    return {"M": M, "K": K, "N": N, "us_per_call": dt * 1e6,
+            "note": "quant + linear, launch-latency bound"}
+
+
+def run_b200(args, world, rank, local):
+    import torch
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}), flush=True)
+        return 1
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    import ternary_weight_token_b200 as bn
+    bn.library()
+    peaks = measured_peaks()
+
+    pre = Prefill(torch, bn, device)
+    for _ in range(max(3, args.warmup)):
+        pre.step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+
+    # ---- timed region: K steps; every GEMM launch is bracketed by CUDA events
+    # recorded on the stream it is launched on (torch's current stream)
+    n_sh = len(pre.shapes)
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(n_sh)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.15)
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    t_wall0 = time.time()
+    start.record()
+    for s in range(args.steps):
+        pre.step(evs[s])
+    end.record()
+    end.synchronize()
+    t_wall1 = time.time()
+    elapsed = start.elapsed_time(end) / 1e3
+    clocks = sampler.stop((t_wall0, t_wall1))
+    gemm_avg = [sum(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps))
+                / args.steps / 1e3 for i in range(n_sh)]
+    if dist is not None:
+        dist.barrier()
+    elapsed = max_over_ranks(elapsed, dist, device)
+
+    ms_per_step = elapsed / args.steps * 1e3
+    value = world * prefill_ops() * args.steps / elapsed / 1e12
+
+    # ---- e2e through the C ABI with host buffers
+    pre.e2e_buffers()
+    e2e_steps = max(3, min(args.steps, 20))
+    for _ in range(2):
+        pre.e2e_step()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    e2e_elapsed = time_loop(torch, pre.e2e_step, e2e_steps)
+    e2e_elapsed = max_over_ranks(e2e_elapsed, dist, device)
+    e2e_value = world * prefill_ops() * e2e_steps / e2e_elapsed / 1e12
+
+    # ---- roofline of the dominant kernel (tcgen05 GEMM)
+    int8_peak = 2.0 * peaks["bf16_tflops"]
+    gemm_ops = [2 * PREFILL_M * N * K for K, N in PREFILL_KN]
+    achieved = sum(gemm_ops) / sum(gemm_avg) / 1e12
+    traffic = profiled_traffic()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": int8_peak, "unit": "TOP/s",
+                "frac": achieved / int8_peak, "traffic": traffic,
+                "kernel": "gemm_tc_kernel (tcgen05.mma kind::i8)",
+                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} TF/s x 2 "
+                               "(int8/bf16 nominal ratio 4.5/2.25)",
+                "per_launch_us": [t * 1e6 for t in gemm_avg],
+                "ops_per_launch": gemm_ops}
+
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8", "data": "synthetic",
+            "config": {"workload": f"prefill BitLinear M={PREFILL_M} tokens per GPU, (K,N)="
+                                   "(2560,6912)+(6912,2560), RMSNorm prelude + per-token int8 "
+                                   "quant + ternary contraction + bf16 dequant",
+                       "M": PREFILL_M, "shapes": [list(s) for s in PREFILL_KN],
+                       "l2": "inputs larger than L2: 155 MB of fp32 activations and 113 MB of "
+                             "bf16 outputs per step",
+                       "parallelism": f"dp{world} (tokens sharded, no data-path collective)"},
+            "roofline": roofline,
+            "e2e": {"value": e2e_value, "unit": "TOPS",
+                    "h2d_bytes_per_step": pre.h2d_bytes(),
+                    "d2h_bytes_per_step": pre.d2h_bytes(), "steps": e2e_steps},
+            "gpu_launches": pre.launches_per_step * args.steps,
+            "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_prefill_sample(target_s=args.cpu_seconds)
+    if rank == 0 and not args.no_extra:
+        dec = bench_decode(torch, bn, device)
+        for d in dec:
+            d["frac_of_hbm"] = d["GB_s"] / peaks["hbm_gbs"]
+        line["workloads"] = {
+            "decode": dec,
+            "decode_peak_source": f"{peaks['source']} HBM copy {peaks['hbm_gbs']} GB/s",
+            "ffn": bench_ffn(torch, bn, device),
+            "hffn": bench_hffn(torch, bn, device),
+            "tiny": bench_tiny(torch, bn, device),
+        }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=("b200", "reference"), default="b200")
+    ap.add_argument("--no-extra", action="store_true", help="skip decode / FFN / tiny workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_env()
+    if args.gpus != world and not (world == 1 and args.gpus == 1):
+        if world == 1:
+            print(json.dumps({"metric": METRIC, "error": f"--gpus {args.gpus} needs torchrun "
+                              f"with {args.gpus} processes"}), flush=True)
+            return 2
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_b200(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

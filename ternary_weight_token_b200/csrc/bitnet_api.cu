@@ -1,0 +1,535 @@
+// bitnet_api.cu -- the C ABI (include/bitnet.h): host-side validation,
+// dispatch and launch of the BitLinear kernels.  The only translation unit of
+// the library: every kernel header is included here so the device error word
+// is a single symbol.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <unordered_map>
+
+#include "../../include/bitnet.h"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "pack_weights.cuh"
+#include "quant_act.cuh"
+
+namespace bitnet {
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+#define BN_CHECK_CUDA(expr)                                                              \
+  do {                                                                                   \
+    cudaError_t e_ = (expr);                                                             \
+    if (e_ != cudaSuccess) return fail(BITNET_ERR_CUDA, "%s: %s", #expr, cudaGetErrorString(e_)); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxK = 16384;
+
+int check_k(int K) {
+  if (K < 16 || K > kMaxK || K % 16 != 0)
+    return fail(BITNET_ERR_INVALID_ARG, "K=%d must be a multiple of 16 in [16, %d]", K, kMaxK);
+  return BITNET_OK;
+}
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+
+int device_info(DeviceInfo& out) {
+  static std::mutex mu;
+  static std::unordered_map<int, DeviceInfo> cache;
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    DeviceInfo di;
+    BN_CHECK_CUDA(cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev));
+    BN_CHECK_CUDA(
+        cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    it = cache.emplace(dev, di).first;
+  }
+  out = it->second;
+  return BITNET_OK;
+}
+
+// ------------------------------------------------------------ TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int get_encode_fn(EncodeTiledFn& fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess)
+      cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (cached == nullptr)
+    return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(err));
+  fn = cached;
+  return BITNET_OK;
+}
+
+struct MapKey {
+  uintptr_t ptr;
+  uint64_t d0, d1, stride;
+  uint32_t b0, b1, swz;
+  int dev;
+  bool operator==(const MapKey& o) const {
+    return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 &&
+           b1 == o.b1 && swz == o.swz && dev == o.dev;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    size_t h = std::hash<uint64_t>()(k.ptr);
+    h = h * 1000003u ^ std::hash<uint64_t>()(k.d0);
+    h = h * 1000003u ^ std::hash<uint64_t>()(k.d1);
+    h = h * 1000003u ^ std::hash<uint64_t>()(k.stride);
+    h = h * 1000003u ^ std::hash<uint64_t>()(((uint64_t)k.b0 << 32) | k.b1);
+    h = h * 1000003u ^ std::hash<uint64_t>()(((uint64_t)k.swz << 32) | (uint32_t)k.dev);
+    return h;
+  }
+};
+
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_map_cache;
+
+// 2-D byte tensor [d1 rows][d0 bytes] with row stride `stride` bytes.
+int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1, uint64_t stride,
+                     uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, stride, b0, b1, (uint32_t)swz, dev};
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    auto it = g_map_cache.find(key);
+    if (it != g_map_cache.end()) {
+      out = it->second;
+      return BITNET_OK;
+    }
+  }
+  EncodeTiledFn enc = nullptr;
+  if (int rc = get_encode_fn(enc)) return rc;
+  cuuint64_t dims[2] = {d0, d1};
+  cuuint64_t strides[1] = {stride};
+  cuuint32_t box[2] = {b0, b1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  g_map_cache[key] = out;
+  return BITNET_OK;
+}
+
+// ------------------------------------------------------------- launchers
+int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const float* gain,
+                 float eps, int8_t* Xq, float* scale, int32_t* rowsum, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  QuantParams p;
+  p.X = X; p.M = M; p.K = K; p.gain = gain; p.eps = eps;
+  p.fwht_c = (float)(1.0 / std::sqrt((double)K));
+  p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
+  const int threads = K >= 2048 ? 256 : 128;
+  const size_t smem = (size_t)K * sizeof(float);
+  const int grid = M < di.sms * 16 ? M : di.sms * 16;
+  void (*kern)(QuantParams) = nullptr;
+  switch (prelude * 2 + (bf16 ? 1 : 0)) {
+    case 0: kern = quant_act_kernel<PRE_NONE, false>; break;
+    case 1: kern = quant_act_kernel<PRE_NONE, true>; break;
+    case 2: kern = quant_act_kernel<PRE_RMSNORM, false>; break;
+    case 3: kern = quant_act_kernel<PRE_RMSNORM, true>; break;
+    case 4: kern = quant_act_kernel<PRE_FWHT, false>; break;
+    default: kern = quant_act_kernel<PRE_FWHT, true>; break;
+  }
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<grid, threads, smem, st>>>(p);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+int launch_gemv(const LinearParams& p, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int MT = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : p.M <= 8 ? 8 : 16;
+  const size_t smem = (size_t)MT * (size_t)p.ldw * 4;
+  if (smem > (size_t)di.max_smem_optin)
+    return fail(BITNET_ERR_UNSUPPORTED, "decode activations (%d x %d) exceed shared memory", p.M,
+                p.K);
+  void (*kern)(LinearParams) = nullptr;
+  switch (MT) {
+    case 1: kern = gemv_kernel<1>; break;
+    case 2: kern = gemv_kernel<2>; break;
+    case 4: kern = gemv_kernel<4>; break;
+    case 8: kern = gemv_kernel<8>; break;
+    default: kern = gemv_kernel<16>; break;
+  }
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int per_sm = 0;
+  BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem));
+  if (per_sm < 1) per_sm = 1;
+  const int rows_per_cta = (kGemvThreads / 32) * kGemvRows;
+  const int need = (p.N + rows_per_cta - 1) / rows_per_cta;
+  const int cap = di.sms * per_sm;
+  const int grid = need < cap ? need : cap;
+  kern<<<grid, kGemvThreads, smem, st>>>(p);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+template <class C>
+int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1,
+                  cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  CUtensorMap mx, mw0, mw1;
+  if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, C::BK,
+                                C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
+    return rc;
+  if (int rc = tensor_map_2d_u8(mw0, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
+                                C::BK / 4, C::BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return rc;
+  mw1 = mw0;
+  if (C::GLU) {
+    if (int rc = tensor_map_2d_u8(mw1, W1, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
+                                  C::BK / 4, C::BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return rc;
+  }
+  TcParams p;
+  p.M = lp.M; p.N = lp.N; p.K = lp.K;
+  p.num_kb = (lp.K + C::BK - 1) / C::BK;
+  p.tiles_n = (lp.N + C::BM - 1) / C::BM;
+  const int tiles_m = (lp.M + C::BN - 1) / C::BN;
+  p.num_tiles = p.tiles_n * tiles_m;
+  p.xs = lp.xs; p.xrs = lp.xrs; p.gamma0 = lp.gamma; p.gamma1 = gamma1;
+  p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type; p.flags = lp.flags;
+  // One CTA per SM: request enough shared memory that two never co-reside
+  // (each holds all 512 tensor-memory columns).
+  size_t smem = C::SMEM_ALLOC;
+  const size_t one_per_sm = (size_t)di.max_smem_optin / 2 + 1024;
+  if (smem < one_per_sm) smem = one_per_sm;
+  if (smem > (size_t)di.max_smem_optin) smem = di.max_smem_optin;
+  auto kern = gemm_tc_kernel<C>;
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
+  kern<<<grid, 384, smem, st>>>(mx, mw0, mw1, p);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+using TcPlain = TcConfig<128, 6, false>;
+using TcGlu = TcConfig<64, 4, true>;
+
+int launch_linear(const LinearParams& p, cudaStream_t st) {
+  if (p.M <= 16) return launch_gemv(p, st);
+  return launch_tc_cfg<TcPlain>(p, nullptr, nullptr, st);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int validate_linear(const int8_t* Xq, const float* xs, const int32_t* xrs, const uint8_t* W,
+                    const float* gamma, int M, int N, int K, const void* Y, int epilogue,
+                    const void* resid) {
+  if (M < 0 || N < 0) return fail(BITNET_ERR_INVALID_ARG, "M=%d, N=%d must be >= 0", M, N);
+  if (int rc = check_k(K)) return rc;
+  const int ot = epilogue & BITNET_EPI_TYPE_MASK;
+  const int flags = epilogue & ~BITNET_EPI_TYPE_MASK;
+  if (ot != BITNET_F32 && ot != BITNET_BF16 && ot != BITNET_I32)
+    return fail(BITNET_ERR_INVALID_ARG, "bad output type %d", ot);
+  if (flags & ~(BITNET_EPI_RESIDUAL | BITNET_EPI_SILU))
+    return fail(BITNET_ERR_INVALID_ARG, "unknown epilogue flags 0x%x", flags);
+  if (ot == BITNET_I32 && flags)
+    return fail(BITNET_ERR_UNSUPPORTED, "the int32 output takes no residual or SiLU");
+  if ((flags & BITNET_EPI_RESIDUAL) && resid == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "residual flag set but residual is NULL");
+  if (!(flags & BITNET_EPI_RESIDUAL) && resid != nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "residual given without BITNET_EPI_RESIDUAL");
+  if (M == 0 || N == 0) return BITNET_OK;
+  if (!Xq || !xs || !xrs || !W || !gamma || !Y)
+    return fail(BITNET_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(Xq) || !aligned16(xs) || !aligned16(xrs) || !aligned16(W) || !aligned16(gamma) ||
+      !aligned16(Y) || (resid && !aligned16(resid)))
+    return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  return BITNET_OK;
+}
+
+}  // namespace
+}  // namespace bitnet
+
+using namespace bitnet;
+
+extern "C" {
+
+size_t bitnet_packed_row_bytes(int K) {
+  if (K <= 0) return 0;
+  return (size_t)16 * (size_t)((K + 63) / 64);
+}
+
+size_t bitnet_pack_workspace_size(int N, int K) {
+  (void)N;
+  (void)K;
+  return (size_t)kPackPartialBlocks * sizeof(double);
+}
+
+int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packed, float* gamma,
+                        void* workspace, size_t ws_bytes, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (N < 0) return fail(BITNET_ERR_INVALID_ARG, "N=%d must be >= 0", N);
+  if (int rc = check_k(K)) return rc;
+  if (w_dtype != BITNET_F32 && w_dtype != BITNET_BF16)
+    return fail(BITNET_ERR_INVALID_ARG, "weight dtype must be F32 or BF16");
+  if (!W || !packed || !gamma) return fail(BITNET_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma))
+    return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (workspace == nullptr || ws_bytes < bitnet_pack_workspace_size(N, K))
+    return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes needed",
+                bitnet_pack_workspace_size(N, K));
+  if (!aligned16(workspace)) return fail(BITNET_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool bf16 = w_dtype == BITNET_BF16;
+  const long long count = (long long)N * K;
+  double* partials = reinterpret_cast<double*>(workspace);
+  if (bf16)
+    absmean_partial_kernel<true><<<kPackPartialBlocks, kPackThreads, 0, st>>>(W, count, partials);
+  else
+    absmean_partial_kernel<false><<<kPackPartialBlocks, kPackThreads, 0, st>>>(W, count, partials);
+  BN_CHECK_CUDA(cudaGetLastError());
+  absmean_final_kernel<<<1, kPackThreads, 0, st>>>(partials, kPackPartialBlocks, count, gamma);
+  BN_CHECK_CUDA(cudaGetLastError());
+  if (N == 0) return BITNET_OK;
+  const int ldw = (int)bitnet_packed_row_bytes(K);
+  const long long words = (long long)N * (ldw / 4);
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  long long blocks = (words + kPackThreads - 1) / kPackThreads;
+  if (blocks > (long long)di.sms * 32) blocks = (long long)di.sms * 32;
+  if (bf16)
+    pack_kernel<true><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
+  else
+    pack_kernel<false><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+int bitnet_quant_act(const void* X, int x_dtype, int M, int K, int prelude,
+                     const float* norm_gain, float eps, int8_t* Xq, float* x_scale,
+                     int32_t* x_rowsum, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (M < 0) return fail(BITNET_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (int rc = check_k(K)) return rc;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16)
+    return fail(BITNET_ERR_INVALID_ARG, "activation dtype must be F32 or BF16");
+  if (prelude != BITNET_PRELUDE_NONE && prelude != BITNET_PRELUDE_RMSNORM &&
+      prelude != BITNET_PRELUDE_FWHT)
+    return fail(BITNET_ERR_INVALID_ARG, "unknown prelude %d", prelude);
+  if (prelude == BITNET_PRELUDE_FWHT && (K & (K - 1)) != 0)
+    return fail(BITNET_ERR_INVALID_ARG, "FWHT width K=%d is not a power of two", K);
+  if (norm_gain != nullptr && prelude != BITNET_PRELUDE_RMSNORM)
+    return fail(BITNET_ERR_INVALID_ARG, "norm_gain is only used by the RMSNorm prelude");
+  if (prelude == BITNET_PRELUDE_RMSNORM && !(eps >= 0.0f && std::isfinite(eps)))
+    return fail(BITNET_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (M == 0) return BITNET_OK;
+  if (!X || !Xq || !x_scale) return fail(BITNET_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(X) || !aligned16(Xq) || !aligned16(x_scale) ||
+      (x_rowsum && !aligned16(x_rowsum)) || (norm_gain && !aligned16(norm_gain)))
+    return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  return launch_quant(X, x_dtype == BITNET_BF16, M, K, prelude, norm_gain, eps, Xq, x_scale,
+                      x_rowsum, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsum,
+                  const uint8_t* packed, const float* gamma, int M, int N, int K, void* Y,
+                  int epilogue, const void* residual, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (int rc = validate_linear(Xq, x_scale, x_rowsum, packed, gamma, M, N, K, Y, epilogue,
+                               residual))
+    return rc;
+  if (M == 0 || N == 0) return BITNET_OK;
+  LinearParams p;
+  p.Xq = Xq; p.xs = x_scale; p.xrs = x_rowsum; p.W = packed; p.gamma = gamma;
+  p.M = M; p.N = N; p.K = K; p.ldw = (int)bitnet_packed_row_bytes(K);
+  p.Y = Y; p.out_type = epilogue & BITNET_EPI_TYPE_MASK;
+  p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = residual;
+  return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant) {
+  if (M < 0 || H <= 0 || I <= 0) return 0;
+  const size_t m = (size_t)M;
+  size_t total = 0;
+  total += align256(m * (size_t)H);            // codes of x
+  total += align256(m * 4) * 2;                // scale and rowsum of x
+  total += align256(m * (size_t)I * 4);        // fp32 hidden activation
+  total += align256(m * (size_t)I);            // codes of the hidden activation
+  total += align256(m * 4) * 2;                // its scale and rowsum
+  (void)variant;
+  return total;
+}
+
+int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W_gate,
+               const float* gamma_gate, const uint8_t* W_up, const float* gamma_up,
+               const uint8_t* W_down, const float* gamma_down, const float* pre_norm_gain,
+               const float* sub_norm_gain, float eps, int variant, void* Y, int y_dtype,
+               void* workspace, size_t ws_bytes, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (M < 0) return fail(BITNET_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (int rc = check_k(H)) return rc;
+  if (int rc = check_k(I)) return rc;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16)
+    return fail(BITNET_ERR_INVALID_ARG, "x dtype must be F32 or BF16");
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16)
+    return fail(BITNET_ERR_INVALID_ARG, "y dtype must be F32 or BF16");
+  if (variant != BITNET_FFN_RELU2_GLU && variant != BITNET_FFN_HADAMARD_SILU)
+    return fail(BITNET_ERR_INVALID_ARG, "unknown FFN variant %d", variant);
+  if (variant == BITNET_FFN_RELU2_GLU) {
+    if (x_dtype != y_dtype)
+      return fail(BITNET_ERR_UNSUPPORTED, "the residual FFN needs x and y of one dtype");
+    if (!W_up || !gamma_up) return fail(BITNET_ERR_INVALID_ARG, "W_up / gamma_up missing");
+    if (!(eps >= 0.0f && std::isfinite(eps)))
+      return fail(BITNET_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  } else {
+    if (W_up || gamma_up)
+      return fail(BITNET_ERR_INVALID_ARG, "the Hadamard FFN has no up projection");
+    if ((H & (H - 1)) || (I & (I - 1)))
+      return fail(BITNET_ERR_INVALID_ARG, "H-BitLinear widths must be powers of two");
+    if (pre_norm_gain || sub_norm_gain)
+      return fail(BITNET_ERR_INVALID_ARG, "the Hadamard FFN takes no norm gains");
+  }
+  if (M == 0) return BITNET_OK;
+  if (!X || !W_gate || !gamma_gate || !W_down || !gamma_down || !Y)
+    return fail(BITNET_ERR_INVALID_ARG, "null pointer argument");
+  if (!aligned16(X) || !aligned16(Y) || !aligned16(W_gate) || !aligned16(W_down) ||
+      !aligned16(gamma_gate) || !aligned16(gamma_down) || (W_up && !aligned16(W_up)) ||
+      (gamma_up && !aligned16(gamma_up)) || (pre_norm_gain && !aligned16(pre_norm_gain)) ||
+      (sub_norm_gain && !aligned16(sub_norm_gain)))
+    return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t need = bitnet_ffn_workspace_size(M, H, I, variant);
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
+  if (!aligned16(workspace)) return fail(BITNET_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t m = (size_t)M;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  int8_t* xq = reinterpret_cast<int8_t*>(ws);            ws += align256(m * H);
+  float* xs = reinterpret_cast<float*>(ws);              ws += align256(m * 4);
+  int32_t* xrs = reinterpret_cast<int32_t*>(ws);         ws += align256(m * 4);
+  float* hid = reinterpret_cast<float*>(ws);             ws += align256(m * I * 4);
+  int8_t* hq = reinterpret_cast<int8_t*>(ws);            ws += align256(m * I);
+  float* hs = reinterpret_cast<float*>(ws);              ws += align256(m * 4);
+  int32_t* hrs = reinterpret_cast<int32_t*>(ws);
+  const bool xbf = x_dtype == BITNET_BF16;
+
+  LinearParams p1;
+  p1.Xq = xq; p1.xs = xs; p1.xrs = xrs; p1.W = W_gate; p1.gamma = gamma_gate;
+  p1.M = M; p1.N = I; p1.K = H; p1.ldw = (int)bitnet_packed_row_bytes(H);
+  p1.Y = hid; p1.out_type = OUT_F32; p1.resid = nullptr;
+  LinearParams p2;
+  p2.Xq = hq; p2.xs = hs; p2.xrs = hrs; p2.W = W_down; p2.gamma = gamma_down;
+  p2.M = M; p2.N = H; p2.K = I; p2.ldw = (int)bitnet_packed_row_bytes(I);
+  p2.Y = Y; p2.out_type = y_dtype == BITNET_BF16 ? OUT_BF16 : OUT_F32;
+
+  if (variant == BITNET_FFN_RELU2_GLU) {
+    if (int rc = launch_quant(X, xbf, M, H, PRE_RMSNORM, pre_norm_gain, eps, xq, xs, xrs, st))
+      return rc;
+    p1.flags = 0;
+    if (int rc = launch_tc_cfg<TcGlu>(p1, W_up, gamma_up, st)) return rc;
+    if (int rc = launch_quant(hid, false, M, I, PRE_RMSNORM, sub_norm_gain, eps, hq, hs, hrs, st))
+      return rc;
+    p2.flags = EPI_RESIDUAL;
+    p2.resid = X;
+    return launch_linear(p2, st);
+  }
+  if (int rc = launch_quant(X, xbf, M, H, PRE_FWHT, nullptr, 0.0f, xq, xs, xrs, st)) return rc;
+  p1.flags = EPI_SILU;
+  if (int rc = launch_linear(p1, st)) return rc;
+  if (int rc = launch_quant(hid, false, M, I, PRE_FWHT, nullptr, 0.0f, hq, hs, hrs, st)) return rc;
+  p2.flags = 0;
+  p2.resid = nullptr;
+  return launch_linear(p2, st);
+}
+
+const char* bitnet_last_error(void) { return g_last_error.c_str(); }
+
+int bitnet_check_device_error(bitnet_stream_t stream) {
+  g_last_error.clear();
+  BN_CHECK_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+  unsigned int word = 0, zero = 0;
+  BN_CHECK_CUDA(cudaMemcpyFromSymbol(&word, g_device_error, sizeof(word)));
+  if (word != 0) {
+    BN_CHECK_CUDA(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)));
+    if (word & DEV_ERR_TIMEOUT)
+      return fail(BITNET_ERR_TIMEOUT, "a bounded device-side wait gave up (error word 0x%x)", word);
+    return fail(BITNET_ERR_CUDA, "device error word 0x%x", word);
+  }
+  return BITNET_OK;
+}
+
+void bitnet_release_cache(void) {
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  g_map_cache.clear();
+}
+
+const char* bitnet_version(void) { return "bitnet-b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"
+
+// The timeout diagnostic lives below the C ABI block so it can use the
+// kernel-side wait helper directly.
+namespace bitnet {
+__device__ int g_wait_probe_result = 0;
+
+__global__ void wait_timeout_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Nobody ever arrives on `bar`: the bounded wait must give up.
+  const bool done = mbar_wait(&bar, 0, &abort_flag, limit_ns);
+  if (threadIdx.x == 0) g_wait_probe_result = done ? 1 : 0;
+}
+}  // namespace bitnet
+
+extern "C" int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (timeout_us < 1 || timeout_us > 1000000)
+    return fail(BITNET_ERR_INVALID_ARG, "timeout_us must be in [1, 1000000]");
+  wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (unsigned long long)timeout_us * 1000ull);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}

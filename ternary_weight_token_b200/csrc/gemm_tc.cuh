@@ -1,0 +1,301 @@
+// gemm_tc.cuh -- prefill BitLinear on the sm_100a tensor cores
+// (tcgen05.mma kind::i8, int32 accumulators in tensor memory).
+//
+// nnterp encyclopedia "bitnet", "The projections quantize their inputs and
+// weights": the output equals the linear map of the rounded (int8) input by
+// the ternarised weight exactly, dequantised by weight_scale / input scale.
+// "The MLP gates with a squared ReLU" and "The block, in order" give the fused
+// gate/up epilogue relu(g)^2 * u and the residual add; "bitnetv2-model"
+// README, "Architecture Overview", the SiLU epilogue.
+//
+// Shape of the computation: D^T[n][m] = sum_k c[n][k] * q[m][k], where c = t + 1
+// are the stored (unsigned) weight codes and q the signed activation codes;
+// the epilogue subtracts sum_k q[m][k] to get the contraction with t.
+//
+//   A operand (M = 128 weight rows)  : tensor memory.  The packed 2-bit tile is
+//       TMA-loaded into shared memory; converter warps expand each 32-bit word
+//       of 16 codes into four words of byte codes (shift + mask) and write them
+//       to tensor memory with tcgen05.st, one thread per row (TMEM lane).
+//   B operand (N = BN tokens)        : shared memory, TMA-loaded int8 rows in the
+//       128-byte swizzled K-major layout the MMA descriptor reads.
+//   D (int32, 128 lanes x BN columns): tensor memory, double-buffered so the
+//       epilogue of one tile overlaps the MMAs of the next.
+//
+// Warp roles (384 threads, one persistent CTA per SM):
+//   warp 0      TMA producer (one thread)
+//   warp 1      MMA issuer (one thread)
+//   warp 2      tensor-memory allocator
+//   warps 4-7   converters (2-bit codes -> byte codes in TMEM)
+//   warps 8-11  epilogue (tcgen05.ld -> dequant -> fused op -> global stores)
+// Every wait is bounded; a wait that gives up records a device error, raises a
+// CTA-wide abort flag, and the CTA drains its tensor-core work, frees tensor
+// memory and exits.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace bitnet {
+
+template <int BN_, int STAGES_, bool GLU_>
+struct TcConfig {
+  static constexpr int BN = BN_;            // tokens per tile (MMA N)
+  static constexpr int STAGES = STAGES_;
+  static constexpr bool GLU = GLU_;         // gate and up weights in one pass
+  static constexpr int BM = 128;            // weight rows per tile (MMA M, TMEM lanes)
+  static constexpr int BK = 128;            // k per pipeline stage
+  static constexpr int NW = GLU ? 2 : 1;    // weight matrices per stage
+  static constexpr int X_STAGE = BN * BK;   // bytes of activation codes per stage
+  static constexpr int W_STAGE = BM * BK / 4;  // bytes of packed weights per matrix per stage
+  static constexpr int ACC_COLS = BN * NW;  // TMEM columns per accumulator buffer
+  static constexpr int A_COLS = (BK / 4) * NW;  // TMEM columns per A slot
+  static constexpr int TMEM_COLS = 512;
+  static_assert(2 * ACC_COLS + STAGES * A_COLS <= TMEM_COLS, "tensor memory overflow");
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static constexpr int OFF_X = 0;
+  static constexpr int OFF_W = OFF_X + STAGES * X_STAGE;
+  static constexpr int OFF_BAR = OFF_W + STAGES * NW * W_STAGE;
+  static constexpr int NUM_BARS = 3 * STAGES + 5;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TOK = (OFF_MISC + 16 + 15) / 16 * 16;
+  static constexpr int TOK_BYTES_PER_WARP = BN * (8 * NW + 4);
+  static constexpr int SMEM_BYTES = OFF_TOK + 4 * TOK_BYTES_PER_WARP;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
+  static constexpr uint32_t TX_BYTES = X_STAGE + NW * W_STAGE;
+};
+
+struct TcParams {
+  int M, N, K;
+  int num_kb;                 // k stages = ceil(K / 128)
+  int tiles_n, num_tiles;
+  const float* xs;            // [M] activation scales
+  const int32_t* xrs;         // [M] sum of activation codes
+  const float* gamma0;        // weight scale (gate weights for GLU)
+  const float* gamma1;        // up weight scale (GLU only)
+  void* Y;                    // [M][N]
+  const void* resid;          // [M][N] or null
+  int out_type;
+  int flags;
+};
+
+template <class C>
+__global__ void __launch_bounds__(384, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_w0,
+                   const __grid_constant__ CUtensorMap tm_w1, TcParams p) {
+  extern __shared__ uint8_t tc_smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sx = smem + C::OFF_X;
+  uint8_t* sw = smem + C::OFF_W;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* full = bars;                       // TMA bytes landed       (count 1 + tx)
+  uint64_t* empty = bars + C::STAGES;          // MMAs done with stage   (tcgen05.commit)
+  uint64_t* afull = bars + 2 * C::STAGES;      // A codes in TMEM        (4 converter warps)
+  uint64_t* accfull = bars + 3 * C::STAGES;    // accumulator ready      (tcgen05.commit)
+  uint64_t* accempty = accfull + 2;            // accumulator drained    (4 epilogue warps)
+  uint64_t* drain = accempty + 2;              // teardown drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&afull[s], 4);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(&tm_w0);
+    if (C::GLU) tma_prefetch_desc(&tm_w1);
+  }
+  if (warp == 2) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_slot;
+  const uint32_t a_col0 = 2 * C::ACC_COLS;
+
+  if (warp == 0) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t it = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) goto producer_done;
+          mbar_arrive_expect_tx(&full[st], C::TX_BYTES);
+          tma_load_2d(sx + st * C::X_STAGE, &tm_x, &full[st], kb * C::BK, tm * C::BN);
+          tma_load_2d(sw + (st * C::NW) * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
+                      tn * C::BM);
+          if (C::GLU)
+            tma_load_2d(sw + (st * C::NW + 1) * C::W_STAGE, &tm_w1, &full[st], kb * (C::BK / 4),
+                        tn * C::BM);
+        }
+      }
+    producer_done:
+      // Never leave bulk copies in flight: wait for the last issued stages.
+      const uint32_t last = it < (uint32_t)C::STAGES ? it : (uint32_t)C::STAGES;
+      for (uint32_t i = 0; i < last; ++i) {
+        const uint32_t j = it - 1 - i;
+        mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, 100000000ull);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc_i8(C::BM, C::BN);
+      uint32_t it = 0, tcount = 0;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+        const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
+        if (!mbar_wait(&accempty[ab], aph ^ 1u, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_col = tbase + ab * C::ACC_COLS;
+        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+          if (!mbar_wait(&full[st], ph, abort_flag)) goto mma_done;
+          if (!mbar_wait(&afull[st], ph, abort_flag)) goto mma_done;
+          tc_fence_after();
+          const uint32_t a_col = tbase + a_col0 + st * C::A_COLS;
+          const uint32_t xaddr = smem_u32(sx + st * C::X_STAGE);
+#pragma unroll
+          for (int j = 0; j < C::BK / 32; ++j) {
+            const uint64_t bdesc = make_sdesc_sw128(xaddr + 32u * j);
+            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
+            mma_i8_ts(d_col, a_col + 8u * j, bdesc, idesc, acc);
+            if (C::GLU) mma_i8_ts(d_col + C::BN, a_col + 32u + 8u * j, bdesc, idesc, acc);
+          }
+          tc_commit(&empty[st]);
+        }
+        tc_commit(&accfull[ab]);
+      }
+    mma_done:
+      tc_commit(drain);
+      mbar_wait(drain, 0, nullptr, 100000000ull);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------- converters
+    const int q = warp & 3;
+    const int row = 32 * q + lane;               // weight row within the tile = TMEM lane
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16) + a_col0;
+    uint32_t it = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+        if (!mbar_wait(&full[st], ph, abort_flag)) goto convert_done;
+        tc_fence_after();
+#pragma unroll
+        for (int w = 0; w < C::NW; ++w) {
+          const uint4* src = reinterpret_cast<const uint4*>(sw + (st * C::NW + w) * C::W_STAGE +
+                                                            row * (C::BK / 4));
+          const uint4 a = src[0], b = src[1];
+          uint32_t e[32];
+          expand_codes(a.x, e[0], e[1], e[2], e[3]);
+          expand_codes(a.y, e[4], e[5], e[6], e[7]);
+          expand_codes(a.z, e[8], e[9], e[10], e[11]);
+          expand_codes(a.w, e[12], e[13], e[14], e[15]);
+          expand_codes(b.x, e[16], e[17], e[18], e[19]);
+          expand_codes(b.y, e[20], e[21], e[22], e[23]);
+          expand_codes(b.z, e[24], e[25], e[26], e[27]);
+          expand_codes(b.w, e[28], e[29], e[30], e[31]);
+          tmem_st_32x32b_x32(lane_base + st * C::A_COLS + 32u * w, e);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[st]);
+      }
+    }
+  convert_done:;
+  } else if (warp >= 8) {
+    // --------------------------------------------------------- epilogue
+    const int q = warp & 3;
+    double* tok_f0 = reinterpret_cast<double*>(smem + C::OFF_TOK + q * C::TOK_BYTES_PER_WARP);
+    double* tok_f1 = tok_f0 + C::BN;             // GLU only
+    int* tok_rs = reinterpret_cast<int*>(tok_f0 + C::NW * C::BN);
+    const double g0 = (double)__ldg(p.gamma0);
+    const double g1 = C::GLU ? (double)__ldg(p.gamma1) : 0.0;
+    const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
+      const int m0 = tm * C::BN;
+      const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
+      __syncwarp();
+      for (int j = lane; j < C::BN; j += 32) {
+        const int m = m0 + j;
+        double f0 = 0.0, f1 = 0.0;
+        int rs = 0;
+        if (m < p.M) {
+          const double s = (double)p.xs[m];
+          f0 = g0 / s;
+          if (C::GLU) f1 = g1 / s;
+          rs = p.xrs[m];
+        }
+        tok_f0[j] = f0;
+        if (C::GLU) tok_f1[j] = f1;
+        tok_rs[j] = rs;
+      }
+      __syncwarp();
+      if (!mbar_wait(&accfull[ab], aph, abort_flag)) break;
+      tc_fence_after();
+      const int n = tn * C::BM + 32 * q + lane;
+      const bool n_ok = n < p.N;
+#pragma unroll 1
+      for (int c = 0; c < C::BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, v);
+        if (C::GLU) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = 32 * c + j, m = m0 + t;
+            if (n_ok && m < p.M) {
+              const int rs = tok_rs[t];
+              const float g = (float)((double)((int)v[j] - rs) * tok_f0[t]);
+              const float uu = (float)((double)((int)u[j] - rs) * tok_f1[t]);
+              const float a = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
+              reinterpret_cast<float*>(p.Y)[(size_t)m * p.N + n] = __fmul_rn(a, uu);
+            }
+          }
+        } else {
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int t = 32 * c + j, m = m0 + t;
+            if (n_ok && m < p.M)
+              store_output(p.Y, p.resid, (size_t)m * p.N + n, (int)v[j] - tok_rs[t], tok_f0[t],
+                           p.out_type, p.flags);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accempty[ab]);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 2) tmem_dealloc(tbase, C::TMEM_COLS);
+}
+
+}  // namespace bitnet

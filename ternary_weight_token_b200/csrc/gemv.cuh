@@ -1,0 +1,153 @@
+// gemv.cuh -- decode BitLinear (M <= 16 tokens): int8 activations x packed
+// ternary weights -> int32 -> dequantised output.
+//
+// nnterp encyclopedia "bitnet", "The projections quantize their inputs and
+// weights": the projection output equals the linear map of the rounded input
+// by the ternarised weight exactly; "BitNet b1.58 2B4T", "How to Use": the
+// efficiency needs specialised kernels.
+//
+// HBM-bound on the packed weights (0.25 byte per weight).  Persistent CTAs
+// stage the M activation rows once in shared memory; each warp then streams
+// R weight rows at a time with 128-bit non-allocating loads, expands every
+// 32-bit word of 16 codes into four words of byte codes with two ALU ops each,
+// and multiplies them against the activation bytes with dp4a (unsigned codes
+// c = t + 1 times signed activations).  The sum over k of q * c minus the
+// token's sum of q is the exact int32 contraction with t.
+#pragma once
+
+#include "common.cuh"
+
+namespace bitnet {
+
+enum { OUT_F32 = 0, OUT_BF16 = 1, OUT_I32 = 2 };
+enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20 };
+
+struct LinearParams {
+  const int8_t* Xq;
+  const float* xs;
+  const int32_t* xrs;
+  const uint8_t* W;
+  const float* gamma;
+  int M, N, K, ldw;
+  void* Y;
+  int out_type;
+  int flags;
+  const void* resid;
+};
+
+// Shared epilogue: int32 contraction -> stored output element.
+__device__ __forceinline__ void store_output(void* Y, const void* resid, size_t idx, int yint,
+                                             double f, int out_type, int flags) {
+  if (out_type == OUT_I32) {
+    reinterpret_cast<int32_t*>(Y)[idx] = yint;
+    return;
+  }
+  float y = (float)((double)yint * f);
+  if (flags & EPI_SILU) {
+    const double d = (double)y;
+    y = (float)(d / (1.0 + exp(-d)));
+  }
+  if (out_type == OUT_BF16) {
+    if (flags & EPI_RESIDUAL) {
+      const float r = __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(resid)[idx]);
+      y = __fadd_rn(r, y);
+    }
+    reinterpret_cast<__nv_bfloat16*>(Y)[idx] = __float2bfloat16_rn(y);
+  } else {
+    if (flags & EPI_RESIDUAL) y = __fadd_rn(reinterpret_cast<const float*>(resid)[idx], y);
+    reinterpret_cast<float*>(Y)[idx] = y;
+  }
+}
+
+constexpr int kGemvThreads = 256;
+constexpr int kGemvRows = 2;   // weight rows per warp task
+
+template <int MT>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
+  extern __shared__ uint4 gemv_smem[];          // [MT][ldw / 4] activation codes (16 B units)
+  __shared__ double tok_f[MT];
+  __shared__ int tok_rs[MT];
+
+  const int chunks = p.ldw / 16;                // 16-byte packed chunks (64 weights) per row
+  const int qv = chunks * 4;                    // 16-byte activation units per row
+  for (int i = threadIdx.x; i < MT * qv; i += blockDim.x) {
+    const int m = i / qv, c = i % qv, k0 = 16 * c;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (m < p.M && k0 < p.K) v = *reinterpret_cast<const uint4*>(p.Xq + (size_t)m * p.K + k0);
+    gemv_smem[i] = v;
+  }
+  if (threadIdx.x < MT) {
+    const int m = threadIdx.x;
+    if (m < p.M) {
+      tok_f[m] = (double)__ldg(p.gamma) / (double)p.xs[m];
+      tok_rs[m] = p.xrs[m];
+    } else {
+      tok_f[m] = 0.0;
+      tok_rs[m] = 0;
+    }
+  }
+  __syncthreads();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = blockDim.x >> 5;
+  for (int n0 = (blockIdx.x * nwarps + warp) * kGemvRows; n0 < p.N;
+       n0 += gridDim.x * nwarps * kGemvRows) {
+    int acc[kGemvRows][MT];
+#pragma unroll
+    for (int r = 0; r < kGemvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+
+#pragma unroll
+    for (int r = 0; r < kGemvRows; ++r) {
+      const int n = n0 + r;
+      if (n < p.N) {
+        const uint8_t* wrow = p.W + (size_t)n * p.ldw;
+        for (int c = lane; c < chunks; c += 32) {
+          const uint4 w = ld_stream_v4(wrow + 16 * c);
+          uint32_t e[16];
+          expand_codes(w.x, e[0], e[1], e[2], e[3]);
+          expand_codes(w.y, e[4], e[5], e[6], e[7]);
+          expand_codes(w.z, e[8], e[9], e[10], e[11]);
+          expand_codes(w.w, e[12], e[13], e[14], e[15]);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const uint4* qp = gemv_smem + m * qv + 4 * c;
+            const uint4 q0 = qp[0], q1 = qp[1], q2 = qp[2], q3 = qp[3];
+            int a = acc[r][m];
+            a = dp4a_us(e[0], q0.x, a);  a = dp4a_us(e[1], q0.y, a);
+            a = dp4a_us(e[2], q0.z, a);  a = dp4a_us(e[3], q0.w, a);
+            a = dp4a_us(e[4], q1.x, a);  a = dp4a_us(e[5], q1.y, a);
+            a = dp4a_us(e[6], q1.z, a);  a = dp4a_us(e[7], q1.w, a);
+            a = dp4a_us(e[8], q2.x, a);  a = dp4a_us(e[9], q2.y, a);
+            a = dp4a_us(e[10], q2.z, a); a = dp4a_us(e[11], q2.w, a);
+            a = dp4a_us(e[12], q3.x, a); a = dp4a_us(e[13], q3.y, a);
+            a = dp4a_us(e[14], q3.z, a); a = dp4a_us(e[15], q3.w, a);
+            acc[r][m] = a;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kGemvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        int v = acc[r][m];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        acc[r][m] = v;
+      }
+#pragma unroll
+    for (int r = 0; r < kGemvRows; ++r)
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int n = n0 + r;
+        if (lane == ((r * MT + m) & 31) && m < p.M && n < p.N) {
+          const size_t idx = (size_t)m * p.N + n;
+          store_output(p.Y, p.resid, idx, acc[r][m] - tok_rs[m], tok_f[m], p.out_type, p.flags);
+        }
+      }
+  }
+}
+
+}  // namespace bitnet

@@ -1,0 +1,132 @@
+"""GPU parity of the BitLinear contraction and its epilogues (decode GEMV for
+M <= 16, tcgen05 GEMM above) against the oracle, through the C ABI.
+
+Each kernel gets the oracle's own codes, scales and packed weights, so the
+int32 contraction must match bit for bit; fp32 outputs must be within 1e-5
+relative (the dequantisation is fp64 on both sides, so they are equal except
+next to an fp32 midpoint); bf16 outputs must be the nearest-even rounding of
+the oracle's fp32 value.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import ternary_weight_token_b200 as bn
+from tests.gpu_util import assert_bf16_matches, assert_f32_close, dev, gpu_linear
+
+pytestmark = pytest.mark.gpu
+
+
+def _case(M, K, N, seed, prelude=oracle.PRELUDE_NONE):
+    rng_w, rng_x = synthetic.streams(seed, 2)
+    W = synthetic.weight(rng_w, N, K)
+    X = synthetic.activations(rng_x, M, K)
+    g, T, P = oracle.quantize_weights(W)
+    q, s, rs = oracle.quant_act(X, prelude)
+    return X, g, T, P, q, s, rs
+
+
+SHAPES = [
+    # decode GEMV
+    (1, 16, 1), (1, 2560, 2560), (2, 80, 33), (3, 256, 512), (4, 2560, 640), (8, 256, 512),
+    (15, 6912, 100), (16, 2560, 257),
+    # tensor-core GEMM: several tiles and ragged tails in M (tokens) and N (weights)
+    (17, 256, 128), (64, 80, 129), (127, 2560, 300), (129, 512, 128), (300, 2560, 300),
+    (256, 6912, 256), (513, 1024, 1000),
+]
+
+
+@pytest.mark.parametrize("M,K,N", SHAPES)
+def test_linear_int32_bit_exact(M, K, N):
+    X, g, T, P, q, s, rs = _case(M, K, N, seed=M * 1000 + N)
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.int32)
+    np.testing.assert_array_equal(got, oracle.contract(q, T))
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 2560, 2560), (16, 6912, 300), (300, 2560, 300),
+                                   (200, 512, 2048)])
+def test_linear_f32_and_bf16(M, K, N):
+    X, g, T, P, q, s, rs = _case(M, K, N, seed=M + N)
+    want = oracle.dequant(oracle.contract(q, T), s, g)
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.float32)
+    assert_f32_close(got, want, what="f32 out")
+    assert np.all(got[want == 0] == 0)
+    gotb = gpu_linear(q, s, rs, P, g, K, N, out=torch.bfloat16)
+    assert_bf16_matches(gotb, want, what="bf16 out")
+
+
+@pytest.mark.parametrize("M", [4, 160])
+def test_linear_residual_and_silu(M):
+    K, N = 512, 384
+    X, g, T, P, q, s, rs = _case(M, K, N, seed=77 + M)
+    y = oracle.dequant(oracle.contract(q, T), s, g)
+    R = synthetic.activations(np.random.default_rng(5), M, N)
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.float32, flags=bn.BITNET_EPI_RESIDUAL,
+                     residual=R)
+    assert_f32_close(got, (R + y).astype(np.float32), what="residual")
+    Rb = oracle.round_bf16(R)
+    gotb = gpu_linear(q, s, rs, P, g, K, N, out=torch.bfloat16, flags=bn.BITNET_EPI_RESIDUAL,
+                      residual=dev(Rb).to(torch.bfloat16))
+    assert_bf16_matches(gotb, (Rb + y).astype(np.float32), what="bf16 residual")
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.float32, flags=bn.BITNET_EPI_SILU)
+    assert_f32_close(got, oracle.silu(y), what="silu")
+
+
+def test_linear_extreme_codes():
+    """All +127 / -128 codes against all +1 / -1 weights at K = 16384: the int32
+    accumulator holds 128 * 16384 with no overflow."""
+    K, N = 16384, 130
+    q = np.full((20, K), 127, np.int8)
+    q[1::2] = -128
+    T = np.ones((N, K), np.int8)
+    T[1::2] = -1
+    P = oracle.pack(T)
+    s = np.ones(20, np.float32)
+    rs = q.astype(np.int64).sum(axis=1).astype(np.int32)
+    for M in (3, 20):
+        got = gpu_linear(q[:M], s[:M], rs[:M], P, np.float32(1.0), K, N, out=torch.int32)
+        np.testing.assert_array_equal(got, oracle.contract(q[:M], T))
+
+
+def test_linear_zero_rows_and_zero_gamma():
+    K, N = 256, 200
+    X, g, T, P, q, s, rs = _case(40, K, N, seed=3)
+    q[5] = 0
+    s[5] = 1.0
+    rs[5] = 0
+    got = gpu_linear(q, s, rs, P, g, K, N)
+    assert np.all(got[5] == 0)
+    Z = np.full_like(P, 0x55)          # every weight 0
+    got = gpu_linear(q, s, rs, Z, np.float32(0.0), K, N)
+    assert np.all(got == 0)
+
+
+def test_linear_empty_is_noop():
+    Y = torch.full((0, 8), 7.0, device="cuda")
+    q = torch.empty((0, 32), dtype=torch.int8, device="cuda")
+    s = torch.empty(0, device="cuda")
+    rs = torch.empty(0, dtype=torch.int32, device="cuda")
+    P = torch.empty((8, 16), dtype=torch.uint8, device="cuda")
+    g = torch.ones(1, device="cuda")
+    bn.bitnet_linear(q, s, rs, P, g, 32, Y)
+    torch.cuda.synchronize()
+
+
+def test_full_chain_matches_oracle():
+    """pack -> quant -> linear all on the device against the oracle's chain."""
+    M, K, N = 96, 2560, 640
+    rng_w, rng_x = synthetic.streams(31, 2)
+    W = synthetic.weight(rng_w, N, K)
+    X = synthetic.activations(rng_x, M, K)
+    Wd, Xd = dev(W), dev(X)
+    packed, gamma, ws = bn.alloc_packed(N, K)
+    bn.bitnet_pack_weights(Wd, packed, gamma, ws)
+    q, s, rs = bn.alloc_quant(M, K)
+    bn.bitnet_quant_act(Xd, q, s, rs)
+    Y = torch.empty((M, N), device="cuda")
+    bn.bitnet_linear(q, s, rs, packed, gamma, K, Y)
+    torch.cuda.synchronize()
+    g, T, _ = oracle.quantize_weights(W)
+    assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="chain")

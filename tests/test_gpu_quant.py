@@ -1,0 +1,133 @@
+"""GPU parity of the activation quantiser (with its preludes) and of the
+weight packer against the oracle, through the C ABI.
+
+Codes, scales and code sums are compared bit for bit.  The RMSNorm prelude
+accumulates the mean square in fp64 on both sides but in a different order;
+the fp32 value it rounds to can then differ only next to an fp32 midpoint, so
+those cases fall under the chain tolerance (<= 0.1 % of codes, +-1 each).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synthetic
+import ternary_weight_token_b200 as bn
+from tests.gpu_util import (assert_codes_chain, bf16_dev, code_mismatch_stats, dev, gpu_pack,
+                            gpu_quant)
+
+pytestmark = pytest.mark.gpu
+
+
+def _acts(M, K, seed, outliers=False):
+    X = synthetic.activations(np.random.default_rng(seed), M, K)
+    if outliers:
+        X = synthetic.outliers(np.random.default_rng(seed + 1), X)
+    return X
+
+
+@pytest.mark.parametrize("M,K", [(1, 16), (8, 256), (3, 80), (129, 2560), (37, 6912), (2, 16384)])
+def test_quant_none_bit_exact(M, K):
+    X = _acts(M, K, seed=M * 7 + K)
+    X[0, :] = 0.0                       # an all-zero token
+    if M > 2:
+        X[2, :] = 0.0
+        X[2, K // 3] = -5.5              # a one-hot token
+    q, s, rs = gpu_quant(X)
+    qo, so, rso = oracle.quant_act(X)
+    np.testing.assert_array_equal(q, qo)
+    np.testing.assert_array_equal(s, so)
+    np.testing.assert_array_equal(rs, rso)
+
+
+@pytest.mark.parametrize("K", [16, 512, 2048, 8192])
+def test_quant_fwht_bit_exact(K):
+    X = _acts(33, K, seed=K, outliers=True)
+    q, s, rs = gpu_quant(X, bn.BITNET_PRELUDE_FWHT)
+    qo, so, rso = oracle.quant_act(X, oracle.PRELUDE_FWHT)
+    np.testing.assert_array_equal(q, qo)
+    np.testing.assert_array_equal(s, so)
+    np.testing.assert_array_equal(rs, rso)
+
+
+@pytest.mark.parametrize("M,K,with_gain", [(64, 2560, False), (17, 6912, True), (5, 48, True)])
+def test_quant_rmsnorm(M, K, with_gain):
+    X = _acts(M, K, seed=K + M)
+    gain = (np.random.default_rng(3).uniform(0.5, 1.5, K).astype(np.float32)
+            if with_gain else None)
+    q, s, rs = gpu_quant(X, bn.BITNET_PRELUDE_RMSNORM, gain=gain, eps=1e-5)
+    qo, so, rso = oracle.quant_act(X, oracle.PRELUDE_RMSNORM, gain=gain, eps=1e-5)
+    assert_codes_chain(q, qo, "rmsnorm codes")
+    n, _ = code_mismatch_stats(q, qo)
+    if n == 0:
+        np.testing.assert_array_equal(s, so)
+        np.testing.assert_array_equal(rs, rso)
+    else:
+        np.testing.assert_allclose(s, so, rtol=1e-6)
+
+
+def test_quant_bf16_input():
+    X = _acts(40, 2560, seed=5)
+    bits = synthetic.to_bf16_bits(X)
+    xw = oracle.bf16_bits_to_f32(bits)
+    q, s, rs = gpu_quant(xw, x_dev=bf16_dev(bits))
+    qo, so, rso = oracle.quant_act(xw)
+    np.testing.assert_array_equal(q, qo)
+    np.testing.assert_array_equal(s, so)
+    np.testing.assert_array_equal(rs, rso)
+    q, s, rs = gpu_quant(xw, bn.BITNET_PRELUDE_RMSNORM, x_dev=bf16_dev(bits))
+    qo, so, rso = oracle.quant_act(xw, oracle.PRELUDE_RMSNORM)
+    assert_codes_chain(q, qo, "bf16 rmsnorm codes")
+
+
+def test_quant_scale_invariance_on_device():
+    """Codes are identical under x -> 2^k x (no prelude, and RMSNorm with eps 0)."""
+    X = _acts(16, 1024, seed=9)
+    q0, s0, _ = gpu_quant(X)
+    q1, s1, _ = gpu_quant(X * np.float32(8.0))
+    np.testing.assert_array_equal(q0, q1)
+    np.testing.assert_array_equal(s0, s1 * np.float32(8.0))
+    r0, _, _ = gpu_quant(X, bn.BITNET_PRELUDE_RMSNORM, eps=0.0)
+    r1, _, _ = gpu_quant(X * np.float32(0.25), bn.BITNET_PRELUDE_RMSNORM, eps=0.0)
+    np.testing.assert_array_equal(r0, r1)
+
+
+@pytest.mark.parametrize("N,K", [(1, 16), (7, 80), (512, 256), (300, 2560), (6912, 2560),
+                                 (2560, 6912)])
+def test_pack_bit_exact(N, K):
+    W = synthetic.weight(np.random.default_rng(N + K), N, K)
+    packed, gamma = gpu_pack(W)
+    go = oracle.absmean(W)
+    assert gamma == go, (gamma, go)
+    np.testing.assert_array_equal(packed, oracle.pack(oracle.ternarize(W, go)))
+
+
+def test_pack_bf16_weights_and_edge_values():
+    rng = np.random.default_rng(4)
+    W = synthetic.weight(rng, 64, 128)
+    bits = synthetic.to_bf16_bits(W)
+    Ww = oracle.bf16_bits_to_f32(bits)
+    N, K = Ww.shape
+    packed, gamma, ws = bn.alloc_packed(N, K)
+    bn.bitnet_pack_weights(bf16_dev(bits), packed, gamma, ws)
+    torch.cuda.synchronize()
+    go = oracle.absmean(Ww)
+    assert gamma.item() == go
+    np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack(oracle.ternarize(Ww, go)))
+    # ties at exactly 0.5 and 1.5 gamma, and an all-zero matrix
+    T = np.array([[0.5, -1.5, 2.5, -0.5, 1.0, 0.0, -1.0, 1.0] * 2], dtype=np.float32)
+    packed, gamma = gpu_pack(T)
+    assert gamma == 1.0
+    np.testing.assert_array_equal(packed, oracle.pack(oracle.ternarize(T, np.float32(1.0))))
+    Z = np.zeros((3, 32), np.float32)
+    packed, gamma = gpu_pack(Z)
+    assert gamma == 0.0
+    assert np.all(packed == 0x55)
+
+
+def test_pack_is_deterministic():
+    W = synthetic.weight(np.random.default_rng(12), 2560, 2560)
+    a = gpu_pack(W)
+    b = gpu_pack(W)
+    assert a[1] == b[1]
+    np.testing.assert_array_equal(a[0], b[0])
