@@ -58,7 +58,7 @@ struct TcConfig {
   static constexpr int NUM_BARS = 3 * STAGES + 5;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TOK = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int TOK_BYTES_PER_WARP = BN * (8 * NW + 4);
+  static constexpr int TOK_BYTES_PER_WARP = BN * (8 * NW + 4);   // (f_hi, f_lo) per matrix + sum q
   static constexpr int SMEM_BYTES = OFF_TOK + 4 * TOK_BYTES_PER_WARP;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
   static constexpr uint32_t TX_BYTES = X_STAGE + NW * W_STAGE;
@@ -224,26 +224,27 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 8) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
-    double* tok_f0 = reinterpret_cast<double*>(smem + C::OFF_TOK + q * C::TOK_BYTES_PER_WARP);
-    double* tok_f1 = tok_f0 + C::BN;             // GLU only
+    float2* tok_f0 = reinterpret_cast<float2*>(smem + C::OFF_TOK + q * C::TOK_BYTES_PER_WARP);
+    float2* tok_f1 = tok_f0 + C::BN;             // GLU only
     int* tok_rs = reinterpret_cast<int*>(tok_f0 + C::NW * C::BN);
-    const double g0 = (double)__ldg(p.gamma0);
-    const double g1 = C::GLU ? (double)__ldg(p.gamma1) : 0.0;
+    const float g0 = __ldg(p.gamma0);
+    const float g1 = C::GLU ? __ldg(p.gamma1) : 0.0f;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
       const int m0 = tm * C::BN;
       const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
+      // per-token dequant factors gamma / s (fp32 head + tail) and sums of codes
       __syncwarp();
       for (int j = lane; j < C::BN; j += 32) {
         const int m = m0 + j;
-        double f0 = 0.0, f1 = 0.0;
+        float2 f0 = make_float2(0.0f, 0.0f), f1 = make_float2(0.0f, 0.0f);
         int rs = 0;
         if (m < p.M) {
-          const double s = (double)p.xs[m];
-          f0 = g0 / s;
-          if (C::GLU) f1 = g1 / s;
+          const float s = p.xs[m];
+          dequant_factor(g0, s, f0.x, f0.y);
+          if (C::GLU) dequant_factor(g1, s, f1.x, f1.y);
           rs = p.xrs[m];
         }
         tok_f0[j] = f0;
@@ -268,8 +269,9 @@ __global__ void __launch_bounds__(384, 1)
             const int t = 32 * c + j, m = m0 + t;
             if (n_ok && m < p.M) {
               const int rs = tok_rs[t];
-              const float g = (float)((double)((int)v[j] - rs) * tok_f0[t]);
-              const float uu = (float)((double)((int)u[j] - rs) * tok_f1[t]);
+              const float2 fa = tok_f0[t], fb = tok_f1[t];
+              const float g = dequant_dw((int)v[j] - rs, fa.x, fa.y);
+              const float uu = dequant_dw((int)u[j] - rs, fb.x, fb.y);
               const float a = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
               reinterpret_cast<float*>(p.Y)[(size_t)m * p.N + n] = __fmul_rn(a, uu);
             }
@@ -279,9 +281,17 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = 32 * c + j, m = m0 + t;
-            if (n_ok && m < p.M)
-              store_output(p.Y, p.resid, (size_t)m * p.N + n, (int)v[j] - tok_rs[t], tok_f0[t],
-                           p.out_type, p.flags);
+            if (n_ok && m < p.M) {
+              const int yint = (int)v[j] - tok_rs[t];
+              const size_t idx = (size_t)m * p.N + n;
+              if (p.out_type == OUT_I32) {
+                reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
+              } else {
+                const float2 fa = tok_f0[t];
+                store_value(p.Y, p.resid, idx, dequant_dw(yint, fa.x, fa.y), p.out_type,
+                            p.flags);
+              }
+            }
           }
         }
       }

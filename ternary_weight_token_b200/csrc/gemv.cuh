@@ -35,14 +35,36 @@ struct LinearParams {
   const void* resid;
 };
 
-// Shared epilogue: int32 contraction -> stored output element.
-__device__ __forceinline__ void store_output(void* Y, const void* resid, size_t idx, int yint,
-                                             double f, int out_type, int flags) {
-  if (out_type == OUT_I32) {
-    reinterpret_cast<int32_t*>(Y)[idx] = yint;
-    return;
-  }
-  float y = (float)((double)yint * f);
+// Exact int -> float for |v| < 2^22 with two ALU/FMA ops (no conversion
+// unit): place v in the mantissa of 1.5 * 2^23 and subtract 1.5 * 2^23.
+__device__ __forceinline__ float int_to_float_exact(int v) {
+  return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
+}
+
+// y = v * (f_hi + f_lo) in fp32 double-word arithmetic, where f_hi + f_lo is
+// gamma / s to about 2^-48 relative: the two-product error term is exact
+// (FMA), so the one rounding of the sum gives the correctly rounded fp32 of
+// v * gamma / s except when that value lies within ~2^-46 of an fp32
+// midpoint.  The accumulator |v| <= 128 * K <= 2^21 is exact in fp32.
+__device__ __forceinline__ float dequant_dw(int v, float f_hi, float f_lo) {
+  const float a = int_to_float_exact(v);
+  const float p = __fmul_rn(a, f_hi);
+  const float e = __fmaf_rn(a, f_hi, -p);
+  const float t = __fmaf_rn(a, f_lo, e);
+  return __fadd_rn(p, t);
+}
+
+// Split gamma / s (computed in fp64) into an fp32 head and tail.
+__device__ __forceinline__ void dequant_factor(float gamma, float s, float& f_hi, float& f_lo) {
+  const double f = (double)gamma / (double)s;
+  f_hi = (float)f;
+  f_lo = (float)(f - (double)f_hi);
+}
+
+// Epilogue tail shared by the decode and prefill kernels: fp32 value ->
+// optional SiLU / residual -> stored element.
+__device__ __forceinline__ void store_value(void* Y, const void* resid, size_t idx, float y,
+                                            int out_type, int flags) {
   if (flags & EPI_SILU) {
     const double d = (double)y;
     y = (float)(d / (1.0 + exp(-d)));
@@ -65,7 +87,7 @@ constexpr int kGemvRows = 2;   // weight rows per warp task
 template <int MT>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
   extern __shared__ uint4 gemv_smem[];          // [MT][ldw / 4] activation codes (16 B units)
-  __shared__ double tok_f[MT];
+  __shared__ float2 tok_f[MT];
   __shared__ int tok_rs[MT];
 
   const int chunks = p.ldw / 16;                // 16-byte packed chunks (64 weights) per row
@@ -78,13 +100,14 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
   }
   if (threadIdx.x < MT) {
     const int m = threadIdx.x;
+    float2 f = make_float2(0.0f, 0.0f);
+    int rs = 0;
     if (m < p.M) {
-      tok_f[m] = (double)__ldg(p.gamma) / (double)p.xs[m];
-      tok_rs[m] = p.xrs[m];
-    } else {
-      tok_f[m] = 0.0;
-      tok_rs[m] = 0;
+      dequant_factor(__ldg(p.gamma), p.xs[m], f.x, f.y);
+      rs = p.xrs[m];
     }
+    tok_f[m] = f;
+    tok_rs[m] = rs;
   }
   __syncthreads();
 
@@ -144,7 +167,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
         const int n = n0 + r;
         if (lane == ((r * MT + m) & 31) && m < p.M && n < p.N) {
           const size_t idx = (size_t)m * p.N + n;
-          store_output(p.Y, p.resid, idx, acc[r][m] - tok_rs[m], tok_f[m], p.out_type, p.flags);
+          const int yint = acc[r][m] - tok_rs[m];
+          if (p.out_type == OUT_I32)
+            reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
+          else
+            store_value(p.Y, p.resid, idx, dequant_dw(yint, tok_f[m].x, tok_f[m].y), p.out_type,
+                        p.flags);
         }
       }
   }
