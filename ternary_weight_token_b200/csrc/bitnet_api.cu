@@ -100,11 +100,11 @@ int get_encode_fn(EncodeTiledFn& fn) {
 struct MapKey {
   uintptr_t ptr;
   uint64_t d0, d1, stride;
-  uint32_t b0, b1, swz;
+  uint32_t b0, b1, swz, dtype;
   int dev;
   bool operator==(const MapKey& o) const {
     return ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && stride == o.stride && b0 == o.b0 &&
-           b1 == o.b1 && swz == o.swz && dev == o.dev;
+           b1 == o.b1 && swz == o.swz && dtype == o.dtype && dev == o.dev;
   }
 };
 struct MapKeyHash {
@@ -114,7 +114,8 @@ struct MapKeyHash {
     h = h * 1000003u ^ std::hash<uint64_t>()(k.d1);
     h = h * 1000003u ^ std::hash<uint64_t>()(k.stride);
     h = h * 1000003u ^ std::hash<uint64_t>()(((uint64_t)k.b0 << 32) | k.b1);
-    h = h * 1000003u ^ std::hash<uint64_t>()(((uint64_t)k.swz << 32) | (uint32_t)k.dev);
+    h = h * 1000003u ^ std::hash<uint64_t>()(((uint64_t)k.swz << 40) | ((uint64_t)k.dtype << 32) |
+                                             (uint32_t)k.dev);
     return h;
   }
 };
@@ -122,12 +123,15 @@ struct MapKeyHash {
 std::mutex g_map_mu;
 std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_map_cache;
 
-// 2-D byte tensor [d1 rows][d0 bytes] with row stride `stride` bytes.
-int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1, uint64_t stride,
-                     uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+// 2-D tensor [d1 rows][d0 elements] of `dtype` with row stride `stride` bytes,
+// box [b1 rows][b0 elements].
+int tensor_map_2d(CUtensorMap& out, const void* ptr, CUtensorMapDataType dtype, uint64_t d0,
+                  uint64_t d1, uint64_t stride, uint32_t b0, uint32_t b1,
+                  CUtensorMapSwizzle swz) {
   int dev = 0;
   BN_CHECK_CUDA(cudaGetDevice(&dev));
-  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, stride, b0, b1, (uint32_t)swz, dev};
+  MapKey key{reinterpret_cast<uintptr_t>(ptr), d0, d1, stride, b0, b1, (uint32_t)swz,
+             (uint32_t)dtype, dev};
   {
     std::lock_guard<std::mutex> lock(g_map_mu);
     auto it = g_map_cache.find(key);
@@ -142,13 +146,18 @@ int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1
   cuuint64_t strides[1] = {stride};
   cuuint32_t box[2] = {b0, b1};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides,
-                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(&out, dtype, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   std::lock_guard<std::mutex> lock(g_map_mu);
   g_map_cache[key] = out;
   return BITNET_OK;
+}
+
+int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1, uint64_t stride,
+                     uint32_t b0, uint32_t b1, CUtensorMapSwizzle swz) {
+  return tensor_map_2d(out, ptr, CU_TENSOR_MAP_DATA_TYPE_UINT8, d0, d1, stride, b0, b1, swz);
 }
 
 // ------------------------------------------------------------- launchers
@@ -213,7 +222,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
   CUtensorMap mx, mw0, mw1;
-  if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, C::BK,
+  if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return rc;
   if (int rc = tensor_map_2d_u8(mw0, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
@@ -225,7 +234,20 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
                                   C::BK / 4, C::BM, CU_TENSOR_MAP_SWIZZLE_NONE))
       return rc;
   }
+  // Output through TMA stores when its rows are whole 16-byte units.
+  const int esz = lp.out_type == OUT_BF16 ? 2 : 4;
+  const bool tma_out = ((size_t)lp.N * esz) % 16 == 0;
+  CUtensorMap my = mx;
+  if (tma_out) {
+    const CUtensorMapDataType dt = lp.out_type == OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : lp.out_type == OUT_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    if (int rc = tensor_map_2d(my, lp.Y, dt, (uint64_t)lp.N, (uint64_t)lp.M,
+                               (uint64_t)lp.N * esz, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return rc;
+  }
   TcParams p;
+  p.tma_out = tma_out ? 1 : 0;
   p.M = lp.M; p.N = lp.N; p.K = lp.K;
   p.num_kb = (lp.K + C::BK - 1) / C::BK;
   p.tiles_n = (lp.N + C::BM - 1) / C::BM;
@@ -242,16 +264,18 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   auto kern = gemm_tc_kernel<C>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
-  kern<<<grid, 384, smem, st>>>(mx, mw0, mw1, p);
+  kern<<<grid, C::THREADS, smem, st>>>(mx, mw0, mw1, my, p);
   BN_CHECK_CUDA(cudaGetLastError());
   return BITNET_OK;
 }
 
-using TcPlain = TcConfig<128, 6, false>;
-using TcGlu = TcConfig<64, 4, true>;
+using TcPlain = TcConfig<128, 256, 4, false>;
+using TcSilu = TcConfig<128, 256, 4, false, true>;
+using TcGlu = TcConfig<64, 128, 4, true>;
 
 int launch_linear(const LinearParams& p, cudaStream_t st) {
   if (p.M <= 16) return launch_gemv(p, st);
+  if (p.flags & EPI_SILU) return launch_tc_cfg<TcSilu>(p, nullptr, nullptr, st);
   return launch_tc_cfg<TcPlain>(p, nullptr, nullptr, st);
 }
 

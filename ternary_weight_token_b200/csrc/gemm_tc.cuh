@@ -21,15 +21,18 @@
 //   D (int32, 128 lanes x BN columns): tensor memory, double-buffered so the
 //       epilogue of one tile overlaps the MMAs of the next.
 //
-// Warp roles (384 threads, one persistent CTA per SM):
-//   warp 0      TMA producer (one thread)
-//   warp 1      MMA issuer (one thread)
-//   warp 2      tensor-memory allocator
-//   warps 4-7   converters (2-bit codes -> byte codes in TMEM)
-//   warps 8-11  epilogue (tcgen05.ld -> dequant -> fused op -> global stores)
+// Warp roles (one persistent CTA per SM; 384 threads with one converter
+// group, which keeps every role under the register cap with no spills):
+//   warp 0        TMA producer (one thread)
+//   warp 1        MMA issuer (one thread): 8 MMAs of K = 32 per 256-k stage
+//   warp 2        tensor-memory allocator
+//   warps 4..     converters (CONV_GROUPS groups of 4 warps alternate stages)
+//   last 4 warps  epilogue: tcgen05.ld -> dequant -> fused op -> a 32 x 32
+//                 tile staged in shared memory and written by a TMA store
+//                 (plain stores when the output rows are not 16-byte multiples)
 // Every wait is bounded; a wait that gives up records a device error, raises a
-// CTA-wide abort flag, and the CTA drains its tensor-core work, frees tensor
-// memory and exits.
+// CTA-wide abort flag, and the CTA drains its tensor-core work and bulk
+// copies, frees tensor memory and exits.
 #pragma once
 
 #include "common.cuh"
@@ -37,13 +40,17 @@
 
 namespace bitnet {
 
-template <int BN_, int STAGES_, bool GLU_>
+template <int BN_, int BK_, int STAGES_, bool GLU_, bool SILU_ = false, int CONV_GROUPS_ = 1>
 struct TcConfig {
+  static constexpr int CONV_GROUPS = CONV_GROUPS_;  // converter warp groups (alternate stages)
+  static constexpr bool SILU = SILU_;       // SiLU epilogue compiled in (H-BitLinear FFN)
   static constexpr int BN = BN_;            // tokens per tile (MMA N)
+  static constexpr int BK = BK_;            // k per pipeline stage (multiple of 128)
   static constexpr int STAGES = STAGES_;
   static constexpr bool GLU = GLU_;         // gate and up weights in one pass
   static constexpr int BM = 128;            // weight rows per tile (MMA M, TMEM lanes)
-  static constexpr int BK = 128;            // k per pipeline stage
+  static constexpr int XSUB = BN * 128;     // one 128-byte-wide swizzled activation sub-tile
+  static_assert(BK % 128 == 0 && BK <= 512, "BK");
   static constexpr int NW = GLU ? 2 : 1;    // weight matrices per stage
   static constexpr int X_STAGE = BN * BK;   // bytes of activation codes per stage
   static constexpr int W_STAGE = BM * BK / 4;  // bytes of packed weights per matrix per stage
@@ -52,14 +59,17 @@ struct TcConfig {
   static constexpr int TMEM_COLS = 512;
   static_assert(2 * ACC_COLS + STAGES * A_COLS <= TMEM_COLS, "tensor memory overflow");
   static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  static_assert(STAGES % CONV_GROUPS == 0, "converter groups alternate stages");
+  static constexpr int EPI_WARP0 = 4 + 4 * CONV_GROUPS;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + 4);
+  static constexpr int STAGE_OUT_BYTES = 32 * 32 * 4;          // one 32x32 output chunk (<= 4 B)
   static constexpr int OFF_X = 0;
   static constexpr int OFF_W = OFF_X + STAGES * X_STAGE;
-  static constexpr int OFF_BAR = OFF_W + STAGES * NW * W_STAGE;
+  static constexpr int OFF_OUT = OFF_W + STAGES * NW * W_STAGE;  // 4 warps x 2 buffers
+  static constexpr int OFF_BAR = OFF_OUT + 4 * 2 * STAGE_OUT_BYTES;
   static constexpr int NUM_BARS = 3 * STAGES + 5;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int OFF_TOK = (OFF_MISC + 16 + 15) / 16 * 16;
-  static constexpr int TOK_BYTES_PER_WARP = BN * (8 * NW + 4);   // (f_hi, f_lo) per matrix + sum q
-  static constexpr int SMEM_BYTES = OFF_TOK + 4 * TOK_BYTES_PER_WARP;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
   static constexpr uint32_t TX_BYTES = X_STAGE + NW * W_STAGE;
 };
@@ -76,14 +86,23 @@ struct TcParams {
   const void* resid;          // [M][N] or null
   int out_type;
   int flags;
+  int tma_out;                // 1: output written through the TMA map tm_y
 };
 
+__device__ __forceinline__ int out_elem_bytes(int out_type) { return out_type == OUT_BF16 ? 2 : 4; }
+
 template <class C>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(C::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ CUtensorMap tm_w0,
-                   const __grid_constant__ CUtensorMap tm_w1, TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_w1,
+                   const __grid_constant__ CUtensorMap tm_y, TcParams p) {
   extern __shared__ uint8_t tc_smem_raw[];
+  // per-token dequant factors (fp32 head, tail) and code sums, one copy per
+  // epilogue warp; static so they never alias the output staging buffers
+  __shared__ float2 s_tok_f[4][C::NW * C::BN];
+  __shared__ int s_tok_rs[4][C::BN];
+
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sx = smem + C::OFF_X;
@@ -118,6 +137,7 @@ __global__ void __launch_bounds__(384, 1)
     tma_prefetch_desc(&tm_x);
     tma_prefetch_desc(&tm_w0);
     if (C::GLU) tma_prefetch_desc(&tm_w1);
+    if (p.tma_out) tma_prefetch_desc(&tm_y);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -139,7 +159,10 @@ __global__ void __launch_bounds__(384, 1)
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) goto producer_done;
           mbar_arrive_expect_tx(&full[st], C::TX_BYTES);
-          tma_load_2d(sx + st * C::X_STAGE, &tm_x, &full[st], kb * C::BK, tm * C::BN);
+#pragma unroll
+          for (int xs = 0; xs < C::BK / 128; ++xs)
+            tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
+                        kb * C::BK + 128 * xs, tm * C::BN);
           tma_load_2d(sw + (st * C::NW) * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
                       tn * C::BM);
           if (C::GLU)
@@ -167,17 +190,20 @@ __global__ void __launch_bounds__(384, 1)
         const uint32_t d_col = tbase + ab * C::ACC_COLS;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
-          if (!mbar_wait(&full[st], ph, abort_flag)) goto mma_done;
+          // The converters arrive on afull[st] only after they observed full[st]
+          // complete, so this one wait also orders the MMA after the TMA bytes.
           if (!mbar_wait(&afull[st], ph, abort_flag)) goto mma_done;
           tc_fence_after();
           const uint32_t a_col = tbase + a_col0 + st * C::A_COLS;
           const uint32_t xaddr = smem_u32(sx + st * C::X_STAGE);
 #pragma unroll
           for (int j = 0; j < C::BK / 32; ++j) {
-            const uint64_t bdesc = make_sdesc_sw128(xaddr + 32u * j);
+            const uint64_t bdesc =
+                make_sdesc_sw128(xaddr + (uint32_t)((j >> 2) * C::XSUB) + 32u * (j & 3));
             const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
             mma_i8_ts(d_col, a_col + 8u * j, bdesc, idesc, acc);
-            if (C::GLU) mma_i8_ts(d_col + C::BN, a_col + 32u + 8u * j, bdesc, idesc, acc);
+            if (C::GLU)
+              mma_i8_ts(d_col + C::BN, a_col + (C::BK / 4) + 8u * j, bdesc, idesc, acc);
           }
           tc_commit(&empty[st]);
         }
@@ -187,22 +213,25 @@ __global__ void __launch_bounds__(384, 1)
       tc_commit(drain);
       mbar_wait(drain, 0, nullptr, 100000000ull);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < C::EPI_WARP0) {
     // ------------------------------------------------------- converters
+    const uint32_t group = (uint32_t)(warp - 4) >> 2;   // stages with it % groups == group
     const int q = warp & 3;
     const int row = 32 * q + lane;               // weight row within the tile = TMEM lane
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16) + a_col0;
-    uint32_t it = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-        const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
-        if (!mbar_wait(&full[st], ph, abort_flag)) goto convert_done;
-        tc_fence_after();
+    const uint32_t total = (uint32_t)((p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) /
+                                      (int)gridDim.x) * (uint32_t)p.num_kb;
+    for (uint32_t it = group; it < total; it += C::CONV_GROUPS) {
+      const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
+      if (!mbar_wait(&full[st], ph, abort_flag)) break;
+      tc_fence_after();
 #pragma unroll
-        for (int w = 0; w < C::NW; ++w) {
-          const uint4* src = reinterpret_cast<const uint4*>(sw + (st * C::NW + w) * C::W_STAGE +
-                                                            row * (C::BK / 4));
-          const uint4 a = src[0], b = src[1];
+      for (int w = 0; w < C::NW; ++w) {
+        const uint4* src = reinterpret_cast<const uint4*>(sw + (st * C::NW + w) * C::W_STAGE +
+                                                          row * (C::BK / 4));
+#pragma unroll
+        for (int h = 0; h < C::BK / 128; ++h) {   // 128 weights -> 32 TMEM columns
+          const uint4 a = src[2 * h], b = src[2 * h + 1];
           uint32_t e[32];
           expand_codes(a.x, e[0], e[1], e[2], e[3]);
           expand_codes(a.y, e[4], e[5], e[6], e[7]);
@@ -212,30 +241,30 @@ __global__ void __launch_bounds__(384, 1)
           expand_codes(b.y, e[20], e[21], e[22], e[23]);
           expand_codes(b.z, e[24], e[25], e[26], e[27]);
           expand_codes(b.w, e[28], e[29], e[30], e[31]);
-          tmem_st_32x32b_x32(lane_base + st * C::A_COLS + 32u * w, e);
+          tmem_st_32x32b_x32(lane_base + st * C::A_COLS + (C::BK / 4) * w + 32u * h, e);
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[st]);
       }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[st]);
     }
-  convert_done:;
-  } else if (warp >= 8) {
+  } else if (warp >= C::EPI_WARP0) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
-    float2* tok_f0 = reinterpret_cast<float2*>(smem + C::OFF_TOK + q * C::TOK_BYTES_PER_WARP);
-    float2* tok_f1 = tok_f0 + C::BN;             // GLU only
-    int* tok_rs = reinterpret_cast<int*>(tok_f0 + C::NW * C::BN);
+    float2* tok_f = s_tok_f[q];                  // [NW][BN]
+    int* tok_rs = s_tok_rs[q];
     const float g0 = __ldg(p.gamma0);
     const float g1 = C::GLU ? __ldg(p.gamma1) : 0.0f;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
-    uint32_t tcount = 0;
+    const int esz = out_elem_bytes(p.out_type);
+    const uint32_t out_base = smem_u32(smem + C::OFF_OUT + q * 2 * C::STAGE_OUT_BYTES);
+    uint32_t tcount = 0, chunk_count = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
       const int m0 = tm * C::BN;
+      const int nq0 = tn * C::BM + 32 * q;       // first weight row of this warp
       const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
-      // per-token dequant factors gamma / s (fp32 head + tail) and sums of codes
       __syncwarp();
       for (int j = lane; j < C::BN; j += 32) {
         const int m = m0 + j;
@@ -247,18 +276,21 @@ __global__ void __launch_bounds__(384, 1)
           if (C::GLU) dequant_factor(g1, s, f1.x, f1.y);
           rs = p.xrs[m];
         }
-        tok_f0[j] = f0;
-        if (C::GLU) tok_f1[j] = f1;
+        tok_f[j] = f0;
+        if (C::GLU) tok_f[C::BN + j] = f1;
         tok_rs[j] = rs;
       }
       __syncwarp();
       if (!mbar_wait(&accfull[ab], aph, abort_flag)) break;
       tc_fence_after();
-      const int n = tn * C::BM + 32 * q + lane;
+      const int n = nq0 + lane;
       const bool n_ok = n < p.N;
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c) {
+      for (int c = 0; c < C::BN / 32; ++c, ++chunk_count) {
+        const int mc = m0 + 32 * c;              // first token of this chunk
+        if (mc >= p.M) break;                    // the rest of the tile is past the last token
         uint32_t v[32];
+        float y[32];
         tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, v);
         if (C::GLU) {
           uint32_t u[32];
@@ -266,31 +298,77 @@ __global__ void __launch_bounds__(384, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int t = 32 * c + j, m = m0 + t;
-            if (n_ok && m < p.M) {
-              const int rs = tok_rs[t];
-              const float2 fa = tok_f0[t], fb = tok_f1[t];
-              const float g = dequant_dw((int)v[j] - rs, fa.x, fa.y);
-              const float uu = dequant_dw((int)u[j] - rs, fb.x, fb.y);
-              const float a = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
-              reinterpret_cast<float*>(p.Y)[(size_t)m * p.N + n] = __fmul_rn(a, uu);
-            }
+            const int t = 32 * c + j;
+            const int rs = tok_rs[t];
+            const float2 fa = tok_f[t], fb = tok_f[C::BN + t];
+            const float g = dequant_dw((int)v[j] - rs, fa.x, fa.y);
+            const float uu = dequant_dw((int)u[j] - rs, fb.x, fb.y);
+            const float a = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
+            y[j] = __fmul_rn(a, uu);
           }
         } else {
           tmem_ld_wait();
+          if (p.out_type == OUT_I32) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) y[j] = __int_as_float((int)v[j] - tok_rs[32 * c + j]);
+          } else {
+            const bool resid = (p.flags & EPI_RESIDUAL) != 0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = 32 * c + j;
+              const float2 fa = tok_f[t];
+              float yy = dequant_dw((int)v[j] - tok_rs[t], fa.x, fa.y);
+              if (C::SILU) {            // only the SiLU instance carries the exp call
+                const double d = (double)yy;
+                yy = (float)(d / (1.0 + exp(-d)));
+              }
+              if (resid) {
+                const int m = mc + j;
+                if (n_ok && m < p.M) {
+                  const size_t idx = (size_t)m * p.N + n;
+                  const float r = p.out_type == OUT_BF16
+                                      ? __bfloat162float(
+                                            reinterpret_cast<const __nv_bfloat16*>(p.resid)[idx])
+                                      : reinterpret_cast<const float*>(p.resid)[idx];
+                  yy = __fadd_rn(r, yy);
+                }
+              }
+              y[j] = yy;
+            }
+          }
+        }
+        if (p.tma_out) {
+          // stage the 32 (tokens) x 32 (weight rows) chunk as rows of the
+          // output, then one TMA store; two buffers per warp alternate
+          const uint32_t buf = out_base + (chunk_count & 1u) * C::STAGE_OUT_BYTES;
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+          if (esz == 2) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              st_shared_u16(buf + (uint32_t)(j * 32 + lane) * 2u,
+                            __bfloat16_as_ushort(__float2bfloat16_rn(y[j])));
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              st_shared_u32(buf + (uint32_t)(j * 32 + lane) * 4u, __float_as_uint(y[j]));
+          }
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0 && nq0 < p.N) {
+            tma_store_2d(&tm_y, smem + (buf - smem_u32(smem)), nq0, mc);
+            bulk_commit_group();
+          }
+        } else if (n_ok) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
-            const int t = 32 * c + j, m = m0 + t;
-            if (n_ok && m < p.M) {
-              const int yint = (int)v[j] - tok_rs[t];
+            const int m = mc + j;
+            if (m < p.M) {
               const size_t idx = (size_t)m * p.N + n;
-              if (p.out_type == OUT_I32) {
-                reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
-              } else {
-                const float2 fa = tok_f0[t];
-                store_value(p.Y, p.resid, idx, dequant_dw(yint, fa.x, fa.y), p.out_type,
-                            p.flags);
-              }
+              if (p.out_type == OUT_BF16)
+                reinterpret_cast<__nv_bfloat16*>(p.Y)[idx] = __float2bfloat16_rn(y[j]);
+              else
+                reinterpret_cast<float*>(p.Y)[idx] = y[j];   // fp32, or int32 bits
             }
           }
         }
@@ -299,6 +377,8 @@ __global__ void __launch_bounds__(384, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[ab]);
     }
+    if (lane == 0) bulk_wait_group_all();      // output stores complete before exit
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown

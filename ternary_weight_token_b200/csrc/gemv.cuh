@@ -54,11 +54,14 @@ __device__ __forceinline__ float dequant_dw(int v, float f_hi, float f_lo) {
   return __fadd_rn(p, t);
 }
 
-// Split gamma / s (computed in fp64) into an fp32 head and tail.
+// Split gamma / s into an fp32 head and tail: the head is the correctly
+// rounded quotient, the remainder gamma - head * s is exact in fp32 (one FMA),
+// and the tail is that remainder divided by s, so head + tail equals gamma / s
+// to about 2^-48 relative.  Only fp32 division and FMA (no fp64 unit).
 __device__ __forceinline__ void dequant_factor(float gamma, float s, float& f_hi, float& f_lo) {
-  const double f = (double)gamma / (double)s;
-  f_hi = (float)f;
-  f_lo = (float)(f - (double)f_hi);
+  f_hi = __fdiv_rn(gamma, s);
+  const float r = __fmaf_rn(-f_hi, s, gamma);
+  f_lo = __fdiv_rn(r, s);
 }
 
 // Epilogue tail shared by the decode and prefill kernels: fp32 value ->
