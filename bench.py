@@ -207,10 +207,10 @@ def oracle_prefill_sample(target_s=12.0, max_tokens=PREFILL_M):
             oracle.round_bf16(y)
         return time.perf_counter() - t0
 
-    tokens = 8
-    dt = run(tokens)
-    if dt < target_s:
-        tokens = int(min(max_tokens, max(8, tokens * target_s / max(dt, 1e-3) * 0.8)))
+    run(4)                                    # warm the oracle (page faults, threads)
+    tokens, dt = 8, run(8)
+    while dt < target_s and tokens < max_tokens:
+        tokens = int(min(max_tokens, max(2 * tokens, tokens * target_s / max(dt, 1e-3) * 1.05)))
         dt = run(tokens)
     ops = sum(2 * tokens * N * K for K, N in PREFILL_KN)
     return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": threads, "kind": "oracle",

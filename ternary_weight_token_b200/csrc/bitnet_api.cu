@@ -161,6 +161,20 @@ int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1
 }
 
 // ------------------------------------------------------------- launchers
+template <int NT, int VPT>
+int launch_quant_reg(const QuantParams& p, bool bf16, int prelude, int grid, cudaStream_t st) {
+  void (*kern)(QuantParams) = nullptr;
+  if (prelude == PRE_RMSNORM)
+    kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_RMSNORM, true>
+                : quant_act_reg_kernel<NT, VPT, PRE_RMSNORM, false>;
+  else
+    kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_NONE, true>
+                : quant_act_reg_kernel<NT, VPT, PRE_NONE, false>;
+  kern<<<grid, NT, 0, st>>>(p);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
 int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const float* gain,
                  float eps, int8_t* Xq, float* scale, int32_t* rowsum, cudaStream_t st) {
   DeviceInfo di;
@@ -169,18 +183,19 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   p.X = X; p.M = M; p.K = K; p.gain = gain; p.eps = eps;
   p.fwht_c = (float)(1.0 / std::sqrt((double)K));
   p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
+  if (prelude != PRE_FWHT) {
+    // register-resident rows: NT threads x VPT float4 must cover K / 4
+    const int grid = M < di.sms * 32 ? M : di.sms * 32;
+    const int k4 = K / 4;
+    if (k4 <= 64 * 4) return launch_quant_reg<64, 4>(p, bf16, prelude, grid, st);
+    if (k4 <= 128 * 6) return launch_quant_reg<128, 6>(p, bf16, prelude, grid, st);
+    if (k4 <= 256 * 8) return launch_quant_reg<256, 8>(p, bf16, prelude, grid, st);
+    return launch_quant_reg<512, 8>(p, bf16, prelude, grid, st);   // K <= 16384
+  }
   const int threads = K >= 2048 ? 256 : 128;
   const size_t smem = (size_t)K * sizeof(float);
   const int grid = M < di.sms * 16 ? M : di.sms * 16;
-  void (*kern)(QuantParams) = nullptr;
-  switch (prelude * 2 + (bf16 ? 1 : 0)) {
-    case 0: kern = quant_act_kernel<PRE_NONE, false>; break;
-    case 1: kern = quant_act_kernel<PRE_NONE, true>; break;
-    case 2: kern = quant_act_kernel<PRE_RMSNORM, false>; break;
-    case 3: kern = quant_act_kernel<PRE_RMSNORM, true>; break;
-    case 4: kern = quant_act_kernel<PRE_FWHT, false>; break;
-    default: kern = quant_act_kernel<PRE_FWHT, true>; break;
-  }
+  void (*kern)(QuantParams) = bf16 ? quant_act_kernel<PRE_FWHT, true> : quant_act_kernel<PRE_FWHT, false>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   kern<<<grid, threads, smem, st>>>(p);
   BN_CHECK_CUDA(cudaGetLastError());

@@ -219,4 +219,106 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
   }
 }
 
+// Register-resident variant for the NONE and RMSNORM preludes: one CTA per
+// token row, NT threads, each holding up to VPT float4 of the row in
+// registers.  Every 16-byte load of the row is in flight before the first
+// reduction, so the kernel streams at HBM bandwidth; the row is read once.
+template <int NT, int VPT, int PRE, bool BF16>
+__global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
+  static_assert(PRE == PRE_NONE || PRE == PRE_RMSNORM, "FWHT uses the shared-memory kernel");
+  static_assert(!BF16 || VPT % 2 == 0, "bf16 rows load 8 values per 16 bytes");
+  __shared__ double red_d[33];
+  __shared__ float red_f[33];
+  __shared__ int red_i[33];
+  const int K = p.K, K4 = p.K / 4;
+  const int tid = threadIdx.x;
+  for (int m = blockIdx.x; m < p.M; m += gridDim.x) {
+    float4 v[VPT];
+    if (BF16) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const __nv_bfloat16*>(p.X) + (size_t)m * K);
+#pragma unroll
+      for (int i = 0; i < VPT / 2; ++i) {
+        const int idx = tid + i * NT;            // 8-value unit
+        uint4 u = make_uint4(0u, 0u, 0u, 0u);
+        if (idx < K / 8) u = src[idx];
+        v[2 * i] = make_float4(bf16_bits_to_f32(u.x & 0xffffu), bf16_bits_to_f32(u.x >> 16),
+                               bf16_bits_to_f32(u.y & 0xffffu), bf16_bits_to_f32(u.y >> 16));
+        v[2 * i + 1] = make_float4(bf16_bits_to_f32(u.z & 0xffffu), bf16_bits_to_f32(u.z >> 16),
+                                   bf16_bits_to_f32(u.w & 0xffffu), bf16_bits_to_f32(u.w >> 16));
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.X) +
+                                                          (size_t)m * K);
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int idx = tid + i * NT;
+        v[i] = idx < K4 ? src[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    // element index of v[i].x: bf16 rows pair float4s inside one 8-value unit
+    auto kbase = [&](int i) -> int {
+      return BF16 ? 8 * (tid + (i / 2) * NT) + 4 * (i & 1) : 4 * (tid + i * NT);
+    };
+    float r = 1.0f;
+    if (PRE == PRE_RMSNORM) {
+      double ss = 0.0;
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        ss += (double)v[i].x * (double)v[i].x;
+        ss += (double)v[i].y * (double)v[i].y;
+        ss += (double)v[i].z * (double)v[i].z;
+        ss += (double)v[i].w * (double)v[i].w;
+      }
+      ss = block_sum_f64(ss, red_d);
+      const float ms = (float)(ss / (double)K);
+      r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int k = kbase(i);
+        if (k < K) {
+          float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+          if (p.gain) g = __ldg(reinterpret_cast<const float4*>(p.gain + k));
+          v[i].x = __fmul_rn(__fmul_rn(v[i].x, r), g.x);
+          v[i].y = __fmul_rn(__fmul_rn(v[i].y, r), g.y);
+          v[i].z = __fmul_rn(__fmul_rn(v[i].z, r), g.z);
+          v[i].w = __fmul_rn(__fmul_rn(v[i].w, r), g.w);
+        }
+      }
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i)
+      amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v[i].x)), fmaxf(fabsf(v[i].y), fabsf(v[i].z))),
+                   fabsf(v[i].w));
+    amax = block_max_f32(amax, red_f);
+    float s = __fdiv_rn(127.0f, amax);
+    const bool zero_row = (amax == 0.0f) || isinf(s);
+    if (zero_row) s = 1.0f;
+    int rsum = 0;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.Xq + (size_t)m * K);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int k = kbase(i);
+      if (k < K) {
+        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+        if (!zero_row) {
+          q0 = quant_code(v[i].x, s);
+          q1 = quant_code(v[i].y, s);
+          q2 = quant_code(v[i].z, s);
+          q3 = quant_code(v[i].w, s);
+        }
+        rsum += q0 + q1 + q2 + q3;
+        dst[k / 4] = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
+                     ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+      }
+    }
+    if (p.rowsum != nullptr) rsum = block_sum_i32(rsum, red_i);
+    if (tid == 0) {
+      p.scale[m] = s;
+      if (p.rowsum != nullptr) p.rowsum[m] = rsum;
+    }
+  }
+}
+
 }  // namespace bitnet
