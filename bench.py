@@ -354,15 +354,16 @@ def bench_decode(torch, bn, device, reps=3):
             q, s, rs = bn.alloc_quant(M, K, device)
             bn.bitnet_quant_act(X[:M].contiguous(), q, s, rs)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            epi = bn.BITNET_BF16 | bn.BITNET_LAUNCH_PDL
             for Pb in pool_bufs[:2]:
-                bn.bitnet_linear(q, s, rs, Pb, g, K, Y)
+                bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi)
             torch.cuda.synchronize()
             graph = torch.cuda.CUDAGraph()
             stream = torch.cuda.Stream(device)
             with torch.cuda.stream(stream):
                 graph.capture_begin(capture_error_mode="thread_local")
                 for Pb in pool_bufs:
-                    bn.bitnet_linear(q, s, rs, Pb, g, K, Y, stream=stream)
+                    bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi, stream=stream)
                 graph.capture_end()
             torch.cuda.synchronize()
             graph.replay()

@@ -87,6 +87,13 @@ extern "C" {
 #define BITNET_EPI_TYPE_MASK  0x0f
 #define BITNET_EPI_RESIDUAL   0x10  /* y = residual[m][n] + y (residual has Y's type; F32/BF16) */
 #define BITNET_EPI_SILU       0x20  /* y = silu(y) = y / (1 + exp(-y)) (F32/BF16)               */
+/* Launch hint for the decode path (M <= 16): the kernel may start before the
+ * preceding work on the stream has finished (programmatic dependent launch)
+ * and stream its packed weights early; activation codes, scales, code sums,
+ * gamma, residual and Y are touched only after that work has completed.  Set
+ * it only when the preceding work does not write the packed weights, e.g. in
+ * a decode loop over static weights.  Ignored for M > 16. */
+#define BITNET_LAUNCH_PDL     0x100
 
 /* ----------------------------------------------------------- FFN variants */
 #define BITNET_FFN_RELU2_GLU      0  /* x + down(subnorm(relu(gate(z))^2 * up(z))), z = RMSNorm(x) */

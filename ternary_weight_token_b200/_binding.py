@@ -19,6 +19,7 @@ BITNET_PRELUDE_NONE, BITNET_PRELUDE_RMSNORM, BITNET_PRELUDE_FWHT = 0, 1, 2
 BITNET_EPI_TYPE_MASK = 0x0F
 BITNET_EPI_RESIDUAL = 0x10
 BITNET_EPI_SILU = 0x20
+BITNET_LAUNCH_PDL = 0x100
 BITNET_FFN_RELU2_GLU, BITNET_FFN_HADAMARD_SILU = 0, 1
 
 _DTYPE_CODE = {torch.float32: BITNET_F32, torch.bfloat16: BITNET_BF16, torch.int32: BITNET_I32}

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_tc.cuh"
 #include "pack_weights.cuh"
 #include "quant_act.cuh"
 
@@ -288,8 +289,64 @@ using TcPlain = TcConfig<128, 256, 4, false>;
 using TcSilu = TcConfig<128, 256, 4, false, true>;
 using TcGlu = TcConfig<64, 128, 4, true>;
 
+// Decode on the tensor cores: 128-row weight tiles, each split over K across a
+// cluster of S CTAs (S <= 8, every slice at most 896 inputs).  Returns
+// BITNET_ERR_UNSUPPORTED when K is too long for that split.
+int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int units = lp.K / 64;
+  if (lp.K % 64 != 0 || units < 1) return BITNET_ERR_UNSUPPORTED;
+  const int s_min = (units + 13) / 14;                    // ceil(units / S) <= 14
+  const int s_max = units < kDecMaxCluster ? units : kDecMaxCluster;
+  if (s_min > s_max) return BITNET_ERR_UNSUPPORTED;
+  const int tiles = (lp.N + 127) / 128;
+  int S = s_min;
+  while (S < s_max && tiles * S < di.sms) ++S;
+  CUtensorMap mx, mw;
+  if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
+                                kDecTokens, CU_TENSOR_MAP_SWIZZLE_128B))
+    return rc;
+  if (int rc = tensor_map_2d_u8(mw, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
+                                kDecChunkK / 4, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return rc;
+  DecParams p;
+  p.M = lp.M; p.N = lp.N; p.K = lp.K; p.units = units;
+  p.xs = lp.xs; p.xrs = lp.xrs; p.gamma = lp.gamma;
+  p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type;
+  p.flags = lp.flags & ~LAUNCH_PDL;
+  static bool attr_set = false;
+  if (!attr_set) {
+    BN_CHECK_CUDA(cudaFuncSetAttribute(gemv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       DecSmem::ALLOC));
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(tiles * S), 1, 1);
+  cfg.blockDim = dim3(kDecThreads, 1, 1);
+  cfg.dynamicSmemBytes = DecSmem::ALLOC;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  attrs[0].id = cudaLaunchAttributeClusterDimension;
+  attrs[0].val.clusterDim.x = (unsigned)S;
+  attrs[0].val.clusterDim.y = 1;
+  attrs[0].val.clusterDim.z = 1;
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attrs[1].val.programmaticStreamSerializationAllowed = (lp.flags & LAUNCH_PDL) ? 1 : 0;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
+  BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, gemv_tc_kernel, mx, mw, p));
+  return BITNET_OK;
+}
+
 int launch_linear(const LinearParams& p, cudaStream_t st) {
-  if (p.M <= 16) return launch_gemv(p, st);
+  if (p.M <= 16) {
+    const int rc = launch_gemv_tc(p, st);
+    if (rc != BITNET_ERR_UNSUPPORTED) return rc;
+    LinearParams q = p;
+    q.flags &= ~LAUNCH_PDL;
+    return launch_gemv(q, st);                 // inputs too long for the cluster split
+  }
   if (p.flags & EPI_SILU) return launch_tc_cfg<TcSilu>(p, nullptr, nullptr, st);
   return launch_tc_cfg<TcPlain>(p, nullptr, nullptr, st);
 }
@@ -305,9 +362,9 @@ int validate_linear(const int8_t* Xq, const float* xs, const int32_t* xrs, const
   const int flags = epilogue & ~BITNET_EPI_TYPE_MASK;
   if (ot != BITNET_F32 && ot != BITNET_BF16 && ot != BITNET_I32)
     return fail(BITNET_ERR_INVALID_ARG, "bad output type %d", ot);
-  if (flags & ~(BITNET_EPI_RESIDUAL | BITNET_EPI_SILU))
+  if (flags & ~(BITNET_EPI_RESIDUAL | BITNET_EPI_SILU | BITNET_LAUNCH_PDL))
     return fail(BITNET_ERR_INVALID_ARG, "unknown epilogue flags 0x%x", flags);
-  if (ot == BITNET_I32 && flags)
+  if (ot == BITNET_I32 && (flags & (BITNET_EPI_RESIDUAL | BITNET_EPI_SILU)))
     return fail(BITNET_ERR_UNSUPPORTED, "the int32 output takes no residual or SiLU");
   if ((flags & BITNET_EPI_RESIDUAL) && resid == nullptr)
     return fail(BITNET_ERR_INVALID_ARG, "residual flag set but residual is NULL");
@@ -419,6 +476,7 @@ int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsu
   p.M = M; p.N = N; p.K = K; p.ldw = (int)bitnet_packed_row_bytes(K);
   p.Y = Y; p.out_type = epilogue & BITNET_EPI_TYPE_MASK;
   p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = residual;
+  if (M > 16) p.flags &= ~LAUNCH_PDL;
   return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -20,7 +20,7 @@
 namespace bitnet {
 
 enum { OUT_F32 = 0, OUT_BF16 = 1, OUT_I32 = 2 };
-enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20 };
+enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20, LAUNCH_PDL = 0x100 };
 
 struct LinearParams {
   const int8_t* Xq;

@@ -130,3 +130,42 @@ def test_full_chain_matches_oracle():
     torch.cuda.synchronize()
     g, T, _ = oracle.quantize_weights(W)
     assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="chain")
+
+
+def test_decode_with_programmatic_dependent_launch():
+    """Decode calls launched with BITNET_LAUNCH_PDL right behind the kernel that
+    writes their activation codes still read the new codes: each step quantises
+    a fresh token batch and immediately runs the projection on it."""
+    M, K, N = 4, 2560, 2560
+    rng_w, rng_x = synthetic.streams(41, 2)
+    W = synthetic.weight(rng_w, N, K)
+    g, T, P = oracle.quantize_weights(W)
+    Pd, gd = dev(P), dev(np.array([g], np.float32))
+    q, s, rs = bn.alloc_quant(M, K)
+    outs, xs = [], []
+    for step in range(6):
+        X = synthetic.activations(rng_x, M, K)
+        xs.append(X)
+        Xd = dev(X)
+        torch.cuda.synchronize()
+        bn.bitnet_quant_act(Xd, q, s, rs)
+        Y = torch.empty((M, N), device="cuda")
+        bn.bitnet_linear(q, s, rs, Pd, gd, K, Y, epilogue=bn.BITNET_F32 | bn.BITNET_LAUNCH_PDL)
+        outs.append(Y)
+    torch.cuda.synchronize()
+    for X, Y in zip(xs, outs):
+        assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="pdl step")
+
+
+@pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 6912), (6912, 2560)])
+def test_decode_shapes_all_m(K, N):
+    """The 2B-model decode shapes for every token count 1..16 (cluster split-K
+    tensor-core path), int32 bit-exact."""
+    rng_w, rng_x = synthetic.streams(K + N, 2)
+    W = synthetic.weight(rng_w, N, K)
+    g, T, P = oracle.quantize_weights(W)
+    X = synthetic.activations(rng_x, 16, K)
+    q, s, rs = oracle.quant_act(X)
+    for M in (1, 2, 3, 5, 8, 13, 16):
+        got = gpu_linear(q[:M], s[:M], rs[:M], P, g, K, N, out=torch.int32)
+        np.testing.assert_array_equal(got, oracle.contract(q[:M], T), err_msg=f"M={M}")
