@@ -191,6 +191,36 @@ BITNET_API int bitnet_ffn(const void *X, int x_dtype, int M, int H, int I,
                int variant, void *Y, int y_dtype,
                void *workspace, size_t ws_bytes, bitnet_stream_t stream);
 
+/* bitnet_ffn without a workspace argument, for callers that cannot allocate
+ * device memory: code running inside a CUDA stream capture whose mode forbids
+ * cudaMalloc, or plugins whose host application owns every device buffer and
+ * hands the library no allocator.  (No counterpart on the method's pages:
+ * this is a property of the library, not of BitLinear.)
+ *   Scratch    The intermediate buffers live in one file-scope device array of
+ *              BITNET_FFN_NOALLOC_SCRATCH_BYTES (8 MiB) inside the library.
+ *              Every GPU that loads the library holds it until the process
+ *              exits.  The request must fit:
+ *              bitnet_ffn_workspace_size(M, H, I, variant) <= that size (about
+ *              225 tokens of the 2560 -> 6912 -> 2560 FFN); a larger request
+ *              returns BITNET_ERR_WORKSPACE and launches nothing.
+ *   Set-up     The first call on each device looks up the device address of
+ *              the array (cudaGetSymbolAddress) with that device current; make
+ *              that first call before any stream capture begins.
+ *   Sharing    All calls on a device share the one array and it keeps the last
+ *              call's contents (nothing in it needs to start at zero).  Calls
+ *              that can overlap on the GPU (different streams, no ordering
+ *              between them) race on it: order them on one stream.
+ *   It allocates and frees nothing and calls no allocating routine.  All other
+ *   arguments, results and errors are those of bitnet_ffn(). */
+#define BITNET_FFN_NOALLOC_SCRATCH_BYTES (8u << 20)
+BITNET_API int bitnet_ffn_noalloc(const void *X, int x_dtype, int M, int H, int I,
+                                  const uint8_t *W_gate, const float *gamma_gate,
+                                  const uint8_t *W_up, const float *gamma_up,
+                                  const uint8_t *W_down, const float *gamma_down,
+                                  const float *pre_norm_gain, const float *sub_norm_gain,
+                                  float eps, int variant, void *Y, int y_dtype,
+                                  bitnet_stream_t stream);
+
 /* Message for the last non-OK status on this host thread ("" if none). */
 BITNET_API const char *bitnet_last_error(void);
 

@@ -41,6 +41,8 @@ from ._binding import (  # noqa: F401
     bitnet_check_device_error,
     bitnet_debug_wait_timeout,
     bitnet_ffn,
+    bitnet_ffn_noalloc,
+    BITNET_FFN_NOALLOC_SCRATCH_BYTES,
     bitnet_ffn_workspace_size,
     bitnet_last_error,
     bitnet_linear,

@@ -57,6 +57,7 @@ def library():
         "bitnet_linear": (I, [P, P, P, P, P, I, I, I, P, I, P, P]),
         "bitnet_ffn_workspace_size": (S, [I, I, I, I]),
         "bitnet_ffn": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P, S, P]),
+        "bitnet_ffn_noalloc": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P]),
         "bitnet_last_error": (ctypes.c_char_p, []),
         "bitnet_check_device_error": (I, [P]),
         "bitnet_debug_wait_timeout": (I, [U, P]),
@@ -167,6 +168,22 @@ def bitnet_ffn(X, W_gate, gamma_gate, W_up, gamma_up, W_down, gamma_down, Y, wor
                                 _ptr(pre_norm_gain), _ptr(sub_norm_gain), float(eps), int(variant),
                                 _ptr(Y), _dtype(Y), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+BITNET_FFN_NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def bitnet_ffn_noalloc(X, W_gate, gamma_gate, W_up, gamma_up, W_down, gamma_down, Y,
+                       variant=BITNET_FFN_RELU2_GLU, pre_norm_gain=None, sub_norm_gain=None,
+                       eps=1e-5, stream=None):
+    """bitnet_ffn on the library's built-in scratch (no workspace argument)."""
+    M, H = X.shape
+    I = W_gate.shape[0]
+    _check(library().bitnet_ffn_noalloc(_ptr(X), _dtype(X), M, H, I, _ptr(W_gate),
+                                        _ptr(gamma_gate), _ptr(W_up), _ptr(gamma_up),
+                                        _ptr(W_down), _ptr(gamma_down), _ptr(pre_norm_gain),
+                                        _ptr(sub_norm_gain), float(eps), int(variant), _ptr(Y),
+                                        _dtype(Y), _stream(stream)))
 
 
 def bitnet_check_device_error(stream=None):

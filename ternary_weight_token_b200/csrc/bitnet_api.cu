@@ -630,3 +630,60 @@ extern "C" int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t st
   BN_CHECK_CUDA(cudaGetLastError());
   return BITNET_OK;
 }
+
+// ------------------------------------------------------------------------
+// FFN without a workspace argument (bitnet_ffn_noalloc): the scratch is this
+// file-scope device array.  In host code `g_ffn_noalloc_scratch` is only a
+// host-side stand-in for the symbol, never a device address, so its device
+// address is looked up with cudaGetSymbolAddress once per device (with that
+// device current) and passed on as the workspace pointer.
+namespace bitnet {
+static __device__ __align__(256) uint8_t g_ffn_noalloc_scratch[BITNET_FFN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices)
+    return fail(BITNET_ERR_UNSUPPORTED, "device ordinal %d beyond %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_ffn_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(BITNET_ERR_CUDA, "cudaGetSymbolAddress of the FFN scratch failed: %s",
+                  cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return BITNET_OK;
+}
+}  // namespace bitnet
+
+extern "C" int bitnet_ffn_noalloc(const void* X, int x_dtype, int M, int H, int I,
+                                  const uint8_t* W_gate, const float* gamma_gate,
+                                  const uint8_t* W_up, const float* gamma_up,
+                                  const uint8_t* W_down, const float* gamma_down,
+                                  const float* pre_norm_gain, const float* sub_norm_gain,
+                                  float eps, int variant, void* Y, int y_dtype,
+                                  bitnet_stream_t stream) {
+  g_last_error.clear();
+  const size_t need = bitnet_ffn_workspace_size(M, H, I, variant);
+  if (need > (size_t)BITNET_FFN_NOALLOC_SCRATCH_BYTES)
+    return fail(BITNET_ERR_WORKSPACE,
+                "M=%d, H=%d, I=%d needs %zu bytes of scratch; the built-in scratch holds %u "
+                "(use bitnet_ffn with a workspace)",
+                M, H, I, need, (unsigned)BITNET_FFN_NOALLOC_SCRATCH_BYTES);
+  if (M <= 0)   // nothing to launch; bitnet_ffn validates the arguments
+    return bitnet_ffn(X, x_dtype, M, H, I, W_gate, gamma_gate, W_up, gamma_up, W_down,
+                      gamma_down, pre_norm_gain, sub_norm_gain, eps, variant, Y, y_dtype,
+                      nullptr, 0, stream);
+  void* scratch = nullptr;
+  if (int rc = noalloc_scratch(&scratch)) return rc;
+  return bitnet_ffn(X, x_dtype, M, H, I, W_gate, gamma_gate, W_up, gamma_up, W_down, gamma_down,
+                    pre_norm_gain, sub_norm_gain, eps, variant, Y, y_dtype, scratch,
+                    (size_t)BITNET_FFN_NOALLOC_SCRATCH_BYTES, stream);
+}
