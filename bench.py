@@ -563,6 +563,43 @@ def run_b200(args, world, rank, local):
     return 0
 
 
+def decode_single(torch, bn, device, M, K, N, iters):
+    """Plain back-to-back launches of one decode shape (no graph): the short
+    command the decode kernel is profiled with."""
+    inp = synthetic.linear_inputs(M, K, N, seed=K + N)
+    W = torch.from_numpy(inp["W"]).to(device)
+    P, g, ws = bn.alloc_packed(N, K, device)
+    bn.bitnet_pack_weights(W, P, g, ws)
+    X = torch.from_numpy(inp["X"]).to(device)
+    q, s, rs = bn.alloc_quant(M, K, device)
+    bn.bitnet_quant_act(X, q, s, rs)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+    def run():
+        bn.bitnet_linear(q, s, rs, P, g, K, Y)
+    for _ in range(3):
+        run()
+    dt = time_loop(torch, run, iters) / iters
+    return {"M": M, "K": K, "N": N, "us_per_call": dt * 1e6,
+            "GB_s": decode_bytes(M, K, N) / dt / 1e9}
+
+
+def run_only(args, local):
+    import torch
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    import ternary_weight_token_b200 as bn
+    if args.only == "decode" and args.decode_shape:
+        M, K, N = (int(v) for v in args.decode_shape.split(","))
+        out = decode_single(torch, bn, device, M, K, N, max(1, args.steps))
+    else:
+        fn = {"decode": bench_decode, "ffn": bench_ffn, "hffn": bench_hffn,
+              "tiny": bench_tiny}[args.only]
+        out = fn(torch, bn, device)
+    print(json.dumps({"only": args.only, "result": out}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -572,6 +609,10 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip decode / FFN / tiny workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny"), default=None,
+                    help="time one secondary workload and print its JSON (profiling aid)")
+    ap.add_argument("--decode-shape", default=None,
+                    help="with --only decode: one 'M,K,N' case, no CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3
@@ -583,6 +624,8 @@ def main(argv=None):
             return 2
     if args.impl == "reference":
         return run_reference(args, world, rank)
+    if args.only is not None:
+        return run_only(args, local)
     return run_b200(args, world, rank, local)
 
 

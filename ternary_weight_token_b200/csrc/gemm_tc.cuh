@@ -24,7 +24,9 @@
 // Warp roles (one persistent CTA per SM; 384 threads with one converter
 // group, which keeps every role under the register cap with no spills):
 //   warp 0        TMA producer (one thread)
-//   warp 1        MMA issuer (one thread): 8 MMAs of K = 32 per 256-k stage
+//   warps 1, 3    MMA issuers (one thread each, alternate stages): 8 MMAs of
+//                 K = 32 per 256-k stage, all accumulating into a buffer the
+//                 epilogue zeroed
 //   warp 2        tensor-memory allocator
 //   warps 4..     converters (CONV_GROUPS groups of 4 warps alternate stages)
 //   last 4 warps  epilogue: tcgen05.ld -> dequant -> fused op -> a 32 x 32
@@ -126,10 +128,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&afull[s], 4);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 4);
+      mbar_init(&accfull[b], 2);             // one commit from each MMA issuer
+      mbar_init(&accempty[b], 4);            // four epilogue warps (zeroed buffer)
     }
-    mbar_init(drain, 1);
+    mbar_init(drain, 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -178,17 +180,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         mbar_wait(&full[j % C::STAGES], (j / C::STAGES) & 1u, nullptr, 100000000ull);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------ MMA issuers
+    // Two threads issue the MMAs of alternate stages, so one waits for its
+    // next stage while the tensor pipe runs the other's.  Every MMA
+    // accumulates (int32 sums are exact in any order); the epilogue zeroes an
+    // accumulator buffer after reading it, before handing it back.
     if (lane == 0) {
+      const uint32_t me = warp == 1 ? 0u : 1u;
       const uint32_t idesc = make_idesc_i8(C::BM, C::BN);
       uint32_t it = 0, tcount = 0;
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-        const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
-        if (!mbar_wait(&accempty[ab], aph ^ 1u, abort_flag)) break;
+        const uint32_t ab = tcount & 1u, use = tcount >> 1;
+        if (!mbar_wait(&accempty[ab], use & 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_col = tbase + ab * C::ACC_COLS;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          if ((it & 1u) != me) continue;
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
           // The converters arrive on afull[st] only after they observed full[st]
           // complete, so this one wait also orders the MMA after the TMA bytes.
@@ -200,10 +208,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int j = 0; j < C::BK / 32; ++j) {
             const uint64_t bdesc =
                 make_sdesc_sw128(xaddr + (uint32_t)((j >> 2) * C::XSUB) + 32u * (j & 3));
-            const uint32_t acc = (kb > 0 || j > 0) ? 1u : 0u;
-            mma_i8_ts(d_col, a_col + 8u * j, bdesc, idesc, acc);
-            if (C::GLU)
-              mma_i8_ts(d_col + C::BN, a_col + (C::BK / 4) + 8u * j, bdesc, idesc, acc);
+            mma_i8_ts(d_col, a_col + 8u * j, bdesc, idesc, 1u);
+            if (C::GLU) mma_i8_ts(d_col + C::BN, a_col + (C::BK / 4) + 8u * j, bdesc, idesc, 1u);
           }
           tc_commit(&empty[st]);
         }
@@ -259,6 +265,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     const int esz = out_elem_bytes(p.out_type);
     const uint32_t out_base = smem_u32(smem + C::OFF_OUT + q * 2 * C::STAGE_OUT_BYTES);
+    uint32_t zero[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) zero[j] = 0u;
+    // both accumulator buffers start at zero: every MMA accumulates
+    for (int col = 0; col < 2 * C::ACC_COLS; col += 32) tmem_st_32x32b_x32(lane_base + col, zero);
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&accempty[0]);
+      mbar_arrive(&accempty[1]);
+    }
     uint32_t tcount = 0, chunk_count = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
@@ -288,7 +306,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll 1
       for (int c = 0; c < C::BN / 32; ++c, ++chunk_count) {
         const int mc = m0 + 32 * c;              // first token of this chunk
-        if (mc >= p.M) break;                    // the rest of the tile is past the last token
+        if (mc >= p.M) {                         // past the last token: only re-zero
+          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
+          if (C::GLU) tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, zero);
+          continue;
+        }
         uint32_t v[32];
         float y[32];
         tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, v);
@@ -296,6 +318,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           uint32_t u[32];
           tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, u);
           tmem_ld_wait();
+          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
+          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, zero);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = 32 * c + j;
@@ -308,6 +332,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         } else {
           tmem_ld_wait();
+          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
           if (p.out_type == OUT_I32) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = __int_as_float((int)v[j] - tok_rs[32 * c + j]);
@@ -373,6 +398,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         }
       }
+      tmem_st_wait();                            // the zeroed buffer is complete
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accempty[ab]);

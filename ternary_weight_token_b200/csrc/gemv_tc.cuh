@@ -64,8 +64,8 @@ struct DecSmem {
   static constexpr int OFF_PART = OFF_W + kDecMaxChunks * W_CHUNK; // [S][16][128] int32
   static constexpr int PART_BYTES = kDecTokens * 128 * 4;          // 8 KB per CTA
   static constexpr int OFF_BAR = OFF_PART + kDecMaxCluster * PART_BYTES;
-  // bars: wfull[chunks], xfull[chunks], afull[chunks], mma_done, reduce
-  static constexpr int NUM_BARS = 3 * kDecMaxChunks + 2;
+  // bars: wfull[chunks], xfull[chunks], aready, mma_done, reduce
+  static constexpr int NUM_BARS = 2 * kDecMaxChunks + 3;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;
@@ -92,9 +92,12 @@ __device__ __forceinline__ uint32_t cluster_nctarank() {
   return r;
 }
 
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // Shared-memory address of the same variable in CTA `rank` of the cluster.
@@ -173,8 +176,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DecSmem::OFF_BAR);
   uint64_t* wfull = bars;                                 // [chunks] weight bytes landed
   uint64_t* xfull = bars + kDecMaxChunks;                 // [chunks] activation bytes landed
-  uint64_t* afull = bars + 2 * kDecMaxChunks;             // [chunks] codes in TMEM
-  uint64_t* mma_done = bars + 3 * kDecMaxChunks;          // accumulator complete
+  uint64_t* aready = bars + 2 * kDecMaxChunks;            // every chunk's codes in TMEM
+  uint64_t* mma_done = aready + 1;                        // accumulator complete
   uint64_t* reduce_bar = mma_done + 1;                    // leader: all partials in
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + DecSmem::OFF_MISC);
 
@@ -192,8 +195,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     for (int c = 0; c < chunks; ++c) {
       mbar_init(&wfull[c], 1);
       mbar_init(&xfull[c], 1);
-      mbar_init(&afull[c], 4);
     }
+    mbar_init(aready, 4);
     mbar_init(mma_done, 1);
     mbar_init(reduce_bar, csize * 4);        // 4 storing warps per CTA
     fence_barrier_init();
@@ -203,8 +206,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     tmem_relinquish();
   }
   tc_fence_before();
-  cluster_sync_all();                        // barriers visible cluster-wide
+  __syncthreads();
   tc_fence_after();
+  // Arrive now, wait only before the first access to a peer's shared memory:
+  // the leader's barrier initialisation then reaches every peer while they
+  // stream their weights.
+  cluster_arrive();
   const uint32_t tbase = *tmem_slot;
   const uint32_t a_col0 = 32;                // D occupies columns [0, 16)
 
@@ -227,8 +234,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const int steps = ks / 32;
       int s = 0;
       bool ok = true;
+      ok = mbar_wait(aready, 0, nullptr);
       for (int c = 0; c < chunks && ok; ++c) {
-        ok = mbar_wait(&afull[c], 0, nullptr) && mbar_wait(&xfull[c], 0, nullptr);
+        ok = mbar_wait(&xfull[c], 0, nullptr);
         if (!ok) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(sx + c * DecSmem::X_CHUNK);
@@ -243,6 +251,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_wait(&xfull[c], 0, nullptr, 100000000ull);
       }
     }
+    __syncwarp();
+    cluster_wait();
   } else if (warp >= 2) {
     const int q = warp & 3;                  // TMEM lane quarter of this warp
     const int row = 32 * q + lane;           // weight row within the tile
@@ -263,11 +273,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       expand_codes(b.z, e[24], e[25], e[26], e[27]);
       expand_codes(b.w, e[28], e[29], e[30], e[31]);
       tmem_st_32x32b_x32(lane_base + a_col0 + 32u * c, e);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&afull[c]);
     }
+    // one wait for every chunk's stores, then one signal to the MMA thread
+    tmem_st_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(aready);
     // partial sums -> the leader's slot for this rank, as [token][row]
     uint32_t d[16];
     if (ok && mbar_wait(mma_done, 0, nullptr)) {
@@ -278,6 +289,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int t = 0; t < 16; ++t) d[t] = 0u;
     }
+    cluster_wait();                          // the leader's barriers are initialised
     const uint32_t part_local =
         smem_u32(smem + DecSmem::OFF_PART + rank * DecSmem::PART_BYTES) + 4u * row;
     const uint32_t part_remote = map_to_rank(part_local, 0);
@@ -287,28 +299,47 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     if (lane == 0) mbar_arrive_remote_release(map_to_rank(smem_u32(reduce_bar), 0));
 
     if (rank == 0) {
-      // leader: add the S partials, subtract sum q, dequantise, store
-      const bool all_in = mbar_wait_cluster(reduce_bar, 0);
+      // leader: token scales and code sums are fetched while the peers'
+      // partials arrive; then all partial sums are read before any output
+      // is stored (no load waits behind a store)
       grid_dependency_wait();
+      const float g = __ldg(p.gamma);
+      float sm[kDecTokens];
+      int rsum[kDecTokens];
+#pragma unroll
+      for (int m = 0; m < kDecTokens; ++m) {
+        sm[m] = m < p.M ? __ldg(p.xs + m) : 1.0f;
+        rsum[m] = m < p.M ? __ldg(p.xrs + m) : 0;
+      }
+      const bool all_in = mbar_wait_cluster(reduce_bar, 0);
       const int n = n0 + row;
       if (all_in && n < p.N) {
-        const float g = __ldg(p.gamma);
         const int32_t* part = reinterpret_cast<const int32_t*>(smem + DecSmem::OFF_PART);
-        for (int m = 0; m < p.M; ++m) {
-          int acc = 0;
-          for (int r = 0; r < (int)csize; ++r) acc += part[(r * 16 + m) * 128 + row];
-          const int yint = acc - p.xrs[m];
-          const size_t idx = (size_t)m * p.N + n;
-          if (p.out_type == OUT_I32) {
-            reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
-          } else {
-            float fh, fl;
-            dequant_factor(g, p.xs[m], fh, fl);
-            store_value(p.Y, p.resid, idx, dequant_dw(yint, fh, fl), p.out_type, p.flags);
+        int acc[kDecTokens];
+#pragma unroll
+        for (int m = 0; m < kDecTokens; ++m) acc[m] = -rsum[m];
+        for (int r = 0; r < (int)csize; ++r) {
+#pragma unroll
+          for (int m = 0; m < kDecTokens; ++m)
+            if (m < p.M) acc[m] += part[(r * 16 + m) * 128 + row];
+        }
+#pragma unroll
+        for (int m = 0; m < kDecTokens; ++m) {
+          if (m < p.M) {
+            const size_t idx = (size_t)m * p.N + n;
+            if (p.out_type == OUT_I32) {
+              reinterpret_cast<int32_t*>(p.Y)[idx] = acc[m];
+            } else {
+              float fh, fl;
+              dequant_factor(g, sm[m], fh, fl);
+              store_value(p.Y, p.resid, idx, dequant_dw(acc[m], fh, fl), p.out_type, p.flags);
+            }
           }
         }
       }
     }
+  } else {
+    cluster_wait();                          // every thread of the cluster barrier waits once
   }
 
   // Peers only write into the leader's shared memory, and the leader leaves
