@@ -223,7 +223,7 @@ def run_reference(args, world, rank):
     """Reference arm: the CPU oracle as it stands, on this host's cores."""
     if rank != 0:
         return 0
-    per_step = max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    per_step = args.ref_step_seconds or max(0.5, min(4.0, 150.0 / max(1, args.steps + args.warmup)))
     import oracle
     threads = oracle.num_threads()
     prepared = []
@@ -609,6 +609,8 @@ def main(argv=None):
     ap.add_argument("--no-extra", action="store_true", help="skip decode / FFN / tiny workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-step-seconds", type=float, default=None,
+                    help="with --impl reference: target seconds of oracle work per step")
     ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny"), default=None,
                     help="time one secondary workload and print its JSON (profiling aid)")
     ap.add_argument("--decode-shape", default=None,
