@@ -241,13 +241,18 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return rc;
+  // packed weight rows of BK/4 bytes, swizzled at that width (conflict-free
+  // 16-byte loads in the converter)
+  const CUtensorMapSwizzle wswz =
+      C::BK / 4 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  static_assert(C::BK / 4 == 64 || C::BK / 4 == 32, "packed stage width");
   if (int rc = tensor_map_2d_u8(mw0, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
-                                C::BK / 4, C::BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                                C::BK / 4, C::BM, wswz))
     return rc;
   mw1 = mw0;
   if (C::GLU) {
     if (int rc = tensor_map_2d_u8(mw1, W1, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
-                                  C::BK / 4, C::BM, CU_TENSOR_MAP_SWIZZLE_NONE))
+                                  C::BK / 4, C::BM, wswz))
       return rc;
   }
   // Output through TMA stores when its rows are whole 16-byte units.

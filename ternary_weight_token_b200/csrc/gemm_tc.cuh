@@ -233,11 +233,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
 #pragma unroll
       for (int w = 0; w < C::NW; ++w) {
+        // Packed rows are BK/4 bytes; TMA wrote them with the matching swizzle
+        // (16-byte chunk j of row r at chunk j ^ ((r / (128 / row_bytes)) %
+        // chunks)), so the 32 lanes' 16-byte loads hit distinct banks.
         const uint4* src = reinterpret_cast<const uint4*>(sw + (st * C::NW + w) * C::W_STAGE +
                                                           row * (C::BK / 4));
+        constexpr int CH = C::BK / 64;            // 16-byte chunks per packed row (2 or 4)
+        const int swz = (row / (8 / CH)) & (CH - 1);
 #pragma unroll
         for (int h = 0; h < C::BK / 128; ++h) {   // 128 weights -> 32 TMEM columns
-          const uint4 a = src[2 * h], b = src[2 * h + 1];
+          const uint4 a = src[(2 * h) ^ swz], b = src[(2 * h + 1) ^ swz];
           uint32_t e[32];
           expand_codes(a.x, e[0], e[1], e[2], e[3]);
           expand_codes(a.y, e[4], e[5], e[6], e[7]);
