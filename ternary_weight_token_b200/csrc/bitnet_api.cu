@@ -186,12 +186,15 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
   if (prelude != PRE_FWHT) {
     // register-resident rows: NT threads x VPT float4 must cover K / 4
-    const int grid = M < di.sms * 32 ? M : di.sms * 32;
+    const int grid = M < di.sms * 64 ? M : di.sms * 64;
+    // Small CTAs keep many rows in flight per SM (the kernel is bound by the
+    // latency of a row's loads and reductions, not by issue).
     const int k4 = K / 4;
     if (k4 <= 64 * 4) return launch_quant_reg<64, 4>(p, bf16, prelude, grid, st);
-    if (k4 <= 128 * 6) return launch_quant_reg<128, 6>(p, bf16, prelude, grid, st);
-    if (k4 <= 256 * 8) return launch_quant_reg<256, 8>(p, bf16, prelude, grid, st);
-    return launch_quant_reg<512, 8>(p, bf16, prelude, grid, st);   // K <= 16384
+    if (k4 <= 64 * 10) return launch_quant_reg<64, 10>(p, bf16, prelude, grid, st);
+    if (k4 <= 128 * 8) return launch_quant_reg<128, 8>(p, bf16, prelude, grid, st);
+    if (k4 <= 128 * 14) return launch_quant_reg<128, 14>(p, bf16, prelude, grid, st);
+    return launch_quant_reg<256, 16>(p, bf16, prelude, grid, st);   // K <= 16384
   }
   const int threads = K >= 2048 ? 256 : 128;
   const size_t smem = (size_t)K * sizeof(float);

@@ -342,7 +342,23 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = __int_as_float((int)v[j] - tok_rs[32 * c + j]);
           } else {
-            const bool resid = (p.flags & EPI_RESIDUAL) != 0;
+            // residual of this chunk: 32 independent loads issued back to back
+            // (one dtype branch for the whole chunk), before the dequant math
+            float r[32];
+            if (!C::SILU && (p.flags & EPI_RESIDUAL)) {
+              if (p.out_type == OUT_BF16) {
+                const __nv_bfloat16* rp = reinterpret_cast<const __nv_bfloat16*>(p.resid);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  r[j] = (n_ok && mc + j < p.M) ? __bfloat162float(rp[(size_t)(mc + j) * p.N + n])
+                                                : 0.0f;
+              } else {
+                const float* rp = reinterpret_cast<const float*>(p.resid);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                  r[j] = (n_ok && mc + j < p.M) ? rp[(size_t)(mc + j) * p.N + n] : 0.0f;
+              }
+            }
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const int t = 32 * c + j;
@@ -352,15 +368,19 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                 const double d = (double)yy;
                 yy = (float)(d / (1.0 + exp(-d)));
               }
-              if (resid) {
-                const int m = mc + j;
-                if (n_ok && m < p.M) {
-                  const size_t idx = (size_t)m * p.N + n;
-                  const float r = p.out_type == OUT_BF16
-                                      ? __bfloat162float(
-                                            reinterpret_cast<const __nv_bfloat16*>(p.resid)[idx])
-                                      : reinterpret_cast<const float*>(p.resid)[idx];
-                  yy = __fadd_rn(r, yy);
+              if (p.flags & EPI_RESIDUAL) {
+                if (C::SILU) {          // rare combination: plain per-element load
+                  const int m = mc + j;
+                  if (n_ok && m < p.M) {
+                    const size_t idx = (size_t)m * p.N + n;
+                    yy = __fadd_rn(p.out_type == OUT_BF16
+                                       ? __bfloat162float(
+                                             reinterpret_cast<const __nv_bfloat16*>(p.resid)[idx])
+                                       : reinterpret_cast<const float*>(p.resid)[idx],
+                                   yy);
+                  }
+                } else {
+                  yy = __fadd_rn(r[j], yy);
                 }
               }
               y[j] = yy;

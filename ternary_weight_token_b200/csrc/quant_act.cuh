@@ -74,6 +74,30 @@ __device__ __forceinline__ float block_max_f32(float v, float* red) {
   return r;
 }
 
+// Sum of a double and max of a float over the block in one pass (two syncs).
+__device__ __forceinline__ void block_sum_max(double& v, float& mx, double* red_d, float* red_f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v += __shfl_xor_sync(0xffffffffu, v, o);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    red_d[warp] = v;
+    red_f[warp] = mx;
+  }
+  __syncthreads();
+  double w = 0.0;
+  float f = 0.0f;
+  for (int i = 0; i < nw; ++i) {        // fixed order: the same sum in every thread
+    w += red_d[i];
+    f = fmaxf(f, red_f[i]);
+  }
+  __syncthreads();
+  v = w;
+  mx = f;
+}
+
 __device__ __forceinline__ int block_sum_i32(int v, int* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
@@ -261,18 +285,29 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
       return BF16 ? 8 * (tid + (i / 2) * NT) + 4 * (i & 1) : 4 * (tid + i * NT);
     };
     float r = 1.0f;
+    float amax = 0.0f;
     if (PRE == PRE_RMSNORM) {
       double ss = 0.0;
+      float xmax = 0.0f;
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         ss += (double)v[i].x * (double)v[i].x;
         ss += (double)v[i].y * (double)v[i].y;
         ss += (double)v[i].z * (double)v[i].z;
         ss += (double)v[i].w * (double)v[i].w;
+        xmax = fmaxf(fmaxf(xmax, fmaxf(fabsf(v[i].x), fabsf(v[i].y))),
+                     fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
       }
-      ss = block_sum_f64(ss, red_d);
+      if (p.gain == nullptr) {
+        // one pass: with r > 0 and no gain, max|fl(x r)| = fl(max|x| r) because
+        // rounding is monotone, so the row maximum needs no second reduction
+        block_sum_max(ss, xmax, red_d, red_f);
+      } else {
+        ss = block_sum_f64(ss, red_d);
+      }
       const float ms = (float)(ss / (double)K);
       r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+      if (p.gain == nullptr) amax = xmax == 0.0f ? 0.0f : __fmul_rn(xmax, r);   // 0 * inf stays 0
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
         const int k = kbase(i);
@@ -286,12 +321,13 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
         }
       }
     }
-    float amax = 0.0f;
+    if (PRE == PRE_NONE || p.gain != nullptr) {
 #pragma unroll
-    for (int i = 0; i < VPT; ++i)
-      amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v[i].x)), fmaxf(fabsf(v[i].y), fabsf(v[i].z))),
-                   fabsf(v[i].w));
-    amax = block_max_f32(amax, red_f);
+      for (int i = 0; i < VPT; ++i)
+        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v[i].x)), fmaxf(fabsf(v[i].y), fabsf(v[i].z))),
+                     fabsf(v[i].w));
+      amax = block_max_f32(amax, red_f);
+    }
     float s = __fdiv_rn(127.0f, amax);
     const bool zero_row = (amax == 0.0f) || isinf(s);
     if (zero_row) s = 1.0f;

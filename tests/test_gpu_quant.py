@@ -131,3 +131,15 @@ def test_pack_is_deterministic():
     b = gpu_pack(W)
     assert a[1] == b[1]
     np.testing.assert_array_equal(a[0], b[0])
+
+
+def test_quant_rmsnorm_zero_row_with_zero_eps():
+    """mean square 0 and eps 0 give r = inf; the all-zero row must still come
+    out as q = 0, s = 1 (the oracle's 0 * inf products never exceed 0)."""
+    X = _acts(6, 2560, seed=77)
+    X[2] = 0.0
+    for gain in (None, np.full(2560, 1.5, np.float32)):
+        q, s, rs = gpu_quant(X, bn.BITNET_PRELUDE_RMSNORM, gain=gain, eps=0.0)
+        qo, so, rso = oracle.quant_act(X, oracle.PRELUDE_RMSNORM, gain=gain, eps=0.0)
+        assert not q[2].any() and s[2] == 1.0 and rs[2] == 0
+        assert_codes_chain(q, qo, "rmsnorm eps 0")
