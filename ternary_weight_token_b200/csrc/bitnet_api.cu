@@ -162,8 +162,12 @@ int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1
 }
 
 // ------------------------------------------------------------- launchers
+// Register-resident rows, NT threads x VPT 16-byte chunks, one CTA per row
+// (grid-stride over at most sms * 64 CTAs).
 template <int NT, int VPT>
-int launch_quant_reg(const QuantParams& p, bool bf16, int prelude, int grid, cudaStream_t st) {
+int launch_quant_rows(const QuantParams& p, bool bf16, int prelude, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
   void (*kern)(QuantParams) = nullptr;
   if (prelude == PRE_RMSNORM)
     kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_RMSNORM, true>
@@ -171,6 +175,7 @@ int launch_quant_reg(const QuantParams& p, bool bf16, int prelude, int grid, cud
   else
     kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_NONE, true>
                 : quant_act_reg_kernel<NT, VPT, PRE_NONE, false>;
+  const int grid = p.M < di.sms * 64 ? p.M : di.sms * 64;
   kern<<<grid, NT, 0, st>>>(p);
   BN_CHECK_CUDA(cudaGetLastError());
   return BITNET_OK;
@@ -185,16 +190,14 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   p.fwht_c = (float)(1.0 / std::sqrt((double)K));
   p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
   if (prelude != PRE_FWHT) {
-    // register-resident rows: NT threads x VPT float4 must cover K / 4
-    const int grid = M < di.sms * 64 ? M : di.sms * 64;
-    // Small CTAs keep many rows in flight per SM (the kernel is bound by the
-    // latency of a row's loads and reductions, not by issue).
+    // NT threads x VPT 16-byte chunks must cover the row (K / 4 fp32 chunks,
+    // K / 8 bf16 units of two chunks)
     const int k4 = K / 4;
-    if (k4 <= 64 * 4) return launch_quant_reg<64, 4>(p, bf16, prelude, grid, st);
-    if (k4 <= 64 * 10) return launch_quant_reg<64, 10>(p, bf16, prelude, grid, st);
-    if (k4 <= 128 * 8) return launch_quant_reg<128, 8>(p, bf16, prelude, grid, st);
-    if (k4 <= 128 * 14) return launch_quant_reg<128, 14>(p, bf16, prelude, grid, st);
-    return launch_quant_reg<256, 16>(p, bf16, prelude, grid, st);   // K <= 16384
+    if (k4 <= 64 * 4) return launch_quant_rows<64, 4>(p, bf16, prelude, st);
+    if (k4 <= 64 * 10) return launch_quant_rows<64, 10>(p, bf16, prelude, st);
+    if (k4 <= 128 * 8) return launch_quant_rows<128, 8>(p, bf16, prelude, st);
+    if (k4 <= 128 * 14) return launch_quant_rows<128, 14>(p, bf16, prelude, st);
+    return launch_quant_rows<256, 16>(p, bf16, prelude, st);   // K <= 16384
   }
   const int threads = K >= 2048 ? 256 : 128;
   const size_t smem = (size_t)K * sizeof(float);

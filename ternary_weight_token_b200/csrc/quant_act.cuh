@@ -10,12 +10,14 @@
 // Hadamard prelude is the H-BitLinear input transform ("bitnetv2-model"
 // README, "Special Features").
 //
-// One CTA per token row (grid-stride).  The row is staged once in shared
-// memory as fp32 with 128-bit loads; the RMS mean square is reduced in fp64;
-// the FWHT runs its butterfly stages in shared memory in the fixed order
-// h = 1, 2, 4, ...; the codes are written with 32-bit stores.  Every fp32
-// operation that decides a code is an explicit round-to-nearest intrinsic, so
-// no FMA contraction can change a result.
+// One CTA per token row (grid-stride).  The NONE and RMSNORM preludes keep
+// the row in registers (quant_act_reg_kernel: every 16-byte load in flight
+// before the first reduction, one exact fp64 FMA per element for the mean
+// square, codes rounded by one fp32 add and packed by byte permutes).  The
+// FWHT prelude stages the row in shared memory as fp32 and runs its butterfly
+// stages there in the fixed order h = 1, 2, 4, ... (quant_act_kernel).  Every
+// fp32 operation that decides a code is an explicit round-to-nearest
+// intrinsic, so no FMA contraction can change a result.
 #pragma once
 
 #include "common.cuh"
@@ -74,30 +76,6 @@ __device__ __forceinline__ float block_max_f32(float v, float* red) {
   return r;
 }
 
-// Sum of a double and max of a float over the block in one pass (two syncs).
-__device__ __forceinline__ void block_sum_max(double& v, float& mx, double* red_d, float* red_f) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    v += __shfl_xor_sync(0xffffffffu, v, o);
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  if (lane == 0) {
-    red_d[warp] = v;
-    red_f[warp] = mx;
-  }
-  __syncthreads();
-  double w = 0.0;
-  float f = 0.0f;
-  for (int i = 0; i < nw; ++i) {        // fixed order: the same sum in every thread
-    w += red_d[i];
-    f = fmaxf(f, red_f[i]);
-  }
-  __syncthreads();
-  v = w;
-  mx = f;
-}
-
 __device__ __forceinline__ int block_sum_i32(int v, int* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
@@ -123,6 +101,21 @@ __device__ __forceinline__ float bf16_bits_to_f32(uint32_t bits16) {
 __device__ __forceinline__ int quant_code(float xh, float s) {
   int q = __float2int_rn(__fmul_rn(xh, s));   // round half to even
   return min(127, max(-128, q));
+}
+
+// Codes of four scaled values y = fl(xh * s), packed little-endian.  For
+// |y| < 2^22 the fp32 sum 1.5 * 2^23 + y lies in a binade of spacing 1, so its
+// round-to-nearest-even is exactly rint(y), and the low byte of its bit
+// pattern is rint(y) mod 256.  |y| <= 127 (within rounding) holds for every
+// element of a row because s = fl(127 / amax) and |xh| <= amax, so the clamp
+// to [-128, 127] of the definition never binds and is not applied.
+__device__ __forceinline__ uint32_t pack_codes4(float y0, float y1, float y2, float y3) {
+  const float kMagic = 12582912.0f;
+  const uint32_t a = __float_as_uint(__fadd_rn(y0, kMagic));
+  const uint32_t b = __float_as_uint(__fadd_rn(y1, kMagic));
+  const uint32_t c = __float_as_uint(__fadd_rn(y2, kMagic));
+  const uint32_t d = __float_as_uint(__fadd_rn(y3, kMagic));
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
 // Prelude value of element k (row[] holds x for NONE / RMSNORM and the
@@ -243,117 +236,238 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
   }
 }
 
-// Register-resident variant for the NONE and RMSNORM preludes: one CTA per
-// token row, NT threads, each holding up to VPT float4 of the row in
-// registers.  Every 16-byte load of the row is in flight before the first
-// reduction, so the kernel streams at HBM bandwidth; the row is read once.
+// ---------------------------------------------------------------------------
+// Register-resident rows (NONE and RMSNORM preludes).
+//
+// Thread t of an NT-thread CTA holds VPT float4 of the row: chunk i is the
+// 16-byte unit t + i * NT of an fp32 row, or for a bf16 row, chunks 2j and 2j+1
+// are the two halves of the 8-value unit t + j * NT.  Chunks past the end of
+// the row hold zeros.  Per element the row costs one exact fp64 FMA of x^2
+// (the square of a 24-bit significand is exact in fp64), one |x| max, the
+// fp32 products of the definition, one add that rounds, and a quarter of a
+// byte permute, dp4a and store each.
+
+template <int NT, int VPT, bool BF16>
+__device__ __forceinline__ bool chunk_valid(int i, int K) {
+  return BF16 ? (int)threadIdx.x + (i / 2) * NT < K / 8 : (int)threadIdx.x + i * NT < K / 4;
+}
+
+template <int NT, int VPT, bool BF16>
+__device__ __forceinline__ int chunk_elem(int i) {
+  return BF16 ? 8 * ((int)threadIdx.x + (i / 2) * NT) + 4 * (i & 1)
+              : 4 * ((int)threadIdx.x + i * NT);
+}
+
+// One barrier: warp partials of an fp64 sum and an fp32 max, combined by every
+// thread in the same fixed order.  The caller alternates between two partial
+// buffers on consecutive rows (and has another barrier per row), so a row's
+// partials are never overwritten while a thread still reads them.
+__device__ __forceinline__ void block_sum_max_1(double& v, float& mx, double* red_d,
+                                                float* red_f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    v += __shfl_xor_sync(0xffffffffu, v, o);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (lane == 0) {
+    red_d[warp] = v;
+    red_f[warp] = mx;
+  }
+  __syncthreads();
+  double w = 0.0;
+  float f = 0.0f;
+  for (int i = 0; i < nw; ++i) {
+    w += red_d[i];
+    f = fmaxf(f, red_f[i]);
+  }
+  v = w;
+  mx = f;
+}
+
+__device__ __forceinline__ float block_max_1(float mx, float* red_f) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red_f[warp] = mx;
+  __syncthreads();
+  float f = 0.0f;
+  for (int i = 0; i < nw; ++i) f = fmaxf(f, red_f[i]);
+  return f;
+}
+
+__device__ __forceinline__ double block_sum_1(double v, double* red_d) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red_d[warp] = v;
+  __syncthreads();
+  double w = 0.0;
+  for (int i = 0; i < nw; ++i) w += red_d[i];
+  return w;
+}
+
+// Reduction scratch of the register kernels: two alternating buffers of warp
+// partials (fp64 sum, fp32 max, fp32 max of a second reduction) and the warp
+// partials of the code sum.
+struct RowRed {
+  double d[2][32];
+  float f[2][32];
+  float g[2][32];
+  int rs[32];
+};
+
+// Statistics, scale and codes of row m held in v[]; leaves the warp partials
+// of the code sum in red.rs (lane 0 of each warp) for the caller to add up
+// after its next barrier.
 template <int NT, int VPT, int PRE, bool BF16>
-__global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
-  static_assert(PRE == PRE_NONE || PRE == PRE_RMSNORM, "FWHT uses the shared-memory kernel");
-  static_assert(!BF16 || VPT % 2 == 0, "bf16 rows load 8 values per 16 bytes");
-  __shared__ double red_d[33];
-  __shared__ float red_f[33];
-  __shared__ int red_i[33];
-  const int K = p.K, K4 = p.K / 4;
-  const int tid = threadIdx.x;
-  for (int m = blockIdx.x; m < p.M; m += gridDim.x) {
-    float4 v[VPT];
-    if (BF16) {
-      const uint4* src = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const __nv_bfloat16*>(p.X) + (size_t)m * K);
+__device__ __forceinline__ void quant_row(const QuantParams& p, int m, float4 (&v)[VPT],
+                                          RowRed& red, int par) {
+  const int K = p.K;
+  float r = 1.0f, amax = 0.0f;
+  if (PRE == PRE_RMSNORM) {
+    double s0 = 0.0, s1 = 0.0;
+    float xmax = 0.0f;
 #pragma unroll
-      for (int i = 0; i < VPT / 2; ++i) {
-        const int idx = tid + i * NT;            // 8-value unit
-        uint4 u = make_uint4(0u, 0u, 0u, 0u);
-        if (idx < K / 8) u = src[idx];
-        v[2 * i] = make_float4(bf16_bits_to_f32(u.x & 0xffffu), bf16_bits_to_f32(u.x >> 16),
-                               bf16_bits_to_f32(u.y & 0xffffu), bf16_bits_to_f32(u.y >> 16));
-        v[2 * i + 1] = make_float4(bf16_bits_to_f32(u.z & 0xffffu), bf16_bits_to_f32(u.z >> 16),
-                                   bf16_bits_to_f32(u.w & 0xffffu), bf16_bits_to_f32(u.w >> 16));
-      }
-    } else {
-      const float4* src = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p.X) +
-                                                          (size_t)m * K);
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const int idx = tid + i * NT;
-        v[i] = idx < K4 ? src[idx] : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+    for (int i = 0; i < VPT; ++i) {
+      s0 = fma((double)v[i].x, (double)v[i].x, s0);
+      s1 = fma((double)v[i].y, (double)v[i].y, s1);
+      s0 = fma((double)v[i].z, (double)v[i].z, s0);
+      s1 = fma((double)v[i].w, (double)v[i].w, s1);
+      xmax = fmaxf(xmax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                               fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
     }
-    // element index of v[i].x: bf16 rows pair float4s inside one 8-value unit
-    auto kbase = [&](int i) -> int {
-      return BF16 ? 8 * (tid + (i / 2) * NT) + 4 * (i & 1) : 4 * (tid + i * NT);
-    };
-    float r = 1.0f;
-    float amax = 0.0f;
-    if (PRE == PRE_RMSNORM) {
-      double ss = 0.0;
-      float xmax = 0.0f;
+    double ss = s0 + s1;
+    block_sum_max_1(ss, xmax, red.d[par], red.f[par]);
+    const float ms = (float)(ss / (double)K);
+    r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+    if (p.gain == nullptr) {
+      // with r > 0 and no gain, max|fl(x r)| = fl(max|x| r) (rounding is
+      // monotone), so the row maximum needs no second reduction; 0 * inf -> 0
+      amax = xmax == 0.0f ? 0.0f : __fmul_rn(xmax, r);
+    } else {
 #pragma unroll
       for (int i = 0; i < VPT; ++i) {
-        ss += (double)v[i].x * (double)v[i].x;
-        ss += (double)v[i].y * (double)v[i].y;
-        ss += (double)v[i].z * (double)v[i].z;
-        ss += (double)v[i].w * (double)v[i].w;
-        xmax = fmaxf(fmaxf(xmax, fmaxf(fabsf(v[i].x), fabsf(v[i].y))),
-                     fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
-      }
-      if (p.gain == nullptr) {
-        // one pass: with r > 0 and no gain, max|fl(x r)| = fl(max|x| r) because
-        // rounding is monotone, so the row maximum needs no second reduction
-        block_sum_max(ss, xmax, red_d, red_f);
-      } else {
-        ss = block_sum_f64(ss, red_d);
-      }
-      const float ms = (float)(ss / (double)K);
-      r = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
-      if (p.gain == nullptr) amax = xmax == 0.0f ? 0.0f : __fmul_rn(xmax, r);   // 0 * inf stays 0
-#pragma unroll
-      for (int i = 0; i < VPT; ++i) {
-        const int k = kbase(i);
-        if (k < K) {
-          float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
-          if (p.gain) g = __ldg(reinterpret_cast<const float4*>(p.gain + k));
+        if (chunk_valid<NT, VPT, BF16>(i, K)) {
+          const float4 g = __ldg(reinterpret_cast<const float4*>(p.gain + chunk_elem<NT, VPT, BF16>(i)));
           v[i].x = __fmul_rn(__fmul_rn(v[i].x, r), g.x);
           v[i].y = __fmul_rn(__fmul_rn(v[i].y, r), g.y);
           v[i].z = __fmul_rn(__fmul_rn(v[i].z, r), g.z);
           v[i].w = __fmul_rn(__fmul_rn(v[i].w, r), g.w);
+          amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                                   fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
         }
       }
+      amax = block_max_1(amax, red.g[par]);
     }
-    if (PRE == PRE_NONE || p.gain != nullptr) {
+  } else {
 #pragma unroll
-      for (int i = 0; i < VPT; ++i)
-        amax = fmaxf(fmaxf(fmaxf(amax, fabsf(v[i].x)), fmaxf(fabsf(v[i].y), fabsf(v[i].z))),
-                     fabsf(v[i].w));
-      amax = block_max_f32(amax, red_f);
+    for (int i = 0; i < VPT; ++i)
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                               fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+    amax = block_max_1(amax, red.f[par]);
+  }
+  float s = __fdiv_rn(127.0f, amax);
+  const bool zero_row = (amax == 0.0f) || isinf(s);
+  if (zero_row) s = 1.0f;
+  if (threadIdx.x == 0) p.scale[m] = s;
+  // the RMS factor is applied here when no gain was (same two roundings)
+  const bool fold_r = PRE == PRE_RMSNORM && p.gain == nullptr;
+  int rsum = 0;
+  uint8_t* dst = reinterpret_cast<uint8_t*>(p.Xq) + (size_t)m * K;
+  auto codes = [&](const float4& x) -> uint32_t {
+    if (fold_r)
+      return pack_codes4(__fmul_rn(__fmul_rn(x.x, r), s), __fmul_rn(__fmul_rn(x.y, r), s),
+                         __fmul_rn(__fmul_rn(x.z, r), s), __fmul_rn(__fmul_rn(x.w, r), s));
+    return pack_codes4(__fmul_rn(x.x, s), __fmul_rn(x.y, s), __fmul_rn(x.z, s),
+                       __fmul_rn(x.w, s));
+  };
+  if (BF16) {
+#pragma unroll
+    for (int j = 0; j < VPT / 2; ++j) {
+      if (chunk_valid<NT, VPT, BF16>(2 * j, K)) {
+        uint2 w = make_uint2(0u, 0u);
+        if (!zero_row) {
+          w.x = codes(v[2 * j]);
+          w.y = codes(v[2 * j + 1]);
+          rsum = __dp4a((int)w.x, 0x01010101, rsum);
+          rsum = __dp4a((int)w.y, 0x01010101, rsum);
+        }
+        *reinterpret_cast<uint2*>(dst + 8 * ((int)threadIdx.x + j * NT)) = w;
+      }
     }
-    float s = __fdiv_rn(127.0f, amax);
-    const bool zero_row = (amax == 0.0f) || isinf(s);
-    if (zero_row) s = 1.0f;
-    int rsum = 0;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(p.Xq + (size_t)m * K);
+  } else {
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int k = kbase(i);
-      if (k < K) {
-        int q0 = 0, q1 = 0, q2 = 0, q3 = 0;
+      if (chunk_valid<NT, VPT, BF16>(i, K)) {
+        uint32_t w = 0u;
         if (!zero_row) {
-          q0 = quant_code(v[i].x, s);
-          q1 = quant_code(v[i].y, s);
-          q2 = quant_code(v[i].z, s);
-          q3 = quant_code(v[i].w, s);
+          w = codes(v[i]);
+          rsum = __dp4a((int)w, 0x01010101, rsum);
         }
-        rsum += q0 + q1 + q2 + q3;
-        dst[k / 4] = (uint32_t)(q0 & 0xff) | ((uint32_t)(q1 & 0xff) << 8) |
-                     ((uint32_t)(q2 & 0xff) << 16) | ((uint32_t)(q3 & 0xff) << 24);
+        reinterpret_cast<uint32_t*>(dst)[(int)threadIdx.x + i * NT] = w;
       }
     }
-    if (p.rowsum != nullptr) rsum = block_sum_i32(rsum, red_i);
-    if (tid == 0) {
-      p.scale[m] = s;
-      if (p.rowsum != nullptr) p.rowsum[m] = rsum;
+  }
+  rsum = __reduce_add_sync(0xffffffffu, rsum);
+  if ((threadIdx.x & 31) == 0) red.rs[threadIdx.x >> 5] = rsum;
+}
+
+// Sum of the warp partials of the code sum of row m (thread 0, after a
+// barrier that follows their writes).
+__device__ __forceinline__ void finish_rowsum(const QuantParams& p, int m, const RowRed& red) {
+  if (threadIdx.x == 0 && p.rowsum != nullptr) {
+    int t = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) t += red.rs[w];
+    p.rowsum[m] = t;
+  }
+}
+
+template <int NT, int VPT, bool BF16>
+__device__ __forceinline__ void unpack_row(const uint4 (&u)[BF16 ? VPT / 2 : VPT],
+                                           float4 (&v)[VPT]) {
+  if (BF16) {
+#pragma unroll
+    for (int j = 0; j < VPT / 2; ++j) {
+      v[2 * j] = make_float4(__uint_as_float(u[j].x << 16), __uint_as_float(u[j].x & 0xffff0000u),
+                             __uint_as_float(u[j].y << 16), __uint_as_float(u[j].y & 0xffff0000u));
+      v[2 * j + 1] =
+          make_float4(__uint_as_float(u[j].z << 16), __uint_as_float(u[j].z & 0xffff0000u),
+                      __uint_as_float(u[j].w << 16), __uint_as_float(u[j].w & 0xffff0000u));
     }
+  } else {
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) v[i] = make_float4(__uint_as_float(u[i].x), __uint_as_float(u[i].y),
+                                                    __uint_as_float(u[i].z), __uint_as_float(u[i].w));
+  }
+}
+
+// One CTA per row (grid-stride): every 16-byte load of the row is issued
+// before the first reduction.
+template <int NT, int VPT, int PRE, bool BF16>
+__global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
+  static_assert(PRE == PRE_NONE || PRE == PRE_RMSNORM, "FWHT uses the shared-memory kernel");
+  static_assert(!BF16 || VPT % 2 == 0, "bf16 rows load 8 values per 16 bytes");
+  constexpr int NU = BF16 ? VPT / 2 : VPT;
+  __shared__ RowRed red;
+  const int K = p.K;
+  const int units = BF16 ? K / 8 : K / 4;
+  const int row_bytes = K * (BF16 ? 2 : 4);
+  int par = 0;
+  for (int m = blockIdx.x; m < p.M; m += gridDim.x, par ^= 1) {
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.X) +
+                                                      (size_t)m * row_bytes);
+    uint4 u[NU];
+#pragma unroll
+    for (int j = 0; j < NU; ++j) {
+      const int idx = (int)threadIdx.x + j * NT;
+      u[j] = idx < units ? ld_stream_v4(src + idx) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float4 v[VPT];
+    unpack_row<NT, VPT, BF16>(u, v);
+    quant_row<NT, VPT, PRE, BF16>(p, m, v, red, par);
+    __syncthreads();
+    finish_rowsum(p, m, red);
   }
 }
 
