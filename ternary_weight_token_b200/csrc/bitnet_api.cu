@@ -269,8 +269,12 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
     const CUtensorMapDataType dt = lp.out_type == OUT_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : lp.out_type == OUT_I32 ? CU_TENSOR_MAP_DATA_TYPE_INT32
                                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    // the bf16 fragment epilogue (no GLU) stages 64-byte rows with the
+    // 64-byte swizzle, so its transposing stores are bank-conflict free
+    const bool frag = !C::GLU && lp.out_type == OUT_BF16;
     if (int rc = tensor_map_2d(my, lp.Y, dt, (uint64_t)lp.N, (uint64_t)lp.M,
-                               (uint64_t)lp.N * esz, 32, 32, CU_TENSOR_MAP_SWIZZLE_NONE))
+                               (uint64_t)lp.N * esz, 32, 32,
+                               frag ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
       return rc;
   }
   TcParams p;

@@ -237,6 +237,31 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
+// 16 lanes x 8 columns per repetition, 4 repetitions along the columns.
+// Thread t receives, for repetition j, r[4j + 0, 1] = lane t/4, columns
+// 8j + 2(t%4) + {0, 1} and r[4j + 2, 3] = lane 8 + t/4, the same columns (the
+// fragment layout of an m16n8 accumulator, which stmatrix stores).
+__device__ __forceinline__ void tmem_ld_16x256b_x4(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x4.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+// Four 8x8 matrices of 16-bit values, stored transposed: register i of thread
+// t holds elements (t/4, 2(t%4) + {0, 1}) of matrix i, and thread 8i + r gives
+// the shared-memory address of row r of the stored (transposed) matrix i.
+__device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, uint32_t r1,
+                                                  uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(
+                   addr),
+               "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -254,6 +279,19 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// Zero 32 lanes x 32 columns of TMEM (four 8-column stores of one zero
+// register block, so no 32-register array stays live around the call).
+__device__ __forceinline__ void tmem_zero_32x32b_x32(uint32_t taddr) {
+  const uint32_t z = 0u;
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+            taddr + 8u * k),
+        "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z), "r"(z)
+        : "memory");
 }
 
 __device__ __forceinline__ void tmem_st_wait() {

@@ -69,7 +69,7 @@ struct TcConfig {
   static constexpr int OFF_W = OFF_X + STAGES * X_STAGE;
   static constexpr int OFF_OUT = OFF_W + STAGES * NW * W_STAGE;  // 4 warps x 2 buffers
   static constexpr int OFF_BAR = OFF_OUT + 4 * 2 * STAGE_OUT_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 5;
+  static constexpr int NUM_BARS = 3 * STAGES + 7;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
@@ -100,10 +100,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_y, TcParams p) {
   extern __shared__ uint8_t tc_smem_raw[];
-  // per-token dequant factors (fp32 head, tail) and code sums, one copy per
-  // epilogue warp; static so they never alias the output staging buffers
-  __shared__ float2 s_tok_f[4][C::NW * C::BN];
-  __shared__ int s_tok_rs[4][C::BN];
+  // per-token dequant factors (fp32 head, tail) and code sums of a tile,
+  // computed once by the four epilogue warps; two buffers alternate between
+  // consecutive tiles.  Static so they never alias the output staging buffers.
+  __shared__ __align__(16) float2 s_tok_f[2][C::NW * C::BN];
+  __shared__ __align__(16) int s_tok_rs[2][C::BN];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -116,6 +117,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* accfull = bars + 3 * C::STAGES;    // accumulator ready      (tcgen05.commit)
   uint64_t* accempty = accfull + 2;            // accumulator drained    (4 epilogue warps)
   uint64_t* drain = accempty + 2;              // teardown drain
+  uint64_t* tokbar = drain + 1;                // tile's token factors written (4 warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -132,6 +134,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(&accempty[b], 4);            // four epilogue warps (zeroed buffer)
     }
     mbar_init(drain, 2);
+    mbar_init(&tokbar[0], 4);
+    mbar_init(&tokbar[1], 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -263,18 +267,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   } else if (warp >= C::EPI_WARP0) {
     // --------------------------------------------------------- epilogue
     const int q = warp & 3;
-    float2* tok_f = s_tok_f[q];                  // [NW][BN]
-    int* tok_rs = s_tok_rs[q];
     const float g0 = __ldg(p.gamma0);
     const float g1 = C::GLU ? __ldg(p.gamma1) : 0.0f;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     const int esz = out_elem_bytes(p.out_type);
     const uint32_t out_base = smem_u32(smem + C::OFF_OUT + q * 2 * C::STAGE_OUT_BYTES);
-    uint32_t zero[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) zero[j] = 0u;
+    // bf16 output through the TMA store: fragment epilogue (16x256b loads,
+    // transposing stmatrix into a 64-byte-swizzled staging tile)
+    const bool frag_path = !C::GLU && p.tma_out && p.out_type == OUT_BF16;
     // both accumulator buffers start at zero: every MMA accumulates
-    for (int col = 0; col < 2 * C::ACC_COLS; col += 32) tmem_st_32x32b_x32(lane_base + col, zero);
+    for (int col = 0; col < 2 * C::ACC_COLS; col += 32) tmem_zero_32x32b_x32(lane_base + col);
     tmem_st_wait();
     tc_fence_before();
     __syncwarp();
@@ -288,8 +290,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int m0 = tm * C::BN;
       const int nq0 = tn * C::BM + 32 * q;       // first weight row of this warp
       const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
-      __syncwarp();
-      for (int j = lane; j < C::BN; j += 32) {
+      float2* tok_f = s_tok_f[ab];               // [NW][BN]
+      int* tok_rs = s_tok_rs[ab];
+      // This buffer was last read for tile tcount - 2; every warp has since
+      // arrived on the other buffer's barrier, so no warp still reads it.
+      for (int j = 32 * q + lane; j < C::BN; j += 128) {
         const int m = m0 + j;
         float2 f0 = make_float2(0.0f, 0.0f), f1 = make_float2(0.0f, 0.0f);
         int rs = 0;
@@ -304,6 +309,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         tok_rs[j] = rs;
       }
       __syncwarp();
+      if (lane == 0) mbar_arrive(&tokbar[ab]);
+      if (!mbar_wait(&tokbar[ab], aph, abort_flag)) break;
       if (!mbar_wait(&accfull[ab], aph, abort_flag)) break;
       tc_fence_after();
       const int n = nq0 + lane;
@@ -312,9 +319,84 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       for (int c = 0; c < C::BN / 32; ++c, ++chunk_count) {
         const int mc = m0 + 32 * c;              // first token of this chunk
         if (mc >= p.M) {                         // past the last token: only re-zero
-          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
-          if (C::GLU) tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, zero);
+          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
+          if (C::GLU) tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c);
           continue;
+        }
+        if constexpr (!C::GLU) {
+          if (frag_path) {
+            // v[16h + 4j + k]: weight row nq0 + 16h + 8(k / 2) + lane / 4,
+            // token mc + 8j + 2(lane % 4) + k % 2
+            uint32_t v[32];
+            tmem_ld_16x256b_x4(lane_base + ab * C::ACC_COLS + 32u * c, v);
+            tmem_ld_16x256b_x4(lane_base + (16u << 16) + ab * C::ACC_COLS + 32u * c, v + 16);
+            const int tq = 2 * (lane & 3);       // this thread's even token offset
+            // residual (bf16) of the same elements, two per register
+            uint32_t rpk[16];
+            if (p.flags & EPI_RESIDUAL) {
+              const uint16_t* rp = reinterpret_cast<const uint16_t*>(p.resid);
+#pragma unroll
+              for (int i = 0; i < 32; i += 2) {
+                const int nn = nq0 + 16 * (i >> 4) + 8 * ((i >> 1) & 1) + (lane >> 2);
+                const int mm = mc + 8 * ((i >> 2) & 3) + tq;
+                const bool ok = nn < p.N;
+                const uint32_t lo = (ok && mm < p.M) ? rp[(size_t)mm * p.N + nn] : 0u;
+                const uint32_t hi = (ok && mm + 1 < p.M) ? rp[(size_t)(mm + 1) * p.N + nn] : 0u;
+                rpk[i >> 1] = lo | (hi << 16);
+              }
+            }
+            tmem_ld_wait();
+            tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
+            // staging tile: 32 token rows of 64 bytes (32 weight rows, bf16),
+            // 16-byte chunk k of row m at chunk k ^ ((m / 2) % 4) (64-byte swizzle)
+            const uint32_t buf = out_base + (chunk_count & 1u) * C::STAGE_OUT_BYTES;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+            const int mi = lane >> 3, rr8 = lane & 7;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {        // weight rows nq0 + 16h .. + 15
+              uint32_t pk[8];                    // bf16x2 of matrix (j, s): pk[2j + s]
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int t = 32 * c + 8 * j + tq;
+                const float4 ff = *reinterpret_cast<const float4*>(&tok_f[t]);
+                const int2 rr = *reinterpret_cast<const int2*>(&tok_rs[t]);
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                  const int i = 16 * h + 4 * j + 2 * s2;
+                  float y0 = dequant_dw((int)v[i] - rr.x, ff.x, ff.y);
+                  float y1 = dequant_dw((int)v[i + 1] - rr.y, ff.z, ff.w);
+                  if (C::SILU) {
+                    const double d0 = (double)y0, d1 = (double)y1;
+                    y0 = (float)(d0 / (1.0 + exp(-d0)));
+                    y1 = (float)(d1 / (1.0 + exp(-d1)));
+                  }
+                  if (p.flags & EPI_RESIDUAL) {
+                    y0 = __fadd_rn(__uint_as_float(rpk[i >> 1] << 16), y0);
+                    y1 = __fadd_rn(__uint_as_float(rpk[i >> 1] & 0xffff0000u), y1);
+                  }
+                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
+                  pk[2 * j + s2] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+              }
+#pragma unroll
+              for (int jp = 0; jp < 2; ++jp) {
+                // matrix mi of this store: token block j = 2 jp + mi / 2,
+                // weight-row block 8 (mi % 2) of half h
+                const int row = 8 * (2 * jp + (mi >> 1)) + rr8;
+                const int chunk = (2 * h + (mi & 1)) ^ ((row >> 1) & 3);
+                stmatrix_x4_trans(buf + (uint32_t)(row * 64 + chunk * 16), pk[4 * jp + 0],
+                                  pk[4 * jp + 1], pk[4 * jp + 2], pk[4 * jp + 3]);
+              }
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0 && nq0 < p.N) {
+              tma_store_2d(&tm_y, smem + (buf - smem_u32(smem)), nq0, mc);
+              bulk_commit_group();
+            }
+            continue;
+          }
         }
         uint32_t v[32];
         float y[32];
@@ -323,8 +405,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           uint32_t u[32];
           tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, u);
           tmem_ld_wait();
-          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
-          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, zero);
+          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
+          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c);
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = 32 * c + j;
@@ -337,7 +419,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           }
         } else {
           tmem_ld_wait();
-          tmem_st_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, zero);
+          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
           if (p.out_type == OUT_I32) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) y[j] = __int_as_float((int)v[j] - tok_rs[32 * c + j]);
