@@ -42,6 +42,11 @@
  *              bitnet_check_device_error() reads.
  *   Inputs     Inputs must be finite; with NaN or Inf in an input the codes
  *              are unspecified.
+ *   Launch     The quantiser and the prefill GEMM (M > 16) are launched with
+ *              programmatic dependent launch: their CTAs may do on-chip setup
+ *              while the preceding work on the stream finishes, and touch no
+ *              global memory before that work has completed, so stream order
+ *              is preserved whatever precedes them.
  *
  * Packed ternary layout (the pages fix only "four to a byte"; this layout is
  * this library's convention)
@@ -92,7 +97,8 @@ extern "C" {
  * and stream its packed weights early; activation codes, scales, code sums,
  * gamma, residual and Y are touched only after that work has completed.  Set
  * it only when the preceding work does not write the packed weights, e.g. in
- * a decode loop over static weights.  Ignored for M > 16. */
+ * a decode loop over static weights.  Ignored for M > 16 (the prefill GEMM
+ * always uses the dependent launch, without early weight reads). */
 #define BITNET_LAUNCH_PDL     0x100
 
 /* ----------------------------------------------------------- FFN variants */

@@ -162,6 +162,26 @@ int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1
 }
 
 // ------------------------------------------------------------- launchers
+
+// Launch with programmatic dependent launch: the kernel may begin its on-chip
+// setup while the preceding grid on the stream finishes; every kernel
+// launched this way executes griddepcontrol.wait before touching global memory.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, args...));
+  return BITNET_OK;
+}
 // Register-resident rows, NT threads x VPT 16-byte chunks, one CTA per row
 // (grid-stride over at most sms * 64 CTAs).
 template <int NT, int VPT>
@@ -176,9 +196,7 @@ int launch_quant_rows(const QuantParams& p, bool bf16, int prelude, cudaStream_t
     kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_NONE, true>
                 : quant_act_reg_kernel<NT, VPT, PRE_NONE, false>;
   const int grid = p.M < di.sms * 64 ? p.M : di.sms * 64;
-  kern<<<grid, NT, 0, st>>>(p);
-  BN_CHECK_CUDA(cudaGetLastError());
-  return BITNET_OK;
+  return launch_pdl(kern, dim3(grid), dim3(NT), 0, st, p);
 }
 
 int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const float* gain,
@@ -204,9 +222,7 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   const int grid = M < di.sms * 16 ? M : di.sms * 16;
   void (*kern)(QuantParams) = bf16 ? quant_act_kernel<PRE_FWHT, true> : quant_act_kernel<PRE_FWHT, false>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<grid, threads, smem, st>>>(p);
-  BN_CHECK_CUDA(cudaGetLastError());
-  return BITNET_OK;
+  return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, p);
 }
 
 int launch_gemv(const LinearParams& p, cudaStream_t st) {
@@ -295,9 +311,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   auto kern = gemm_tc_kernel<C>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
-  kern<<<grid, C::THREADS, smem, st>>>(mx, mw0, mw1, my, p);
-  BN_CHECK_CUDA(cudaGetLastError());
-  return BITNET_OK;
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mw0, mw1, my, p);
 }
 
 using TcPlain = TcConfig<128, 256, 4, false>;

@@ -303,6 +303,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch
+// Wait until the grids this one depends on have completed and their memory
+// is visible (returns at once for a launch without the PDL attribute).
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next grid on the stream start launching (its CTAs then wait in
+// grid_dependency_wait until this grid has completed).
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // --------------------------------------------------------------- misc ALU
 // Four unsigned bytes of `a` times four signed bytes of `b`, summed into c.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {

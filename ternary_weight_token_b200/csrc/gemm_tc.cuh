@@ -152,6 +152,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // Launched with programmatic dependent launch: the setup above touches no
+  // global memory; everything below runs after the preceding grid completed.
+  grid_launch_dependents();
+  grid_dependency_wait();
   const uint32_t tbase = *tmem_slot;
   const uint32_t a_col0 = 2 * C::ACC_COLS;
 

@@ -142,6 +142,8 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
 
   const int K = p.K;
   const int tid = threadIdx.x, nt = blockDim.x;
+  grid_launch_dependents();       // launched with programmatic dependent launch:
+  grid_dependency_wait();         // no global access before the preceding grid completed
   for (int m = blockIdx.x; m < p.M; m += gridDim.x) {
     // 1. stage the row as fp32; the RMS sum of squares is exact per term in fp64
     double ss = 0.0;
@@ -453,6 +455,8 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
   const int K = p.K;
   const int units = BF16 ? K / 8 : K / 4;
   const int row_bytes = K * (BF16 ? 2 : 4);
+  grid_launch_dependents();       // launched with programmatic dependent launch:
+  grid_dependency_wait();         // no global access before the preceding grid completed
   int par = 0;
   for (int m = blockIdx.x; m < p.M; m += gridDim.x, par ^= 1) {
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.X) +
