@@ -337,9 +337,14 @@ def time_loop(torch, fn, steps):
 
 def bench_decode(torch, bn, device, reps=3):
     """Steady-state decode GEMV streaming: a CUDA graph of back-to-back calls
-    over a pool of distinct packed-weight copies larger than twice the L2."""
+    over a pool of distinct packed-weight copies larger than twice the L2, all
+    reading one set of activation codes.  Two launch modes: the calls as the
+    independent projections they are here (BITNET_LAUNCH_PDL_INPUTS: only the
+    output stores wait for the preceding call), and as a dependent chain
+    (BITNET_LAUNCH_PDL: activation loads also wait)."""
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     out = []
+    modes = (("independent", bn.BITNET_LAUNCH_PDL_INPUTS), ("dependent", bn.BITNET_LAUNCH_PDL))
     for (K, N) in DECODE_KN:
         inp = synthetic.linear_inputs(max(DECODE_M), K, N, seed=K + N)
         W = torch.from_numpy(inp["W"]).to(device)
@@ -354,29 +359,32 @@ def bench_decode(torch, bn, device, reps=3):
             q, s, rs = bn.alloc_quant(M, K, device)
             bn.bitnet_quant_act(X[:M].contiguous(), q, s, rs)
             Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
-            epi = bn.BITNET_BF16 | bn.BITNET_LAUNCH_PDL
-            for Pb in pool_bufs[:2]:
-                bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi)
-            torch.cuda.synchronize()
-            graph = torch.cuda.CUDAGraph()
-            stream = torch.cuda.Stream(device)
-            with torch.cuda.stream(stream):
-                graph.capture_begin(capture_error_mode="thread_local")
-                for Pb in pool_bufs:
-                    bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi, stream=stream)
-                graph.capture_end()
-            torch.cuda.synchronize()
-            graph.replay()
-            torch.cuda.synchronize()
-            best = None
-            for _ in range(reps):
-                dt = time_loop(torch, graph.replay, 4)
-                best = dt if best is None else min(best, dt)
-            calls = 4 * pool
-            gbs = decode_bytes(M, K, N) * calls / best / 1e9
-            out.append({"M": M, "K": K, "N": N, "us_per_call": best / calls * 1e6,
-                        "GB_s": gbs, "weights_in_pool": pool})
-            del graph
+            rec = {"M": M, "K": K, "N": N, "weights_in_pool": pool}
+            for name, flag in modes:
+                epi = bn.BITNET_BF16 | flag
+                for Pb in pool_bufs[:2]:
+                    bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi)
+                torch.cuda.synchronize()
+                graph = torch.cuda.CUDAGraph()
+                stream = torch.cuda.Stream(device)
+                with torch.cuda.stream(stream):
+                    graph.capture_begin(capture_error_mode="thread_local")
+                    for Pb in pool_bufs:
+                        bn.bitnet_linear(q, s, rs, Pb, g, K, Y, epilogue=epi, stream=stream)
+                    graph.capture_end()
+                torch.cuda.synchronize()
+                graph.replay()
+                torch.cuda.synchronize()
+                best = None
+                for _ in range(reps):
+                    dt = time_loop(torch, graph.replay, 4)
+                    best = dt if best is None else min(best, dt)
+                calls = 4 * pool
+                key = "" if name == "independent" else "_dependent"
+                rec["us_per_call" + key] = best / calls * 1e6
+                rec["GB_s" + key] = decode_bytes(M, K, N) * calls / best / 1e9
+                del graph
+            out.append(rec)
         del pool_bufs
         torch.cuda.empty_cache()
     return out
@@ -548,6 +556,7 @@ def run_b200(args, world, rank, local):
         dec = bench_decode(torch, bn, device)
         for d in dec:
             d["frac_of_hbm"] = d["GB_s"] / peaks["hbm_gbs"]
+            d["frac_of_hbm_dependent"] = d["GB_s_dependent"] / peaks["hbm_gbs"]
         line["workloads"] = {
             "decode": dec,
             "decode_peak_source": f"{peaks['source']} HBM copy {peaks['hbm_gbs']} GB/s",

@@ -100,6 +100,14 @@ extern "C" {
  * a decode loop over static weights.  Ignored for M > 16 (the prefill GEMM
  * always uses the dependent launch, without early weight reads). */
 #define BITNET_LAUNCH_PDL     0x100
+/* Stronger launch hint for the decode path (implies BITNET_LAUNCH_PDL): the
+ * preceding work on the stream writes none of this call's inputs (packed
+ * weights, gamma, activation codes, scales, code sums, residual), as for the
+ * q/k/v or gate/up projections of a decode step, which read one quantised
+ * input.  Everything up to the output stores (loads, MMAs, the cross-CTA
+ * reduction, dequantisation) may then overlap the preceding work; only the
+ * writes of Y wait for it to finish.  Ignored for M > 16. */
+#define BITNET_LAUNCH_PDL_INPUTS 0x200
 
 /* ----------------------------------------------------------- FFN variants */
 #define BITNET_FFN_RELU2_GLU      0  /* x + down(subnorm(relu(gate(z))^2 * up(z))), z = RMSNorm(x) */
@@ -165,7 +173,8 @@ BITNET_API int bitnet_quant_act(const void *X, int x_dtype, int M, int K,
  *             y = fp32( acc * gamma / s[m] ) (evaluated in fp64, rounded once),
  *             then the optional SiLU / residual add in fp32, then the cast.
  *   residual  [M][N] of Y's type when BITNET_EPI_RESIDUAL is set, else NULL.
- * M <= 16 runs the decode GEMV (HBM-bound), larger M the tcgen05 GEMM.
+ * M <= 2 (K a multiple of 64) runs the dp4a streaming GEMV, M <= 16 the cluster
+ * tensor-core GEMV (both HBM-bound), larger M the tcgen05 GEMM.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 BITNET_API int bitnet_linear(const int8_t *Xq, const float *x_scale, const int32_t *x_rowsum,
                   const uint8_t *packed, const float *gamma,

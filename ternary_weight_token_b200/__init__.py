@@ -30,6 +30,7 @@ from ._binding import (  # noqa: F401
     BITNET_FFN_RELU2_GLU,
     BITNET_I32,
     BITNET_LAUNCH_PDL,
+    BITNET_LAUNCH_PDL_INPUTS,
     BITNET_OK,
     BITNET_PRELUDE_FWHT,
     BITNET_PRELUDE_NONE,

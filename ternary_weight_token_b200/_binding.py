@@ -20,6 +20,7 @@ BITNET_EPI_TYPE_MASK = 0x0F
 BITNET_EPI_RESIDUAL = 0x10
 BITNET_EPI_SILU = 0x20
 BITNET_LAUNCH_PDL = 0x100
+BITNET_LAUNCH_PDL_INPUTS = 0x200
 BITNET_FFN_RELU2_GLU, BITNET_FFN_HADAMARD_SILU = 0, 1
 
 _DTYPE_CODE = {torch.float32: BITNET_F32, torch.bfloat16: BITNET_BF16, torch.int32: BITNET_I32}

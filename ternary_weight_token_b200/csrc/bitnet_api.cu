@@ -167,8 +167,8 @@ int tensor_map_2d_u8(CUtensorMap& out, const void* ptr, uint64_t d0, uint64_t d1
 // setup while the preceding grid on the stream finishes; every kernel
 // launched this way executes griddepcontrol.wait before touching global memory.
 template <typename... KArgs, typename... Args>
-int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-               Args... args) {
+int launch_pdl_if(bool pdl, void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                  cudaStream_t st, Args... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -176,11 +176,17 @@ int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaS
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, args...));
   return BITNET_OK;
+}
+
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+               Args... args) {
+  return launch_pdl_if(true, kern, grid, block, smem, st, args...);
 }
 // Register-resident rows, NT threads x VPT 16-byte chunks, one CTA per row
 // (grid-stride over at most sms * 64 CTAs).
@@ -343,7 +349,7 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   p.M = lp.M; p.N = lp.N; p.K = lp.K; p.units = units;
   p.xs = lp.xs; p.xrs = lp.xrs; p.gamma = lp.gamma;
   p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type;
-  p.flags = lp.flags & ~LAUNCH_PDL;
+  p.flags = lp.flags & ~LAUNCH_PDL;     // keeps LAUNCH_PDL_INPUTS for the kernel
   static bool attr_set = false;
   if (!attr_set) {
     BN_CHECK_CUDA(cudaFuncSetAttribute(gemv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -368,12 +374,51 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   return BITNET_OK;
 }
 
+// Decode for 1..2 tokens with K a multiple of 64: the dp4a streaming kernel
+// (a warp per R rows, all of a lane's weight loads in flight at once).
+template <int MT>
+int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaStream_t st) {
+  void (*kern)(LinearParams) = nullptr;
+  switch (R) {
+    case 1: kern = gemv_stream_kernel<MT, 1, 8>; break;
+    case 2: kern = gemv_stream_kernel<MT, 2, 8>; break;
+    case 4: kern = gemv_stream_kernel<MT, 4, 8>; break;
+    default: kern = gemv_stream_kernel<MT, 8, 8>; break;
+  }
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  LinearParams q = p;
+  q.flags &= ~LAUNCH_PDL;
+  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(kStreamThreads), smem,
+                       st, q);
+}
+
+int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64)
+  const int warps = kStreamThreads / 32;
+  // rows per warp: as many as 8 loads per lane allow while the grid still
+  // covers every SM
+  int R = 1;
+  while (R < 8 && 2 * R * C <= 32 * 8 && (p.N + warps * 2 * R - 1) / (warps * 2 * R) >= di.sms)
+    R *= 2;
+  const int grid = (p.N + warps * R - 1) / (warps * R);
+  const int MT = p.M <= 1 ? 1 : 2;
+  const size_t smem = (size_t)MT * (size_t)p.K;
+  if (MT == 1) return launch_stream_mt<1>(p, R, grid, smem, st);
+  return launch_stream_mt<2>(p, R, grid, smem, st);
+}
+
 int launch_linear(const LinearParams& p, cudaStream_t st) {
+  // 1-2 tokens: the dp4a streaming kernel (measured faster than the cluster
+  // tensor-core path there; from 4 tokens on, its dp4a work and shared-memory
+  // reads sit on the critical path of dependent calls)
+  if (p.M <= 2 && p.K % 64 == 0 && p.ldw / 16 <= 32 * 8) return launch_gemv_stream(p, st);
   if (p.M <= 16) {
     const int rc = launch_gemv_tc(p, st);
     if (rc != BITNET_ERR_UNSUPPORTED) return rc;
     LinearParams q = p;
-    q.flags &= ~LAUNCH_PDL;
+    q.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
     return launch_gemv(q, st);                 // inputs too long for the cluster split
   }
   if (p.flags & EPI_SILU) return launch_tc_cfg<TcSilu>(p, nullptr, nullptr, st);
@@ -391,7 +436,7 @@ int validate_linear(const int8_t* Xq, const float* xs, const int32_t* xrs, const
   const int flags = epilogue & ~BITNET_EPI_TYPE_MASK;
   if (ot != BITNET_F32 && ot != BITNET_BF16 && ot != BITNET_I32)
     return fail(BITNET_ERR_INVALID_ARG, "bad output type %d", ot);
-  if (flags & ~(BITNET_EPI_RESIDUAL | BITNET_EPI_SILU | BITNET_LAUNCH_PDL))
+  if (flags & ~(BITNET_EPI_RESIDUAL | BITNET_EPI_SILU | BITNET_LAUNCH_PDL | BITNET_LAUNCH_PDL_INPUTS))
     return fail(BITNET_ERR_INVALID_ARG, "unknown epilogue flags 0x%x", flags);
   if (ot == BITNET_I32 && (flags & (BITNET_EPI_RESIDUAL | BITNET_EPI_SILU)))
     return fail(BITNET_ERR_UNSUPPORTED, "the int32 output takes no residual or SiLU");
@@ -505,7 +550,8 @@ int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsu
   p.M = M; p.N = N; p.K = K; p.ldw = (int)bitnet_packed_row_bytes(K);
   p.Y = Y; p.out_type = epilogue & BITNET_EPI_TYPE_MASK;
   p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = residual;
-  if (M > 16) p.flags &= ~LAUNCH_PDL;
+  if (p.flags & LAUNCH_PDL_INPUTS) p.flags |= LAUNCH_PDL;
+  if (M > 16) p.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
   return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
 }
 

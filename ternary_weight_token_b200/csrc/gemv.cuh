@@ -20,7 +20,7 @@
 namespace bitnet {
 
 enum { OUT_F32 = 0, OUT_BF16 = 1, OUT_I32 = 2 };
-enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20, LAUNCH_PDL = 0x100 };
+enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20, LAUNCH_PDL = 0x100, LAUNCH_PDL_INPUTS = 0x200 };
 
 struct LinearParams {
   const int8_t* Xq;
@@ -178,6 +178,128 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
                         p.flags);
         }
       }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Streaming decode for 1..2 tokens (dp4a on the CUDA cores, no tensor memory,
+// no cluster).  A warp owns R whole weight rows; its R * C 16-byte packed
+// chunks (C = row_bytes / 16) are spread over the 32 lanes, J per lane, and
+// every lane issues all of its loads before anything waits: for a decode
+// call the whole matrix is a few tens of KB per SM, so the call is bound by
+// load latency, and consecutive calls are meant to overlap (several of these
+// small CTAs fit on an SM next to the previous call's).  Activation codes are
+// staged in shared memory (K a multiple of 64).  The weights are read before griddepcontrol.wait
+// (the caller's LAUNCH_PDL statement covers them); with LAUNCH_PDL_INPUTS the
+// activations and the whole contraction also precede it, and only the output
+// stores wait.
+
+constexpr int kStreamThreads = 128;
+
+template <int MT, int R, int J>
+__global__ void __launch_bounds__(kStreamThreads) gemv_stream_kernel(LinearParams p) {
+  // activation codes as [MT][4][C] 16-byte units: unit u of a token row (its
+  // inputs 16u .. 16u + 15) sits in plane u % 4 at index u / 4, so the lanes
+  // of a warp, which hold consecutive chunks, read consecutive 16-byte words
+  extern __shared__ uint4 gs_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = p.ldw / 16;                    // packed chunks per row
+  const int n0 = (blockIdx.x * (kStreamThreads / 32) + warp) * R;
+  const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
+  grid_launch_dependents();
+
+  // 1. every packed chunk of this warp's rows, in flight at once
+  uint4 w[J];
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int f = lane + 32 * j;
+    const int r = f / C, c = f - r * C;
+    w[j] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // t = 0
+    if (r < R && n0 + r < p.N) w[j] = ld_stream_v4(p.W + (size_t)(n0 + r) * p.ldw + 16 * c);
+  }
+
+  // 2. activation codes, token scales and code sums
+  if (!inputs_ready) grid_dependency_wait();
+  const int units = p.K / 16;
+  for (int i = threadIdx.x; i < MT * units; i += kStreamThreads) {
+    const int m = i / units, u = i - m * units;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (m < p.M) v = *reinterpret_cast<const uint4*>(p.Xq + (size_t)m * p.K + 16 * u);
+    gs_smem[(m * 4 + (u & 3)) * C + (u >> 2)] = v;
+  }
+  const int mt = lane < MT ? lane : 0;
+  const bool tok = lane < p.M;
+  const float s_m = tok ? p.xs[mt] : 1.0f;
+  const int rs_m = tok ? p.xrs[mt] : 0;
+  float fh_m = 0.0f, fl_m = 0.0f;
+  if (p.out_type != OUT_I32) dequant_factor(__ldg(p.gamma), s_m, fh_m, fl_m);
+  __syncthreads();
+
+  // 3. unsigned codes x signed activations, per row and token
+  int acc[R][MT];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int f = lane + 32 * j;
+    const int r = f / C, c = f - r * C;
+    if (r < R) {
+      uint32_t e[16];
+      expand_codes(w[j].x, e[0], e[1], e[2], e[3]);
+      expand_codes(w[j].y, e[4], e[5], e[6], e[7]);
+      expand_codes(w[j].z, e[8], e[9], e[10], e[11]);
+      expand_codes(w[j].w, e[12], e[13], e[14], e[15]);
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4* qp = gs_smem + m * 4 * C + c;       // 64 activation codes
+        const uint4 q0 = qp[0], q1 = qp[C], q2 = qp[2 * C], q3 = qp[3 * C];
+        int a = 0;
+        a = dp4a_us(e[0], q0.x, a);  a = dp4a_us(e[1], q0.y, a);
+        a = dp4a_us(e[2], q0.z, a);  a = dp4a_us(e[3], q0.w, a);
+        a = dp4a_us(e[4], q1.x, a);  a = dp4a_us(e[5], q1.y, a);
+        a = dp4a_us(e[6], q1.z, a);  a = dp4a_us(e[7], q1.w, a);
+        a = dp4a_us(e[8], q2.x, a);  a = dp4a_us(e[9], q2.y, a);
+        a = dp4a_us(e[10], q2.z, a); a = dp4a_us(e[11], q2.w, a);
+        a = dp4a_us(e[12], q3.x, a); a = dp4a_us(e[13], q3.y, a);
+        a = dp4a_us(e[14], q3.z, a); a = dp4a_us(e[15], q3.w, a);
+#pragma unroll
+        for (int rr = 0; rr < R; ++rr)
+          if (rr == r) acc[rr][m] += a;
+      }
+    }
+  }
+
+  // 4. warp sums; lane r * MT + m holds row r, token m
+  float y = 0.0f;
+  int yint = 0;
+  int my_r = -1, my_m = 0;
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      int v = acc[r][m];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      const int rs = __shfl_sync(0xffffffffu, rs_m, m);
+      const float fh = __shfl_sync(0xffffffffu, fh_m, m);
+      const float fl = __shfl_sync(0xffffffffu, fl_m, m);
+      if (lane == r * MT + m) {
+        my_r = r;
+        my_m = m;
+        yint = v - rs;
+        y = p.out_type == OUT_I32 ? 0.0f : dequant_dw(yint, fh, fl);
+      }
+    }
+  if (inputs_ready) grid_dependency_wait();    // Y may still be read or written before
+  const int n = n0 + my_r;
+  if (my_r >= 0 && my_m < p.M && n < p.N) {
+    const size_t idx = (size_t)my_m * p.N + n;
+    if (p.out_type == OUT_I32)
+      reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
+    else
+      store_value(p.Y, p.resid, idx, y, p.out_type, p.flags);
   }
 }
 

@@ -25,7 +25,10 @@
 //     token's code sum, dequantises and writes the outputs.
 // With programmatic dependent launch the weight loads and their expansion
 // start before the preceding kernel on the stream has finished; activation
-// codes, scales and outputs are touched only after griddepcontrol.wait.
+// codes, scales and outputs are touched only after griddepcontrol.wait.  When
+// the caller states that the preceding work writes none of the inputs
+// (LAUNCH_PDL_INPUTS), everything up to the leader's output stores runs
+// before that wait.
 #pragma once
 
 #include "common.cuh"
@@ -181,6 +184,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   int k0, ks;
   dec_slice(p.units, (int)csize, (int)rank, k0, ks);
   const int chunks = (ks + kDecChunkK - 1) / kDecChunkK;
+  // inputs not written by the preceding work: only the output stores wait
+  const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
 
   grid_launch_dependents();
   if (threadIdx.x == 0) {
@@ -215,7 +220,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         mbar_arrive_expect_tx(&wfull[c], DecSmem::W_CHUNK);
         tma_load_2d(sw + c * DecSmem::W_CHUNK, &tm_w, &wfull[c], (k0 + c * kDecChunkK) / 4, n0);
       }
-      grid_dependency_wait();                // activation codes come from the previous kernel
+      if (!inputs_ready) grid_dependency_wait();   // activation codes from the previous kernel
       tma_prefetch_desc(&tm_x);
       for (int c = 0; c < chunks; ++c) {
         mbar_arrive_expect_tx(&xfull[c], DecSmem::X_CHUNK);
@@ -292,40 +297,49 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
     if (rank == 0) {
       // leader: token scales and code sums are fetched while the peers'
-      // partials arrive; then all partial sums are read before any output
-      // is stored (no load waits behind a store)
-      grid_dependency_wait();
+      // partials arrive; each token's dequant factor is formed once per warp
+      // (lane m for token m, then shuffled); all partial sums are read and
+      // every output value is computed before the first store, and with
+      // LAUNCH_PDL_INPUTS before the wait for the preceding grid, so only
+      // the stores follow it.
+      if (!inputs_ready) grid_dependency_wait();
       const float g = __ldg(p.gamma);
-      float sm[kDecTokens];
-      int rsum[kDecTokens];
-#pragma unroll
-      for (int m = 0; m < kDecTokens; ++m) {
-        sm[m] = m < p.M ? __ldg(p.xs + m) : 1.0f;
-        rsum[m] = m < p.M ? __ldg(p.xrs + m) : 0;
-      }
+      const int mt = lane < kDecTokens ? lane : 0;
+      const bool tok = lane < p.M;
+      const float s_m = tok ? __ldg(p.xs + mt) : 1.0f;
+      const int rs_m = tok ? __ldg(p.xrs + mt) : 0;
+      float fh_m = 0.0f, fl_m = 0.0f;
+      if (p.out_type != OUT_I32) dequant_factor(g, s_m, fh_m, fl_m);
       const bool all_in = mbar_wait_cluster(reduce_bar, 0);
       const int n = n0 + row;
-      if (all_in && n < p.N) {
-        const int32_t* part = reinterpret_cast<const int32_t*>(smem + DecSmem::OFF_PART);
-        int acc[kDecTokens];
+      const int32_t* part = reinterpret_cast<const int32_t*>(smem + DecSmem::OFF_PART);
+      int acc[kDecTokens];
 #pragma unroll
-        for (int m = 0; m < kDecTokens; ++m) acc[m] = -rsum[m];
+      for (int m = 0; m < kDecTokens; ++m) acc[m] = -__shfl_sync(0xffffffffu, rs_m, m);
+      if (all_in) {
         for (int r = 0; r < (int)csize; ++r) {
 #pragma unroll
           for (int m = 0; m < kDecTokens; ++m)
             if (m < p.M) acc[m] += part[(r * 16 + m) * 128 + row];
         }
+      }
+      float y[kDecTokens];
+#pragma unroll
+      for (int m = 0; m < kDecTokens; ++m) {
+        const float fh = __shfl_sync(0xffffffffu, fh_m, m);
+        const float fl = __shfl_sync(0xffffffffu, fl_m, m);
+        y[m] = p.out_type == OUT_I32 ? __int_as_float(acc[m]) : dequant_dw(acc[m], fh, fl);
+      }
+      if (inputs_ready) grid_dependency_wait();  // Y may still be read or written before
+      if (all_in && n < p.N) {
 #pragma unroll
         for (int m = 0; m < kDecTokens; ++m) {
           if (m < p.M) {
             const size_t idx = (size_t)m * p.N + n;
-            if (p.out_type == OUT_I32) {
-              reinterpret_cast<int32_t*>(p.Y)[idx] = acc[m];
-            } else {
-              float fh, fl;
-              dequant_factor(g, sm[m], fh, fl);
-              store_value(p.Y, p.resid, idx, dequant_dw(acc[m], fh, fl), p.out_type, p.flags);
-            }
+            if (p.out_type == OUT_I32)
+              reinterpret_cast<int32_t*>(p.Y)[idx] = __float_as_int(y[m]);
+            else
+              store_value(p.Y, p.resid, idx, y[m], p.out_type, p.flags);
           }
         }
       }

@@ -157,6 +157,40 @@ def test_decode_with_programmatic_dependent_launch():
         assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="pdl step")
 
 
+def test_decode_independent_projections_overlap():
+    """BITNET_LAUNCH_PDL_INPUTS: consecutive decode calls that read one set of
+    activation codes (as q/k/v or gate/up do) may run everything but their
+    output stores under the preceding call.  Distinct weights, a shared
+    output written by every call (the last call's values must remain) and
+    distinct outputs, all bit-exact against the oracle (int32)."""
+    M, K = 16, 2560
+    rng_w, rng_x = synthetic.streams(43, 2)
+    X = synthetic.activations(rng_x, M, K)
+    q, s, rs = oracle.quant_act(X)
+    qd, sd, rsd = dev(q), dev(s), dev(rs)
+    shapes = [(2560, 0), (640, 1), (640, 2), (6912, 3), (2560, 4), (6912, 5)]
+    packs = []
+    for N, i in shapes:
+        W = synthetic.weight(rng_w, N, K)
+        g, T, P = oracle.quantize_weights(W)
+        packs.append((N, T, dev(P), dev(np.array([g], np.float32))))
+    shared = torch.empty((M, 6912), dtype=torch.int32, device="cuda")
+    outs = []
+    flags = bn.BITNET_I32 | bn.BITNET_LAUNCH_PDL_INPUTS
+    for rnd in range(3):
+        for N, T, Pd, gd in packs:
+            Y = torch.empty((M, N), dtype=torch.int32, device="cuda")
+            bn.bitnet_linear(qd, sd, rsd, Pd, gd, K, Y, epilogue=flags)
+            if N == 6912:
+                bn.bitnet_linear(qd, sd, rsd, Pd, gd, K, shared, epilogue=flags)
+            outs.append((Y, T))
+    torch.cuda.synchronize()
+    for Y, T in outs:
+        np.testing.assert_array_equal(Y.cpu().numpy(), oracle.contract(q, T))
+    np.testing.assert_array_equal(shared.cpu().numpy(), oracle.contract(q, packs[-1][1]))
+    assert bn.bitnet_check_device_error() == bn.BITNET_OK
+
+
 @pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 6912), (6912, 2560)])
 def test_decode_shapes_all_m(K, N):
     """The 2B-model decode shapes for every token count 1..16 (cluster split-K
