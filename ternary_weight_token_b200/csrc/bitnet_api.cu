@@ -223,6 +223,22 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
     if (k4 <= 128 * 14) return launch_quant_rows<128, 14>(p, bf16, prelude, st);
     return launch_quant_rows<256, 16>(p, bf16, prelude, st);   // K <= 16384
   }
+  // FWHT rows of 128 (fp32) / 256 (bf16) up to 2048 inputs: one warp per row
+  // in registers; other widths: the row staged in shared memory
+  if (K <= 2048 && K >= (bf16 ? 256 : 128)) {
+    void (*kw)(QuantParams) = nullptr;
+    switch (K) {
+      case 128: kw = quant_fwht_warp_kernel<128, false>; break;
+      case 256: kw = bf16 ? quant_fwht_warp_kernel<256, true> : quant_fwht_warp_kernel<256, false>; break;
+      case 512: kw = bf16 ? quant_fwht_warp_kernel<512, true> : quant_fwht_warp_kernel<512, false>; break;
+      case 1024: kw = bf16 ? quant_fwht_warp_kernel<1024, true> : quant_fwht_warp_kernel<1024, false>; break;
+      default: kw = bf16 ? quant_fwht_warp_kernel<2048, true> : quant_fwht_warp_kernel<2048, false>; break;
+    }
+    const int rows_per_cta = 4;
+    const int need = (M + rows_per_cta - 1) / rows_per_cta;
+    const int cap = di.sms * 16;
+    return launch_pdl(kw, dim3(need < cap ? need : cap), dim3(128), 0, st, p);
+  }
   const int threads = K >= 2048 ? 256 : 128;
   const size_t smem = (size_t)K * sizeof(float);
   const int grid = M < di.sms * 16 ? M : di.sms * 16;

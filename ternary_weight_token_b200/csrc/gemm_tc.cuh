@@ -371,9 +371,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                   float y0 = dequant_dw((int)v[i] - rr.x, ff.x, ff.y);
                   float y1 = dequant_dw((int)v[i + 1] - rr.y, ff.z, ff.w);
                   if (C::SILU) {
-                    const double d0 = (double)y0, d1 = (double)y1;
-                    y0 = (float)(d0 / (1.0 + exp(-d0)));
-                    y1 = (float)(d1 / (1.0 + exp(-d1)));
+                    y0 = silu_f32(y0);
+                    y1 = silu_f32(y1);
                   }
                   if (p.flags & EPI_RESIDUAL) {
                     y0 = __fadd_rn(__uint_as_float(rpk[i >> 1] << 16), y0);
@@ -450,10 +449,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
               const int t = 32 * c + j;
               const float2 fa = tok_f[t];
               float yy = dequant_dw((int)v[j] - tok_rs[t], fa.x, fa.y);
-              if (C::SILU) {            // only the SiLU instance carries the exp call
-                const double d = (double)yy;
-                yy = (float)(d / (1.0 + exp(-d)));
-              }
+              if (C::SILU) yy = silu_f32(yy);   // only the SiLU instance carries expf
               if (p.flags & EPI_RESIDUAL) {
                 if (C::SILU) {          // rare combination: plain per-element load
                   const int m = mc + j;

@@ -475,4 +475,120 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// FWHT prelude, one warp per token row, the row in registers (K = 2^n with
+// VEC * 32 <= K <= 2048).  Lane l holds the 16-byte vectors j = 0 .. J-1 at
+// elements k = VEC * l + 32 * VEC * j + e.  The butterfly stages run in the
+// fixed order h = 1, 2, 4, ...: h < VEC inside a vector, VEC <= h < 32 VEC
+// between lanes (shuffle with lane ^ (h / VEC); the lower partner keeps a + b,
+// the upper a - b, the same fp32 operations as the staged kernel), h >= 32 VEC
+// between a lane's own vectors.  No block barrier anywhere.
+template <int K, bool BF16>
+__global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
+  constexpr int VEC = BF16 ? 8 : 4;
+  constexpr int J = K / (32 * VEC);
+  static_assert(J >= 1 && J * 32 * VEC == K, "row width");
+  const int lane = threadIdx.x & 31;
+  const int warp_g = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int nwarps = gridDim.x * 4;
+  grid_launch_dependents();       // launched with programmatic dependent launch:
+  grid_dependency_wait();         // no global access before the preceding grid completed
+  for (int m = warp_g; m < p.M; m += nwarps) {
+    float v[J][VEC];
+    if (BF16) {
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const uint16_t*>(p.X) + (size_t)m * K) + lane;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const uint4 u = ld_stream_v4(src + 32 * j);
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[j][2 * e] = __uint_as_float(w4[e] << 16);
+          v[j][2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+        }
+      }
+    } else {
+      const float4* src = reinterpret_cast<const float4*>(
+          reinterpret_cast<const float*>(p.X) + (size_t)m * K) + lane;
+#pragma unroll
+      for (int j = 0; j < J; ++j) {
+        const uint4 u = ld_stream_v4(src + 32 * j);
+        v[j][0] = __uint_as_float(u.x); v[j][1] = __uint_as_float(u.y);
+        v[j][2] = __uint_as_float(u.z); v[j][3] = __uint_as_float(u.w);
+      }
+    }
+    // h < VEC: inside each vector
+#pragma unroll
+    for (int h = 1; h < VEC; h <<= 1)
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e)
+          if ((e & h) == 0) {
+            const float a = v[j][e], b = v[j][e + h];
+            v[j][e] = __fadd_rn(a, b);
+            v[j][e + h] = __fsub_rn(a, b);
+          }
+    // VEC <= h < 32 VEC: between lanes
+#pragma unroll
+    for (int lb = 1; lb < 32; lb <<= 1) {
+      const bool upper = (lane & lb) != 0;
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float mine = v[j][e];
+          const float other = __shfl_xor_sync(0xffffffffu, mine, lb);
+          v[j][e] = upper ? __fsub_rn(other, mine) : __fadd_rn(mine, other);
+        }
+    }
+    // h >= 32 VEC: between this lane's vectors
+#pragma unroll
+    for (int hj = 1; hj < J; hj <<= 1)
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+        if ((j & hj) == 0)
+#pragma unroll
+          for (int e = 0; e < VEC; ++e) {
+            const float a = v[j][e], b = v[j + hj][e];
+            v[j][e] = __fadd_rn(a, b);
+            v[j + hj][e] = __fsub_rn(a, b);
+          }
+    // normalisation, absmax, codes
+    float amax = 0.0f;
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) {
+        v[j][e] = __fmul_rn(v[j][e], p.fwht_c);
+        amax = fmaxf(amax, fabsf(v[j][e]));
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    float s = __fdiv_rn(127.0f, amax);
+    const bool zero_row = (amax == 0.0f) || isinf(s);
+    if (zero_row) s = 1.0f;
+    int rsum = 0;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.Xq + (size_t)m * K);
+#pragma unroll
+    for (int j = 0; j < J; ++j)
+#pragma unroll
+      for (int e = 0; e < VEC; e += 4) {
+        uint32_t w = 0u;
+        if (!zero_row) {
+          w = pack_codes4(__fmul_rn(v[j][e], s), __fmul_rn(v[j][e + 1], s),
+                          __fmul_rn(v[j][e + 2], s), __fmul_rn(v[j][e + 3], s));
+          rsum = __dp4a((int)w, 0x01010101, rsum);
+        }
+        dst[(VEC * lane + 32 * VEC * j + e) / 4] = w;
+      }
+    rsum = __reduce_add_sync(0xffffffffu, rsum);
+    if (lane == 0) {
+      p.scale[m] = s;
+      if (p.rowsum != nullptr) p.rowsum[m] = rsum;
+    }
+  }
+}
+
 }  // namespace bitnet

@@ -40,11 +40,26 @@ def test_quant_none_bit_exact(M, K):
     np.testing.assert_array_equal(rs, rso)
 
 
-@pytest.mark.parametrize("K", [16, 512, 2048, 8192])
+@pytest.mark.parametrize("K", [16, 64, 128, 256, 512, 1024, 2048, 4096, 8192])
 def test_quant_fwht_bit_exact(K):
+    """Both FWHT kernels: one warp per row in registers (128..2048 inputs) and
+    the row staged in shared memory (other widths)."""
     X = _acts(33, K, seed=K, outliers=True)
+    X[5] = 0.0                                  # an all-zero token
     q, s, rs = gpu_quant(X, bn.BITNET_PRELUDE_FWHT)
     qo, so, rso = oracle.quant_act(X, oracle.PRELUDE_FWHT)
+    np.testing.assert_array_equal(q, qo)
+    np.testing.assert_array_equal(s, so)
+    np.testing.assert_array_equal(rs, rso)
+
+
+@pytest.mark.parametrize("K", [128, 256, 2048])
+def test_quant_fwht_bf16_bit_exact(K):
+    X = _acts(21, K, seed=K + 1, outliers=True)
+    bits = synthetic.to_bf16_bits(X)
+    xw = oracle.bf16_bits_to_f32(bits)
+    q, s, rs = gpu_quant(xw, bn.BITNET_PRELUDE_FWHT, x_dev=bf16_dev(bits))
+    qo, so, rso = oracle.quant_act(xw, oracle.PRELUDE_FWHT)
     np.testing.assert_array_equal(q, qo)
     np.testing.assert_array_equal(s, so)
     np.testing.assert_array_equal(rs, rso)
