@@ -49,6 +49,8 @@ def _load():
         "orc_packed_row_bytes": (i64, [i32]),
         "orc_pack": (None, [P, i32, i32, P]),
         "orc_unpack": (i32, [P, i32, i32, P]),
+        "orc_pack_tw2": (None, [P, i32, i32, P]),
+        "orc_unpack_tw2": (i32, [P, i32, i32, P]),
         "orc_rmsnorm": (None, [P, i32, i32, P, f32, P]),
         "orc_fwht": (i32, [P, i32, i32, P]),
         "orc_quant_act": (i32, [P, i32, i32, i32, P, f32, P, P, P]),
@@ -125,6 +127,26 @@ def unpack(P, K):
     N = P.shape[0]
     t = np.empty((N, K), dtype=np.int8)
     _check(_load().orc_unpack(_p(P), N, int(K), _p(t)), "unpack")
+    return t
+
+
+def pack_tw2(T):
+    """Ternary codes [N][K] -> the canonical exchange layout TW2, uint8
+    [N][K/4]: code t + 1 of weight k at bits 2 (k mod 4) of byte k / 4."""
+    T = _i8(T)
+    N, K = T.shape
+    if K % 4:
+        raise OracleError("TW2 needs K to be a multiple of 4")
+    out = np.empty((N, K // 4), dtype=np.uint8)
+    _load().orc_pack_tw2(_p(T), N, K, _p(out))
+    return out
+
+
+def unpack_tw2(P, K):
+    P = np.ascontiguousarray(P, dtype=np.uint8)
+    N = P.shape[0]
+    t = np.empty((N, K), dtype=np.int8)
+    _check(_load().orc_unpack_tw2(_p(P), N, int(K), _p(t)), "unpack_tw2")
     return t
 
 

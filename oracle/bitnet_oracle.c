@@ -110,6 +110,35 @@ int orc_unpack(const uint8_t *packed, int N, int K, int8_t *t)
     return ORC_OK;
 }
 
+/* The canonical exchange layout TW2: row n occupies bytes [n K/4, (n+1) K/4)
+ * and weight k of row n is the code c = t + 1 at bits 2 (k mod 4) of byte
+ * n K/4 + floor(k / 4) (four to a byte, [NN] "stored ternary, four to a
+ * byte"; the low-bits-first order is this library's stated convention).
+ * K must be a multiple of 4. */
+void orc_pack_tw2(const int8_t *t, int N, int K, uint8_t *tw2)
+{
+    int64_t rb = K / 4;
+    memset(tw2, 0, (size_t)(rb * N));
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            unsigned code = (unsigned)(t[(int64_t)n * K + k] + 1);
+            tw2[(int64_t)n * rb + k / 4] |= (uint8_t)(code << (2 * (k % 4)));
+        }
+}
+
+/* Inverse of orc_pack_tw2.  Returns ORC_ERR_ARG if any code is 3. */
+int orc_unpack_tw2(const uint8_t *tw2, int N, int K, int8_t *t)
+{
+    int64_t rb = K / 4;
+    for (int n = 0; n < N; ++n)
+        for (int k = 0; k < K; ++k) {
+            unsigned code = (tw2[(int64_t)n * rb + k / 4] >> (2 * (k % 4))) & 3u;
+            if (code == 3u) return ORC_ERR_ARG;
+            t[(int64_t)n * K + k] = (int8_t)((int)code - 1);
+        }
+    return ORC_OK;
+}
+
 /* ------------------------------------------------------------- preludes */
 
 /* RMSNorm with gain, no bias, eps 1e-5 in the model ([NN] "Config":

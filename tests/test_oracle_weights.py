@@ -144,6 +144,37 @@ def test_golden_pack_example():
     np.testing.assert_array_equal(p[0], np.array(ex["packed"], dtype=np.uint8))
 
 
+def test_golden_tw2_example():
+    ex = _load("tw2_example.json")
+    t = np.array([ex["t"]], dtype=np.int8)
+    p = oracle.pack_tw2(t)
+    assert p.shape == (1, 4)
+    np.testing.assert_array_equal(p[0], np.array(ex["tw2"], dtype=np.uint8))
+    np.testing.assert_array_equal(oracle.unpack_tw2(p, 16), t)
+
+
+@pytest.mark.parametrize("K", [16, 64, 2560, 6912])
+def test_tw2_roundtrip_and_bit_positions(K):
+    """Both layouts hold the same codes: each unpacks to t, a direct bit read
+    of TW2 gives t + 1, and code 3 never appears."""
+    rng = np.random.default_rng(K + 7)
+    N = 3
+    t = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    p = oracle.pack_tw2(t)
+    assert p.shape == (N, K // 4)
+    np.testing.assert_array_equal(oracle.unpack_tw2(p, K), t)
+    np.testing.assert_array_equal(oracle.unpack(oracle.pack(t), K), t)
+    for n in range(N):
+        for k in list(range(min(K, 24))) + [K - 1]:
+            assert ((p[n, k // 4] >> (2 * (k % 4))) & 3) == t[n, k] + 1
+    codes = np.stack([(p >> s) & 3 for s in (0, 2, 4, 6)], axis=-1)
+    assert not np.any(codes == 3)
+    bad = p.copy()
+    bad[0, 0] |= 3
+    with pytest.raises(oracle.OracleError):
+        oracle.unpack_tw2(bad, K)
+
+
 @pytest.mark.parametrize("K", [16, 48, 64, 80, 256, 2560, 6912])
 def test_pack_roundtrip_and_padding(K):
     rng = np.random.default_rng(K)
