@@ -142,6 +142,21 @@ BITNET_API int bitnet_pack_weights(const void *W, int w_dtype, int N, int K,
                         uint8_t *packed, float *gamma,
                         void *workspace, size_t ws_bytes, bitnet_stream_t stream);
 
+/* The canonical exchange layout TW2 and this library's device layout.
+ * TW2: [N][K/4] bytes, weight k of row n is the code t + 1 at bits 2 (k % 4)
+ * of byte n K/4 + k/4 (four to a byte, [NN] "stored ternary, four to a byte";
+ * low bits first is this library's convention).  bitnet_pack_weights() and
+ * bitnet_linear() use the device layout above (16 codes per 32-bit word
+ * arranged so that two ALU ops expand four of them); these two calls convert.
+ *   packed  [N][bitnet_packed_row_bytes(K)] device layout.
+ *   tw2     [N][K/4] TW2.  An input code 3 is invalid (unspecified result).
+ * K must be a multiple of 16 in [16, 16384]; pointers 16-byte aligned; N = 0
+ * is a no-op.  Errors: INVALID_ARG, CUDA. */
+BITNET_API int bitnet_export_tw2(const uint8_t *packed, int N, int K, uint8_t *tw2,
+                                 bitnet_stream_t stream);
+BITNET_API int bitnet_import_tw2(const uint8_t *tw2, int N, int K, uint8_t *packed,
+                                 bitnet_stream_t stream);
+
 /* Per-token int8 absmax quantisation with an optional fused prelude
  * (nnterp "bitnet", same section: round(x * 127 / max|x|) per token; "BitNet
  * b1.58 2B4T", "Model Details": absmax per token; sub-norm RMSNorm, nnterp

@@ -41,11 +41,13 @@ from ._binding import (  # noqa: F401
     alloc_quant,
     bitnet_check_device_error,
     bitnet_debug_wait_timeout,
+    bitnet_export_tw2,
     bitnet_ffn,
     bitnet_ffn_noalloc,
     BITNET_FFN_NOALLOC_SCRATCH_BYTES,
     bitnet_ffn_workspace_size,
     bitnet_last_error,
+    bitnet_import_tw2,
     bitnet_linear,
     bitnet_pack_weights,
     bitnet_pack_workspace_size,

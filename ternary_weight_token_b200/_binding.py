@@ -54,6 +54,8 @@ def library():
         "bitnet_packed_row_bytes": (S, [I]),
         "bitnet_pack_workspace_size": (S, [I, I]),
         "bitnet_pack_weights": (I, [P, I, I, I, P, P, P, S, P]),
+        "bitnet_export_tw2": (I, [P, I, I, P, P]),
+        "bitnet_import_tw2": (I, [P, I, I, P, P]),
         "bitnet_quant_act": (I, [P, I, I, I, I, P, F, P, P, P, P]),
         "bitnet_linear": (I, [P, P, P, P, P, I, I, I, P, I, P, P]),
         "bitnet_ffn_workspace_size": (S, [I, I, I, I]),
@@ -135,6 +137,19 @@ def bitnet_pack_weights(W, packed, gamma, workspace, stream=None):
     _check(library().bitnet_pack_weights(_ptr(W), _dtype(W), N, K, _ptr(packed), _ptr(gamma),
                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
+
+
+def bitnet_export_tw2(packed, K, tw2, stream=None):
+    """Device-layout packed weights [N][packed_row_bytes(K)] -> the canonical
+    exchange layout TW2 [N][K/4] (four codes to a byte, low bits first)."""
+    _check(library().bitnet_export_tw2(_ptr(packed), packed.shape[0], int(K), _ptr(tw2),
+                                       _stream(stream)))
+
+
+def bitnet_import_tw2(tw2, K, packed, stream=None):
+    """TW2 [N][K/4] -> device-layout packed weights [N][packed_row_bytes(K)]."""
+    _check(library().bitnet_import_tw2(_ptr(tw2), tw2.shape[0], int(K), _ptr(packed),
+                                       _stream(stream)))
 
 
 def bitnet_quant_act(X, Xq, x_scale, x_rowsum=None, prelude=BITNET_PRELUDE_NONE, norm_gain=None,

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -392,37 +393,41 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
 
 // Decode for 1..2 tokens with K a multiple of 64: the dp4a streaming kernel
 // (a warp per R rows, all of a lane's weight loads in flight at once).
-template <int MT>
+template <int MT, int NT>
 int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaStream_t st) {
   void (*kern)(LinearParams) = nullptr;
   switch (R) {
-    case 1: kern = gemv_stream_kernel<MT, 1, 8>; break;
-    case 2: kern = gemv_stream_kernel<MT, 2, 8>; break;
-    case 4: kern = gemv_stream_kernel<MT, 4, 8>; break;
-    default: kern = gemv_stream_kernel<MT, 8, 8>; break;
+    case 1: kern = gemv_stream_kernel<MT, 1, 8, NT>; break;
+    case 2: kern = gemv_stream_kernel<MT, 2, 8, NT>; break;
+    case 3: kern = gemv_stream_kernel<MT, 3, 8, NT>; break;
+    case 4: kern = gemv_stream_kernel<MT, 4, 8, NT>; break;
+    case 5: kern = gemv_stream_kernel<MT, 5, 8, NT>; break;
+    case 6: kern = gemv_stream_kernel<MT, 6, 8, NT>; break;
+    case 7: kern = gemv_stream_kernel<MT, 7, 8, NT>; break;
+    default: kern = gemv_stream_kernel<MT, 8, 8, NT>; break;
   }
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   LinearParams q = p;
   q.flags &= ~LAUNCH_PDL;
-  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(kStreamThreads), smem,
-                       st, q);
+  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(NT), smem, st, q);
 }
+
+constexpr int kStreamThreads = 256;
 
 int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
   const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64)
   const int warps = kStreamThreads / 32;
-  // rows per warp: as many as 8 loads per lane allow while the grid still
-  // covers every SM
-  int R = 1;
-  while (R < 8 && 2 * R * C <= 32 * 8 && (p.N + warps * 2 * R - 1) / (warps * 2 * R) >= di.sms)
-    R *= 2;
+  // about one CTA per SM per call (so several back-to-back calls can be
+  // resident at once): R rows per warp, at most 8 loads per lane
+  int R = (p.N + di.sms * warps - 1) / (di.sms * warps);
+  if (R > 8) R = 8;
+  while (R > 1 && R * C > 32 * 8) --R;
   const int grid = (p.N + warps * R - 1) / (warps * R);
-  const int MT = p.M <= 1 ? 1 : 2;
-  const size_t smem = (size_t)MT * (size_t)p.K;
-  if (MT == 1) return launch_stream_mt<1>(p, R, grid, smem, st);
-  return launch_stream_mt<2>(p, R, grid, smem, st);
+  const size_t smem = (size_t)(p.M <= 1 ? 1 : 2) * (size_t)p.K;
+  if (p.M <= 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
+  return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
 }
 
 int launch_linear(const LinearParams& p, cudaStream_t st) {
@@ -523,6 +528,47 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
     pack_kernel<true><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
   else
     pack_kernel<false><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+static int validate_tw2(const void* a, const void* b, int N, int K) {
+  if (a == nullptr || b == nullptr) return fail(BITNET_ERR_INVALID_ARG, "null pointer");
+  if (N < 0) return fail(BITNET_ERR_INVALID_ARG, "N=%d must be >= 0", N);
+  if (int rc = check_k(K)) return rc;
+  if (!aligned16(a) || !aligned16(b))
+    return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  return BITNET_OK;
+}
+
+int bitnet_export_tw2(const uint8_t* packed, int N, int K, uint8_t* tw2, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (int rc = validate_tw2(packed, tw2, N, K)) return rc;
+  if (N == 0) return BITNET_OK;
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int ldw_words = (int)(bitnet_packed_row_bytes(K) / 4), tw2_words = K / 16;
+  const int64_t total = (int64_t)N * tw2_words;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)di.sms * 8);
+  export_tw2_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(packed), N, ldw_words, tw2_words,
+      reinterpret_cast<uint32_t*>(tw2));
+  BN_CHECK_CUDA(cudaGetLastError());
+  return BITNET_OK;
+}
+
+int bitnet_import_tw2(const uint8_t* tw2, int N, int K, uint8_t* packed, bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (int rc = validate_tw2(tw2, packed, N, K)) return rc;
+  if (N == 0) return BITNET_OK;
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int ldw_words = (int)(bitnet_packed_row_bytes(K) / 4), tw2_words = K / 16;
+  const int64_t total = (int64_t)N * ldw_words;
+  const int grid = (int)std::min<int64_t>((total + 255) / 256, (int64_t)di.sms * 8);
+  import_tw2_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(tw2), N, ldw_words, tw2_words,
+      reinterpret_cast<uint32_t*>(packed));
   BN_CHECK_CUDA(cudaGetLastError());
   return BITNET_OK;
 }

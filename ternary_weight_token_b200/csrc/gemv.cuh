@@ -201,17 +201,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
 // activations and the whole contraction also precede it, and only the output
 // stores wait.
 
-constexpr int kStreamThreads = 128;
-
-template <int MT, int R, int J>
-__global__ void __launch_bounds__(kStreamThreads) gemv_stream_kernel(LinearParams p) {
+template <int MT, int R, int J, int NT>
+__global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
   // activation codes as [MT][4][C] 16-byte units: unit u of a token row (its
   // inputs 16u .. 16u + 15) sits in plane u % 4 at index u / 4, so the lanes
   // of a warp, which hold consecutive chunks, read consecutive 16-byte words
   extern __shared__ uint4 gs_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.ldw / 16;                    // packed chunks per row
-  const int n0 = (blockIdx.x * (kStreamThreads / 32) + warp) * R;
+  const int n0 = (blockIdx.x * (NT / 32) + warp) * R;
   const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
   grid_launch_dependents();
 
@@ -228,7 +226,7 @@ __global__ void __launch_bounds__(kStreamThreads) gemv_stream_kernel(LinearParam
   // 2. activation codes, token scales and code sums
   if (!inputs_ready) grid_dependency_wait();
   const int units = p.K / 16;
-  for (int i = threadIdx.x; i < MT * units; i += kStreamThreads) {
+  for (int i = threadIdx.x; i < MT * units; i += NT) {
     const int m = i / units, u = i - m * units;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (m < p.M) v = *reinterpret_cast<const uint4*>(p.Xq + (size_t)m * p.K + 16 * u);

@@ -130,4 +130,42 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
   }
 }
 
+// ---------------------------------------------------------------------------
+// Canonical exchange layout TW2 <-> the device layout.  Both keep 16 codes in
+// each 32-bit word of a row: the device layout holds weight 4i + j of the word
+// at bits 8j + 2i (so (word >> 2i) & 0x03030303 gives four byte codes), TW2
+// at bits 8i + 2j (byte i = weights 4i .. 4i + 3, low bits first).  The
+// conversion transposes that 4 x 4 grid of 2-bit fields and is its own
+// inverse.  One thread per word.
+__device__ __forceinline__ uint32_t transpose_code_grid(uint32_t w) {
+  uint32_t o = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) o |= ((w >> (8 * j + 2 * i)) & 3u) << (8 * i + 2 * j);
+  return o;
+}
+
+// device layout (rows of ldw bytes) -> TW2 (rows of K / 4 bytes)
+__global__ void export_tw2_kernel(const uint32_t* __restrict__ packed, int N, int ldw_words,
+                                  int tw2_words, uint32_t* __restrict__ tw2) {
+  const int64_t total = (int64_t)N * tw2_words;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = i / tw2_words, w = i - n * tw2_words;
+    tw2[i] = transpose_code_grid(packed[n * ldw_words + w]);
+  }
+}
+
+// TW2 -> device layout; the padded words past K hold code 1 (t = 0)
+__global__ void import_tw2_kernel(const uint32_t* __restrict__ tw2, int N, int ldw_words,
+                                  int tw2_words, uint32_t* __restrict__ packed) {
+  const int64_t total = (int64_t)N * ldw_words;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t n = i / ldw_words, w = i - n * ldw_words;
+    packed[i] = w < tw2_words ? transpose_code_grid(tw2[n * tw2_words + w]) : 0x55555555u;
+  }
+}
+
 }  // namespace bitnet

@@ -117,6 +117,17 @@ def test_pack_rejects_bad_arguments():
     assert p(FAKE, 0, 8, 64, FAKE, FAKE, None, ws, None) == bn.BITNET_ERR_WORKSPACE
 
 
+def test_tw2_conversions_reject_bad_arguments():
+    for fn in (bn.library().bitnet_export_tw2, bn.library().bitnet_import_tw2):
+        assert fn(FAKE, 8, 60, FAKE2, None) == bn.BITNET_ERR_INVALID_ARG      # K % 16
+        assert fn(FAKE, 8, 32768, FAKE2, None) == bn.BITNET_ERR_INVALID_ARG   # K too large
+        assert fn(None, 8, 64, FAKE2, None) == bn.BITNET_ERR_INVALID_ARG
+        assert fn(FAKE, 8, 64, None, None) == bn.BITNET_ERR_INVALID_ARG
+        assert fn(MISALIGNED, 8, 64, FAKE2, None) == bn.BITNET_ERR_INVALID_ARG
+        assert fn(FAKE, -1, 64, FAKE2, None) == bn.BITNET_ERR_INVALID_ARG
+        assert fn(FAKE, 0, 64, FAKE2, None) == bn.BITNET_OK                   # no-op
+
+
 def test_ffn_rejects_bad_arguments():
     f = bn.library().bitnet_ffn
     ws = bn.bitnet_ffn_workspace_size(4, 64, 128, 0)

@@ -140,6 +140,24 @@ def test_pack_bf16_weights_and_edge_values():
     assert np.all(packed == 0x55)
 
 
+@pytest.mark.parametrize("N,K", [(1, 16), (7, 80), (300, 2560), (2560, 6912)])
+def test_tw2_export_and_import(N, K):
+    """The device layout converts to the canonical TW2 bytes of the oracle and
+    back, bit for bit (padding words of ragged rows come back as code 1)."""
+    W = synthetic.weight(np.random.default_rng(N * 3 + K), N, K)
+    packed, gamma = gpu_pack(W)
+    t = oracle.ternarize(W, oracle.absmean(W))
+    want = oracle.pack_tw2(t)
+    tw2 = torch.empty((N, K // 4), dtype=torch.uint8, device="cuda")
+    bn.bitnet_export_tw2(dev(packed), K, tw2)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(tw2.cpu().numpy(), want)
+    back = torch.full((N, bn.bitnet_packed_row_bytes(K)), 0xEE, dtype=torch.uint8, device="cuda")
+    bn.bitnet_import_tw2(dev(want), K, back)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(back.cpu().numpy(), oracle.pack(t))
+
+
 def test_pack_is_deterministic():
     W = synthetic.weight(np.random.default_rng(12), 2560, 2560)
     a = gpu_pack(W)
