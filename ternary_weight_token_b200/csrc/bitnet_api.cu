@@ -291,13 +291,15 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   const CUtensorMapSwizzle wswz =
       C::BK / 4 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   static_assert(C::BK / 4 == 64 || C::BK / 4 == 32, "packed stage width");
+  // GLU: 64 gate rows and 64 up rows per tile (two boxes), else 128 rows
+  const uint32_t wrows = C::GLU ? C::BM / 2 : C::BM;
   if (int rc = tensor_map_2d_u8(mw0, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
-                                C::BK / 4, C::BM, wswz))
+                                C::BK / 4, wrows, wswz))
     return rc;
   mw1 = mw0;
   if (C::GLU) {
     if (int rc = tensor_map_2d_u8(mw1, W1, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
-                                  C::BK / 4, C::BM, wswz))
+                                  C::BK / 4, wrows, wswz))
       return rc;
   }
   // Output through TMA stores when its rows are whole 16-byte units.
@@ -320,7 +322,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   p.tma_out = tma_out ? 1 : 0;
   p.M = lp.M; p.N = lp.N; p.K = lp.K;
   p.num_kb = (lp.K + C::BK - 1) / C::BK;
-  p.tiles_n = (lp.N + C::BM - 1) / C::BM;
+  p.tiles_n = (lp.N + C::TILE_N - 1) / C::TILE_N;
   const int tiles_m = (lp.M + C::BN - 1) / C::BN;
   p.num_tiles = p.tiles_n * tiles_m;
   p.xs = lp.xs; p.xrs = lp.xrs; p.gamma0 = lp.gamma; p.gamma1 = gamma1;
@@ -339,7 +341,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
 
 using TcPlain = TcConfig<128, 256, 4, false>;
 using TcSilu = TcConfig<128, 256, 4, false, true>;
-using TcGlu = TcConfig<64, 128, 4, true>;
+using TcGlu = TcConfig<128, 256, 4, true>;
 
 // Decode on the tensor cores: 128-row weight tiles, each split over K across a
 // cluster of S CTAs (S <= 8, every slice at most 896 inputs).  Returns

@@ -49,11 +49,15 @@ struct TcConfig {
   static constexpr int BN = BN_;            // tokens per tile (MMA N)
   static constexpr int BK = BK_;            // k per pipeline stage (multiple of 128)
   static constexpr int STAGES = STAGES_;
-  static constexpr bool GLU = GLU_;         // gate and up weights in one pass
+  // gate and up in one pass: the 128-row A tile stacks 64 gate rows over the
+  // same 64 rows of the up weights, so a tile yields 64 output features
+  static constexpr bool GLU = GLU_;
   static constexpr int BM = 128;            // weight rows per tile (MMA M, TMEM lanes)
+  static constexpr int TILE_N = GLU ? BM / 2 : BM;   // output features per tile
+  static constexpr int TOKF = GLU ? 2 : 1;  // dequant factors per token (gate, up)
   static constexpr int XSUB = BN * 128;     // one 128-byte-wide swizzled activation sub-tile
   static_assert(BK % 128 == 0 && BK <= 512, "BK");
-  static constexpr int NW = GLU ? 2 : 1;    // weight matrices per stage
+  static constexpr int NW = 1;              // weight tiles per stage
   static constexpr int X_STAGE = BN * BK;   // bytes of activation codes per stage
   static constexpr int W_STAGE = BM * BK / 4;  // bytes of packed weights per matrix per stage
   static constexpr int ACC_COLS = BN * NW;  // TMEM columns per accumulator buffer
@@ -69,7 +73,7 @@ struct TcConfig {
   static constexpr int OFF_W = OFF_X + STAGES * X_STAGE;
   static constexpr int OFF_OUT = OFF_W + STAGES * NW * W_STAGE;  // 4 warps x 2 buffers
   static constexpr int OFF_BAR = OFF_OUT + 4 * 2 * STAGE_OUT_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 7;
+  static constexpr int NUM_BARS = 3 * STAGES + 11;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
@@ -103,7 +107,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // per-token dequant factors (fp32 head, tail) and code sums of a tile,
   // computed once by the four epilogue warps; two buffers alternate between
   // consecutive tiles.  Static so they never alias the output staging buffers.
-  __shared__ __align__(16) float2 s_tok_f[2][C::NW * C::BN];
+  __shared__ __align__(16) float2 s_tok_f[2][C::TOKF * C::BN];
   __shared__ __align__(16) int s_tok_rs[2][C::BN];
 
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -118,6 +122,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* accempty = accfull + 2;            // accumulator drained    (4 epilogue warps)
   uint64_t* drain = accempty + 2;              // teardown drain
   uint64_t* tokbar = drain + 1;                // tile's token factors written (4 warps)
+  uint64_t* upready = tokbar + 2;              // GLU: up values of a chunk staged (2 warps)
+  uint64_t* upfree = upready + 2;              // GLU: staged up values consumed (2 warps)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -136,6 +142,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(drain, 2);
     mbar_init(&tokbar[0], 4);
     mbar_init(&tokbar[1], 4);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&upready[b], 2);
+      mbar_init(&upfree[b], 2);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -173,11 +183,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
           for (int xs = 0; xs < C::BK / 128; ++xs)
             tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
                         kb * C::BK + 128 * xs, tm * C::BN);
-          tma_load_2d(sw + (st * C::NW) * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
-                      tn * C::BM);
-          if (C::GLU)
-            tma_load_2d(sw + (st * C::NW + 1) * C::W_STAGE, &tm_w1, &full[st], kb * (C::BK / 4),
-                        tn * C::BM);
+          if (C::GLU) {                       // rows 0-63 gate, 64-127 up
+            tma_load_2d(sw + st * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
+                        tn * C::TILE_N);
+            tma_load_2d(sw + st * C::W_STAGE + (C::BM / 2) * (C::BK / 4), &tm_w1, &full[st],
+                        kb * (C::BK / 4), tn * C::TILE_N);
+          } else {
+            tma_load_2d(sw + st * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4), tn * C::BM);
+          }
         }
       }
     producer_done:
@@ -217,7 +230,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             const uint64_t bdesc =
                 make_sdesc_sw128(xaddr + (uint32_t)((j >> 2) * C::XSUB) + 32u * (j & 3));
             mma_i8_ts(d_col, a_col + 8u * j, bdesc, idesc, 1u);
-            if (C::GLU) mma_i8_ts(d_col + C::BN, a_col + (C::BK / 4) + 8u * j, bdesc, idesc, 1u);
           }
           tc_commit(&empty[st]);
         }
@@ -288,11 +300,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_arrive(&accempty[0]);
       mbar_arrive(&accempty[1]);
     }
-    uint32_t tcount = 0, chunk_count = 0;
+    uint32_t tcount = 0, chunk_count = 0, xcount = 0;
     for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
       const int m0 = tm * C::BN;
-      const int nq0 = tn * C::BM + 32 * q;       // first weight row of this warp
+      // first output feature of this warp (GLU: warps 0-1 hold gate rows,
+      // warps 2-3 the up rows of the same features)
+      const int nq0 = tn * C::TILE_N + 32 * (C::GLU ? (q & 1) : q);
       const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
       float2* tok_f = s_tok_f[ab];               // [NW][BN]
       int* tok_rs = s_tok_rs[ab];
@@ -324,7 +338,6 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int mc = m0 + 32 * c;              // first token of this chunk
         if (mc >= p.M) {                         // past the last token: only re-zero
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
-          if (C::GLU) tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c);
           continue;
         }
         if constexpr (!C::GLU) {
@@ -405,21 +418,40 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         float y[32];
         tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, v);
         if (C::GLU) {
-          uint32_t u[32];
-          tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c, u);
+          // up warps dequantise their rows and stage them token-major in the
+          // exchange buffer (the up warps' own output staging area); gate
+          // warps combine relu(g)^2 * u and store
           tmem_ld_wait();
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
-          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + C::BN + 32u * c);
+          const uint32_t xb = (uint32_t)(xcount & 1u), xuse = xcount >> 1;
+          ++xcount;
+          float* xbuf = reinterpret_cast<float*>(smem + C::OFF_OUT + 2 * 2 * C::STAGE_OUT_BYTES +
+                                                 xb * (C::BM / 2) * 32 * 4);
+          const int xrow = 32 * (q & 1) + lane;   // feature within the tile
+          if (q >= 2) {
+            if (!mbar_wait(&upfree[xb], (xuse & 1u) ^ 1u, abort_flag)) break;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int t = 32 * c + j;
+              const float2 fb = tok_f[C::BN + t];
+              xbuf[j * (C::BM / 2) + xrow] = dequant_dw((int)v[j] - tok_rs[t], fb.x, fb.y);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&upready[xb]);
+            continue;                            // up warps store nothing
+          }
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int t = 32 * c + j;
-            const int rs = tok_rs[t];
-            const float2 fa = tok_f[t], fb = tok_f[C::BN + t];
-            const float g = dequant_dw((int)v[j] - rs, fa.x, fa.y);
-            const float uu = dequant_dw((int)u[j] - rs, fb.x, fb.y);
-            const float a = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
-            y[j] = __fmul_rn(a, uu);
+            const float2 fa = tok_f[t];
+            const float g = dequant_dw((int)v[j] - tok_rs[t], fa.x, fa.y);
+            y[j] = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
           }
+          if (!mbar_wait(&upready[xb], xuse & 1u, abort_flag)) break;
+#pragma unroll
+          for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(y[j], xbuf[j * (C::BM / 2) + xrow]);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&upfree[xb]);
         } else {
           tmem_ld_wait();
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
