@@ -390,6 +390,69 @@ def bench_decode(torch, bn, device, reps=3):
     return out
 
 
+QKV_N = (2560, 640, 640)          # q, k, v projections of the 2B model (K = 2560)
+
+
+def bench_decode_qkv(torch, bn, device, reps=3):
+    """The q, k and v decode projections of one input: one bitnet_linear_multi
+    call per step (one launch) against three bitnet_linear calls, both as
+    independent projections in a CUDA graph over a pool of weight sets larger
+    than twice the L2."""
+    K = 2560
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    inp = synthetic.linear_inputs(max(DECODE_M), K, sum(QKV_N), seed=11)
+    W = torch.from_numpy(inp["W"]).to(device)
+    sets, row = [], 0
+    base = []
+    for N in QKV_N:
+        P, g, ws = bn.alloc_packed(N, K, device)
+        bn.bitnet_pack_weights(W[row:row + N].contiguous(), P, g, ws)
+        base.append((P, g))
+        row += N
+    del W
+    set_bytes = sum(P.numel() for P, _ in base)
+    pool = max(8, int(2 * l2 // set_bytes) + 2)
+    sets = [[(P.clone(), g) for P, g in base] for _ in range(pool)]
+    X = torch.from_numpy(inp["X"]).to(device)
+    out = []
+    for M in DECODE_M:
+        q, s, rs = bn.alloc_quant(M, K, device)
+        bn.bitnet_quant_act(X[:M].contiguous(), q, s, rs)
+        Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=device) for N in QKV_N]
+        epi = bn.BITNET_BF16 | bn.BITNET_LAUNCH_PDL_INPUTS
+        bytes_step = sum(decode_bytes(M, K, N) for N in QKV_N)
+
+        def fused(st, ws_):
+            bn.bitnet_linear_multi(q, s, rs, [P for P, _ in ws_], [g for _, g in ws_], K, Ys,
+                                   epilogue=epi, stream=st)
+
+        def separate(st, ws_):
+            for (P, g), Y in zip(ws_, Ys):
+                bn.bitnet_linear(q, s, rs, P, g, K, Y, epilogue=epi, stream=st)
+        rec = {"M": M, "K": K, "N": list(QKV_N), "weight_sets_in_pool": pool}
+        for name, fn in (("fused", fused), ("separate", separate)):
+            fn(None, sets[0])
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            stream = torch.cuda.Stream(device)
+            with torch.cuda.stream(stream):
+                graph.capture_begin(capture_error_mode="thread_local")
+                for ws_ in sets:
+                    fn(stream, ws_)
+                graph.capture_end()
+            torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            best = min(time_loop(torch, graph.replay, 4) for _ in range(reps))
+            rec["us_per_step_" + name] = best / (4 * pool) * 1e6
+            rec["GB_s_" + name] = bytes_step * 4 * pool / best / 1e9
+            del graph
+        out.append(rec)
+    del sets
+    torch.cuda.empty_cache()
+    return out
+
+
 def bench_ffn(torch, bn, device, iters=20):
     cfg = synthetic.WORKLOADS["ffn"].dims
     M, H, I = cfg["M"], cfg["H"], cfg["I"]
@@ -559,6 +622,7 @@ def run_b200(args, world, rank, local):
             d["frac_of_hbm_dependent"] = d["GB_s_dependent"] / peaks["hbm_gbs"]
         line["workloads"] = {
             "decode": dec,
+            "decode_qkv": bench_decode_qkv(torch, bn, device),
             "decode_peak_source": f"{peaks['source']} HBM copy {peaks['hbm_gbs']} GB/s",
             "ffn": bench_ffn(torch, bn, device),
             "hffn": bench_hffn(torch, bn, device),
@@ -603,7 +667,7 @@ def run_only(args, local):
         out = decode_single(torch, bn, device, M, K, N, max(1, args.steps))
     else:
         fn = {"decode": bench_decode, "ffn": bench_ffn, "hffn": bench_hffn,
-              "tiny": bench_tiny}[args.only]
+              "tiny": bench_tiny, "qkv": bench_decode_qkv}[args.only]
         out = fn(torch, bn, device)
     print(json.dumps({"only": args.only, "result": out}), flush=True)
     return 0
@@ -620,7 +684,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=None,
                     help="with --impl reference: target seconds of oracle work per step")
-    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny"), default=None,
+    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny", "qkv"), default=None,
                     help="time one secondary workload and print its JSON (profiling aid)")
     ap.add_argument("--decode-shape", default=None,
                     help="with --only decode: one 'M,K,N' case, no CUDA graph")

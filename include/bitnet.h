@@ -197,6 +197,23 @@ BITNET_API int bitnet_linear(const int8_t *Xq, const float *x_scale, const int32
                   void *Y, int epilogue, const void *residual,
                   bitnet_stream_t stream);
 
+/* Several projections of one quantised input in one call -- the q, k and v
+ * projections of an attention block (2560 -> 2560 + 640 + 640 in the 2B
+ * model, nnterp "bitnet", "Printout"), or gate and up -- as bitnet_linear()
+ * for each, with one launch for all of them on the decode path (M <= 16).
+ *   count       projections, 1..4
+ *   packed[i], gamma[i], N[i], Y[i]
+ *               weight i [N[i]][K] (device layout) with its gamma, and its
+ *               output [M][N[i]]; host arrays of device pointers
+ *   epilogue    as bitnet_linear() without BITNET_EPI_RESIDUAL
+ * M > 16 runs the projections as consecutive prefill GEMMs.
+ * Errors: INVALID_ARG, UNSUPPORTED (residual requested), CUDA. */
+BITNET_API int bitnet_linear_multi(const int8_t *Xq, const float *x_scale,
+                                   const int32_t *x_rowsum, int count,
+                                   const uint8_t *const *packed, const float *const *gamma,
+                                   const int *N, int M, int K, void *const *Y, int epilogue,
+                                   bitnet_stream_t stream);
+
 /* Workspace bytes bitnet_ffn() needs. */
 BITNET_API size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant);
 

@@ -49,6 +49,7 @@ from ._binding import (  # noqa: F401
     bitnet_last_error,
     bitnet_import_tw2,
     bitnet_linear,
+    bitnet_linear_multi,
     bitnet_pack_weights,
     bitnet_pack_workspace_size,
     bitnet_packed_row_bytes,

@@ -55,6 +55,7 @@ def library():
         "bitnet_pack_workspace_size": (S, [I, I]),
         "bitnet_pack_weights": (I, [P, I, I, I, P, P, P, S, P]),
         "bitnet_export_tw2": (I, [P, I, I, P, P]),
+        "bitnet_linear_multi": (I, [P, P, P, I, P, P, P, I, I, P, I, P]),
         "bitnet_import_tw2": (I, [P, I, I, P, P]),
         "bitnet_quant_act": (I, [P, I, I, I, I, P, F, P, P, P, P]),
         "bitnet_linear": (I, [P, P, P, P, P, I, I, I, P, I, P, P]),
@@ -137,6 +138,21 @@ def bitnet_pack_weights(W, packed, gamma, workspace, stream=None):
     _check(library().bitnet_pack_weights(_ptr(W), _dtype(W), N, K, _ptr(packed), _ptr(gamma),
                                          _ptr(workspace), workspace.numel() * workspace.element_size(),
                                          _stream(stream)))
+
+
+def bitnet_linear_multi(Xq, x_scale, x_rowsum, packed, gamma, K, Y, epilogue=None, stream=None):
+    """Several projections of one quantised input: packed, gamma and Y are
+    lists (one entry per projection, outputs [M][N_i])."""
+    count = len(packed)
+    if not (len(gamma) == len(Y) == count):
+        raise ValueError("packed, gamma and Y need one entry per projection")
+    ptrs = lambda ts: (ctypes.c_void_p * count)(*[_ptr(t) for t in ts])
+    Ns = (ctypes.c_int * count)(*[int(y.shape[1]) for y in Y])
+    if epilogue is None:
+        epilogue = _dtype(Y[0])
+    _check(library().bitnet_linear_multi(_ptr(Xq), _ptr(x_scale), _ptr(x_rowsum), count,
+                                         ptrs(packed), ptrs(gamma), Ns, Xq.shape[0], int(K),
+                                         ptrs(Y), int(epilogue), _stream(stream)))
 
 
 def bitnet_export_tw2(packed, K, tw2, stream=None):

@@ -354,20 +354,34 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   const int s_min = (units + 13) / 14;                    // ceil(units / S) <= 14
   const int s_max = units < kDecMaxCluster ? units : kDecMaxCluster;
   if (s_min > s_max) return BITNET_ERR_UNSUPPORTED;
-  const int tiles = (lp.N + 127) / 128;
+  // every projection of the call: its 128-row tiles and packed-weight map
+  DecParams p;
+  DecMaps maps;
+  int tiles = 0;
+  p.nseg = lp.nseg;
+  for (int i = 0; i < lp.nseg; ++i) {
+    const int Ni = lp.seg_row0[i + 1] - lp.seg_row0[i];
+    p.seg_tile0[i] = tiles;
+    p.seg_N[i] = Ni;
+    p.seg_gamma[i] = lp.seg_gamma[i];
+    p.seg_Y[i] = lp.seg_Y[i];
+    if (int rc = tensor_map_2d_u8(maps.w[i], lp.seg_W[i], (uint64_t)lp.ldw, (uint64_t)Ni,
+                                  (uint64_t)lp.ldw, kDecChunkK / 4, 128,
+                                  CU_TENSOR_MAP_SWIZZLE_NONE))
+      return rc;
+    tiles += (Ni + 127) / 128;
+  }
+  for (int i = lp.nseg; i <= kMaxSegments; ++i) p.seg_tile0[i] = tiles;
+  for (int i = lp.nseg; i < kMaxSegments; ++i) maps.w[i] = maps.w[0];
   int S = s_min;
   while (S < s_max && tiles * S < di.sms) ++S;
-  CUtensorMap mx, mw;
+  CUtensorMap mx;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 kDecTokens, CU_TENSOR_MAP_SWIZZLE_128B))
     return rc;
-  if (int rc = tensor_map_2d_u8(mw, lp.W, (uint64_t)lp.ldw, (uint64_t)lp.N, (uint64_t)lp.ldw,
-                                kDecChunkK / 4, 128, CU_TENSOR_MAP_SWIZZLE_NONE))
-    return rc;
-  DecParams p;
-  p.M = lp.M; p.N = lp.N; p.K = lp.K; p.units = units;
-  p.xs = lp.xs; p.xrs = lp.xrs; p.gamma = lp.gamma;
-  p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type;
+  p.M = lp.M; p.K = lp.K; p.units = units;
+  p.xs = lp.xs; p.xrs = lp.xrs;
+  p.resid = lp.resid; p.out_type = lp.out_type;
   p.flags = lp.flags & ~LAUNCH_PDL;     // keeps LAUNCH_PDL_INPUTS for the kernel
   static bool attr_set = false;
   if (!attr_set) {
@@ -389,7 +403,7 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   attrs[1].val.programmaticStreamSerializationAllowed = (lp.flags & LAUNCH_PDL) ? 1 : 0;
   cfg.attrs = attrs;
   cfg.numAttrs = 2;
-  BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, gemv_tc_kernel, mx, mw, p));
+  BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, gemv_tc_kernel, mx, maps, p));
   return BITNET_OK;
 }
 
@@ -432,20 +446,43 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
 }
 
+// Projection i of a call as a call of its own.
+LinearParams segment_params(const LinearParams& p, int i) {
+  LinearParams q = p;
+  q.W = p.seg_W[i];
+  q.gamma = p.seg_gamma[i];
+  q.Y = p.seg_Y[i];
+  q.N = p.seg_row0[i + 1] - p.seg_row0[i];
+  single_segment(q);
+  return q;
+}
+
 int launch_linear(const LinearParams& p, cudaStream_t st) {
   // 1-2 tokens: the dp4a streaming kernel (measured faster than the cluster
   // tensor-core path there; from 4 tokens on, its dp4a work and shared-memory
-  // reads sit on the critical path of dependent calls)
+  // reads sit on the critical path of dependent calls).  Both decode kernels
+  // run every projection of the call in one launch.
   if (p.M <= 2 && p.K % 64 == 0 && p.ldw / 16 <= 32 * 8) return launch_gemv_stream(p, st);
   if (p.M <= 16) {
     const int rc = launch_gemv_tc(p, st);
     if (rc != BITNET_ERR_UNSUPPORTED) return rc;
-    LinearParams q = p;
-    q.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
-    return launch_gemv(q, st);                 // inputs too long for the cluster split
   }
-  if (p.flags & EPI_SILU) return launch_tc_cfg<TcSilu>(p, nullptr, nullptr, st);
-  return launch_tc_cfg<TcPlain>(p, nullptr, nullptr, st);
+  // one launch per projection: the prefill GEMM, or decode inputs too long
+  // for the cluster split (the plain dp4a kernel)
+  for (int i = 0; i < p.nseg; ++i) {
+    LinearParams q = segment_params(p, i);
+    int rc;
+    if (q.M <= 16) {
+      q.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
+      rc = launch_gemv(q, st);
+    } else if (q.flags & EPI_SILU) {
+      rc = launch_tc_cfg<TcSilu>(q, nullptr, nullptr, st);
+    } else {
+      rc = launch_tc_cfg<TcPlain>(q, nullptr, nullptr, st);
+    }
+    if (rc) return rc;
+  }
+  return BITNET_OK;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -616,6 +653,46 @@ int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsu
   p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = residual;
   if (p.flags & LAUNCH_PDL_INPUTS) p.flags |= LAUNCH_PDL;
   if (M > 16) p.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
+  single_segment(p);
+  return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_linear_multi(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsum,
+                        int count, const uint8_t* const* packed, const float* const* gamma,
+                        const int* N, int M, int K, void* const* Y, int epilogue,
+                        bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (count < 1 || count > kMaxSegments)
+    return fail(BITNET_ERR_INVALID_ARG, "count=%d must be in [1, %d]", count, kMaxSegments);
+  if (packed == nullptr || gamma == nullptr || N == nullptr || Y == nullptr)
+    return fail(BITNET_ERR_INVALID_ARG, "null pointer array");
+  if (epilogue & BITNET_EPI_RESIDUAL)
+    return fail(BITNET_ERR_UNSUPPORTED, "no residual for several projections");
+  int total = 0;
+  for (int i = 0; i < count; ++i) {
+    if (N[i] < 1) return fail(BITNET_ERR_INVALID_ARG, "N[%d]=%d must be >= 1", i, N[i]);
+    if (int rc = validate_linear(Xq, x_scale, x_rowsum, packed[i], gamma[i], M, N[i], K, Y[i],
+                                 epilogue, nullptr))
+      return rc;
+    if (total > (1 << 30) - N[i]) return fail(BITNET_ERR_INVALID_ARG, "too many rows");
+    total += N[i];
+  }
+  if (M == 0) return BITNET_OK;
+  LinearParams p;
+  p.Xq = Xq; p.xs = x_scale; p.xrs = x_rowsum; p.W = packed[0]; p.gamma = gamma[0];
+  p.M = M; p.N = total; p.K = K; p.ldw = (int)bitnet_packed_row_bytes(K);
+  p.Y = Y[0]; p.out_type = epilogue & BITNET_EPI_TYPE_MASK;
+  p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = nullptr;
+  if (p.flags & LAUNCH_PDL_INPUTS) p.flags |= LAUNCH_PDL;
+  if (M > 16) p.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
+  p.nseg = count;
+  p.seg_row0[0] = 0;
+  for (int i = 0; i < count; ++i) {
+    p.seg_row0[i + 1] = p.seg_row0[i] + N[i];
+    p.seg_W[i] = packed[i];
+    p.seg_gamma[i] = gamma[i];
+    p.seg_Y[i] = Y[i];
+  }
   return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -694,6 +771,8 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   p2.Xq = hq; p2.xs = hs; p2.xrs = hrs; p2.W = W_down; p2.gamma = gamma_down;
   p2.M = M; p2.N = H; p2.K = I; p2.ldw = (int)bitnet_packed_row_bytes(I);
   p2.Y = Y; p2.out_type = y_dtype == BITNET_BF16 ? OUT_BF16 : OUT_F32;
+  single_segment(p1);
+  single_segment(p2);
 
   if (variant == BITNET_FFN_RELU2_GLU) {
     if (int rc = launch_quant(X, xbf, M, H, PRE_RMSNORM, pre_norm_gain, eps, xq, xs, xrs, st))

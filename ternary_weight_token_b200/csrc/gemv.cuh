@@ -22,6 +22,8 @@ namespace bitnet {
 enum { OUT_F32 = 0, OUT_BF16 = 1, OUT_I32 = 2 };
 enum { EPI_RESIDUAL = 0x10, EPI_SILU = 0x20, LAUNCH_PDL = 0x100, LAUNCH_PDL_INPUTS = 0x200 };
 
+constexpr int kMaxSegments = 4;
+
 struct LinearParams {
   const int8_t* Xq;
   const float* xs;
@@ -33,7 +35,35 @@ struct LinearParams {
   int out_type;
   int flags;
   const void* resid;
+  // Projections sharing the activations (the decode kernels run them in one
+  // launch): projection i owns rows [seg_row0[i], seg_row0[i + 1]) of the
+  // concatenated output rows, N above being their total.  A single
+  // projection is the table {0, N} with W, gamma, Y.
+  int nseg;
+  int seg_row0[kMaxSegments + 1];
+  const uint8_t* seg_W[kMaxSegments];
+  const float* seg_gamma[kMaxSegments];
+  void* seg_Y[kMaxSegments];
 };
+
+__host__ __device__ inline void single_segment(LinearParams& p) {
+  p.nseg = 1;
+  p.seg_row0[0] = 0;
+  p.seg_row0[1] = p.N;
+  p.seg_W[0] = p.W;
+  p.seg_gamma[0] = p.gamma;
+  p.seg_Y[0] = p.Y;
+}
+
+// Projection of concatenated row n, and its row within that projection.
+__device__ __forceinline__ int segment_of(const LinearParams& p, int n, int& local) {
+  int s = 0;
+#pragma unroll
+  for (int i = 1; i < kMaxSegments; ++i)
+    if (i < p.nseg && n >= p.seg_row0[i]) s = i;
+  local = n - p.seg_row0[s];
+  return s;
+}
 
 // Exact int -> float for |v| < 2^22 with two ALU/FMA ops (no conversion
 // unit): place v in the mantissa of 1.5 * 2^23 and subtract 1.5 * 2^23.
@@ -213,14 +243,19 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
   const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
   grid_launch_dependents();
 
-  // 1. every packed chunk of this warp's rows, in flight at once
+  // 1. every packed chunk of this warp's rows, in flight at once (rows are
+  // the concatenated rows of the call's projections)
   uint4 w[J];
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int f = lane + 32 * j;
     const int r = f / C, c = f - r * C;
     w[j] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // t = 0
-    if (r < R && n0 + r < p.N) w[j] = ld_stream_v4(p.W + (size_t)(n0 + r) * p.ldw + 16 * c);
+    if (r < R && n0 + r < p.N) {
+      int nl;
+      const int sg = segment_of(p, n0 + r, nl);
+      w[j] = ld_stream_v4(p.seg_W[sg] + (size_t)nl * p.ldw + 16 * c);
+    }
   }
 
   // 2. activation codes, token scales and code sums
@@ -236,8 +271,6 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
   const bool tok = lane < p.M;
   const float s_m = tok ? p.xs[mt] : 1.0f;
   const int rs_m = tok ? p.xrs[mt] : 0;
-  float fh_m = 0.0f, fl_m = 0.0f;
-  if (p.out_type != OUT_I32) dequant_factor(__ldg(p.gamma), s_m, fh_m, fl_m);
   __syncthreads();
 
   // 3. unsigned codes x signed activations, per row and token
@@ -276,7 +309,8 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
     }
   }
 
-  // 4. warp sums; lane r * MT + m holds row r, token m
+  // 4. warp sums; lane r * MT + m holds row r, token m, and forms its own
+  // dequant factor (the row's projection sets gamma)
   float y = 0.0f;
   int yint = 0;
   int my_r = -1, my_m = 0;
@@ -288,23 +322,33 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       const int rs = __shfl_sync(0xffffffffu, rs_m, m);
-      const float fh = __shfl_sync(0xffffffffu, fh_m, m);
-      const float fl = __shfl_sync(0xffffffffu, fl_m, m);
+      const float sm = __shfl_sync(0xffffffffu, s_m, m);
       if (lane == r * MT + m) {
         my_r = r;
         my_m = m;
         yint = v - rs;
-        y = p.out_type == OUT_I32 ? 0.0f : dequant_dw(yint, fh, fl);
+        y = sm;                                  // the token's scale, for now
       }
     }
-  if (inputs_ready) grid_dependency_wait();    // Y may still be read or written before
   const int n = n0 + my_r;
-  if (my_r >= 0 && my_m < p.M && n < p.N) {
-    const size_t idx = (size_t)my_m * p.N + n;
+  int nl = 0, sg = 0;
+  const bool valid = my_r >= 0 && my_m < p.M && n < p.N;
+  if (valid) {
+    sg = segment_of(p, n, nl);
+    if (p.out_type != OUT_I32) {
+      float fh, fl;
+      dequant_factor(__ldg(p.seg_gamma[sg]), y, fh, fl);
+      y = dequant_dw(yint, fh, fl);
+    }
+  }
+  if (inputs_ready) grid_dependency_wait();    // Y may still be read or written before
+  if (valid) {
+    const int Ns = p.seg_row0[sg + 1] - p.seg_row0[sg];
+    const size_t idx = (size_t)my_m * Ns + nl;
     if (p.out_type == OUT_I32)
-      reinterpret_cast<int32_t*>(p.Y)[idx] = yint;
+      reinterpret_cast<int32_t*>(p.seg_Y[sg])[idx] = yint;
     else
-      store_value(p.Y, p.resid, idx, y, p.out_type, p.flags);
+      store_value(p.seg_Y[sg], p.resid, idx, y, p.out_type, p.flags);
   }
 }
 

@@ -48,15 +48,25 @@ constexpr int kDecTmemCols = 256;
 constexpr int kDecMinSmem = 80 * 1024;          // at most two CTAs per SM
 
 struct DecParams {
-  int M, N, K;
+  int M, K;
   int units;              // K / 64
   const float* xs;
   const int32_t* xrs;
-  const float* gamma;
-  void* Y;
   const void* resid;
   int out_type;
   int flags;
+  // projections sharing the activations: projection i owns the 128-row
+  // tiles [seg_tile0[i], seg_tile0[i + 1]) and has seg_N[i] rows
+  int nseg;
+  int seg_tile0[kMaxSegments + 1];
+  int seg_N[kMaxSegments];
+  const float* seg_gamma[kMaxSegments];
+  void* seg_Y[kMaxSegments];
+};
+
+// packed-weight tensor maps, one per projection
+struct DecMaps {
+  CUtensorMap w[kMaxSegments];
 };
 
 struct DecSmem {
@@ -162,7 +172,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
 
 __global__ void __launch_bounds__(kDecThreads, 1)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_w, DecParams p) {
+                   const __grid_constant__ DecMaps maps, DecParams p) {
   extern __shared__ uint8_t dec_smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(dec_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -180,7 +190,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const uint32_t csize = cluster_nctarank();
   const int tile = blockIdx.x / (int)csize;               // 128-row weight tile
-  const int n0 = tile * 128;
+  int sg = 0;                                             // its projection
+#pragma unroll
+  for (int i = 1; i < kMaxSegments; ++i)
+    if (i < p.nseg && tile >= p.seg_tile0[i]) sg = i;
+  const int n0 = (tile - p.seg_tile0[sg]) * 128;          // first row within it
+  const int Ns = p.seg_N[sg];
+  const CUtensorMap* tm_w = &maps.w[sg];
   int k0, ks;
   dec_slice(p.units, (int)csize, (int)rank, k0, ks);
   const int chunks = (ks + kDecChunkK - 1) / kDecChunkK;
@@ -215,10 +231,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == 0) {
     if (lane == 0) {
       // weights do not depend on the preceding kernel: load them first
-      tma_prefetch_desc(&tm_w);
+      tma_prefetch_desc(tm_w);
       for (int c = 0; c < chunks; ++c) {
         mbar_arrive_expect_tx(&wfull[c], DecSmem::W_CHUNK);
-        tma_load_2d(sw + c * DecSmem::W_CHUNK, &tm_w, &wfull[c], (k0 + c * kDecChunkK) / 4, n0);
+        tma_load_2d(sw + c * DecSmem::W_CHUNK, tm_w, &wfull[c], (k0 + c * kDecChunkK) / 4, n0);
       }
       if (!inputs_ready) grid_dependency_wait();   // activation codes from the previous kernel
       tma_prefetch_desc(&tm_x);
@@ -303,7 +319,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       // LAUNCH_PDL_INPUTS before the wait for the preceding grid, so only
       // the stores follow it.
       if (!inputs_ready) grid_dependency_wait();
-      const float g = __ldg(p.gamma);
+      const float g = __ldg(p.seg_gamma[sg]);
       const int mt = lane < kDecTokens ? lane : 0;
       const bool tok = lane < p.M;
       const float s_m = tok ? __ldg(p.xs + mt) : 1.0f;
@@ -331,15 +347,15 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         y[m] = p.out_type == OUT_I32 ? __int_as_float(acc[m]) : dequant_dw(acc[m], fh, fl);
       }
       if (inputs_ready) grid_dependency_wait();  // Y may still be read or written before
-      if (all_in && n < p.N) {
+      if (all_in && n < Ns) {
 #pragma unroll
         for (int m = 0; m < kDecTokens; ++m) {
           if (m < p.M) {
-            const size_t idx = (size_t)m * p.N + n;
+            const size_t idx = (size_t)m * Ns + n;
             if (p.out_type == OUT_I32)
-              reinterpret_cast<int32_t*>(p.Y)[idx] = __float_as_int(y[m]);
+              reinterpret_cast<int32_t*>(p.seg_Y[sg])[idx] = __float_as_int(y[m]);
             else
-              store_value(p.Y, p.resid, idx, y[m], p.out_type, p.flags);
+              store_value(p.seg_Y[sg], p.resid, idx, y[m], p.out_type, p.flags);
           }
         }
       }

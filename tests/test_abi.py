@@ -128,6 +128,32 @@ def test_tw2_conversions_reject_bad_arguments():
         assert fn(FAKE, 0, 64, FAKE2, None) == bn.BITNET_OK                   # no-op
 
 
+def test_linear_multi_rejects_bad_arguments():
+    import ctypes
+    f = bn.library().bitnet_linear_multi
+    arr = lambda *v: (ctypes.c_void_p * len(v))(*v)
+    ns = lambda *v: (ctypes.c_int * len(v))(*v)
+    P = arr(FAKE, FAKE2)
+    G = arr(FAKE, FAKE)
+    Ys = arr(FAKE2, FAKE2)
+    ok = f(FAKE, FAKE, FAKE, 2, P, G, ns(64, 32), 0, 64, Ys, bn.BITNET_F32, None)
+    assert ok == bn.BITNET_OK                                         # M = 0: validated no-op
+    assert f(FAKE, FAKE, FAKE, 0, P, G, ns(64, 32), 4, 64, Ys, bn.BITNET_F32, None) == \
+        bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 5, P, G, ns(64, 32), 4, 64, Ys, bn.BITNET_F32, None) == \
+        bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2, None, G, ns(64, 32), 4, 64, Ys, bn.BITNET_F32, None) == \
+        bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2, P, G, ns(64, 0), 4, 64, Ys, bn.BITNET_F32, None) == \
+        bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2, arr(FAKE, None), G, ns(64, 32), 4, 64, Ys, bn.BITNET_F32,
+             None) == bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2, P, G, ns(64, 32), 4, 60, Ys, bn.BITNET_F32, None) == \
+        bn.BITNET_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2, P, G, ns(64, 32), 4, 64, Ys,
+             bn.BITNET_F32 | bn.BITNET_EPI_RESIDUAL, None) == bn.BITNET_ERR_UNSUPPORTED
+
+
 def test_ffn_rejects_bad_arguments():
     f = bn.library().bitnet_ffn
     ws = bn.bitnet_ffn_workspace_size(4, 64, 128, 0)

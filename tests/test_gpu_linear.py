@@ -191,6 +191,37 @@ def test_decode_independent_projections_overlap():
     assert bn.bitnet_check_device_error() == bn.BITNET_OK
 
 
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 16, 64])
+@pytest.mark.parametrize("Ns", [(2560, 640, 640), (300, 77, 640, 1000)])
+def test_linear_multi_matches_separate_projections(M, Ns):
+    """bitnet_linear_multi: the q/k/v shapes of the 2B model (and ragged
+    widths, four projections) in one call, each output bit-exact (int32) and
+    equal to the bf16 rounding of the oracle, on the dp4a (M <= 2), cluster
+    tensor-core (M <= 16) and prefill (M = 64) paths."""
+    K = 2560
+    rng_w, rng_x = synthetic.streams(sum(Ns) + M, 2)
+    X = synthetic.activations(rng_x, M, K)
+    q, s, rs = oracle.quant_act(X)
+    packs = []
+    for N in Ns:
+        g, T, P = oracle.quantize_weights(synthetic.weight(rng_w, N, K))
+        packs.append((N, g, T, dev(P), dev(np.array([g], np.float32))))
+    for out in (torch.int32, torch.bfloat16):
+        Ys = [torch.empty((M, N), dtype=out, device="cuda") for N, *_ in packs]
+        flags = bn.BITNET_I32 if out == torch.int32 else bn.BITNET_BF16
+        bn.bitnet_linear_multi(dev(q), dev(s), dev(rs), [pk[3] for pk in packs],
+                               [pk[4] for pk in packs], K, Ys,
+                               epilogue=flags | (bn.BITNET_LAUNCH_PDL if M <= 16 else 0))
+        torch.cuda.synchronize()
+        for Y, (N, g, T, _, _) in zip(Ys, packs):
+            if out == torch.int32:
+                np.testing.assert_array_equal(Y.cpu().numpy(), oracle.contract(q, T))
+            else:
+                want = oracle.dequant(oracle.contract(q, T), s, g)
+                assert_bf16_matches(Y.float().cpu().numpy(), want, what=f"multi N={N}")
+    assert bn.bitnet_check_device_error() == bn.BITNET_OK
+
+
 @pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 6912), (6912, 2560)])
 def test_decode_shapes_all_m(K, N):
     """The 2B-model decode shapes for every token count 1..16 (cluster split-K
