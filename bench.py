@@ -522,6 +522,37 @@ def bench_tiny(torch, bn, device, iters=200):
             "note": "quant + linear, launch-latency bound"}
 
 
+def bench_online(torch, bn, device, iters=20):
+    """Online ternarisation: the bf16 master weights re-ternarised every
+    forward (absmean pass + pack) ahead of the prefill projection, against
+    the same projection on stored packed weights.  M = 4096, K = 2560,
+    N = 6912, RMSNorm prelude, bf16 out."""
+    M, K, N = PREFILL_M, 2560, 6912
+    inp = synthetic.linear_inputs(M, K, N, seed=0)
+    Wb = torch.from_numpy(inp["W"]).to(device).to(torch.bfloat16)
+    X = torch.from_numpy(inp["X"]).to(device)
+    P, g, ws = bn.alloc_packed(N, K, device)
+    q, s, rs = bn.alloc_quant(M, K, device)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+
+    def pack():
+        bn.bitnet_pack_weights(Wb, P, g, ws)
+
+    def project():
+        bn.bitnet_quant_act(X, q, s, rs, prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
+        bn.bitnet_linear(q, s, rs, P, g, K, Y)
+
+    def online():
+        pack()
+        project()
+    out = {"M": M, "K": K, "N": N, "weights": "bf16 master copy, re-packed per forward"}
+    for name, fn in (("pack_us", pack), ("stored_weights_us", project), ("online_us", online)):
+        for _ in range(3):
+            fn()
+        out[name] = time_loop(torch, fn, iters) / iters * 1e6
+    return out
+
+
 def run_b200(args, world, rank, local):
     import torch
     if not torch.cuda.is_available():
@@ -627,6 +658,7 @@ def run_b200(args, world, rank, local):
             "ffn": bench_ffn(torch, bn, device),
             "hffn": bench_hffn(torch, bn, device),
             "tiny": bench_tiny(torch, bn, device),
+            "online_ternarisation": bench_online(torch, bn, device),
         }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -667,7 +699,7 @@ def run_only(args, local):
         out = decode_single(torch, bn, device, M, K, N, max(1, args.steps))
     else:
         fn = {"decode": bench_decode, "ffn": bench_ffn, "hffn": bench_hffn,
-              "tiny": bench_tiny, "qkv": bench_decode_qkv}[args.only]
+              "tiny": bench_tiny, "qkv": bench_decode_qkv, "online": bench_online}[args.only]
         out = fn(torch, bn, device)
     print(json.dumps({"only": args.only, "result": out}), flush=True)
     return 0
@@ -684,7 +716,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=None,
                     help="with --impl reference: target seconds of oracle work per step")
-    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny", "qkv"), default=None,
+    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny", "qkv", "online"),
+                    default=None,
                     help="time one secondary workload and print its JSON (profiling aid)")
     ap.add_argument("--decode-shape", default=None,
                     help="with --only decode: one 'M,K,N' case, no CUDA graph")
