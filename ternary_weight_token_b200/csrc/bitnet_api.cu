@@ -549,13 +549,13 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
   const bool bf16 = w_dtype == BITNET_BF16;
   const long long count = (long long)N * K;
   double* partials = reinterpret_cast<double*>(workspace);
-  if (bf16)
-    absmean_partial_kernel<true><<<kPackPartialBlocks, kPackThreads, 0, st>>>(W, count, partials);
-  else
-    absmean_partial_kernel<false><<<kPackPartialBlocks, kPackThreads, 0, st>>>(W, count, partials);
-  BN_CHECK_CUDA(cudaGetLastError());
-  absmean_final_kernel<<<1, kPackThreads, 0, st>>>(partials, kPackPartialBlocks, count, gamma);
-  BN_CHECK_CUDA(cudaGetLastError());
+  if (int rc = launch_pdl(bf16 ? absmean_partial_kernel<true> : absmean_partial_kernel<false>,
+                          dim3(kPackPartialBlocks), dim3(kPackThreads), 0, st, W, count,
+                          partials))
+    return rc;
+  if (int rc = launch_pdl(absmean_final_kernel, dim3(1), dim3(kPackThreads), 0, st,
+                          (const double*)partials, (int)kPackPartialBlocks, count, gamma))
+    return rc;
   if (N == 0) return BITNET_OK;
   const int ldw = (int)bitnet_packed_row_bytes(K);
   const long long words = (long long)N * (ldw / 4);
@@ -563,12 +563,8 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
   if (int rc = device_info(di)) return rc;
   long long blocks = (words + kPackThreads - 1) / kPackThreads;
   if (blocks > (long long)di.sms * 32) blocks = (long long)di.sms * 32;
-  if (bf16)
-    pack_kernel<true><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
-  else
-    pack_kernel<false><<<(int)blocks, kPackThreads, 0, st>>>(W, N, K, ldw, gamma, packed);
-  BN_CHECK_CUDA(cudaGetLastError());
-  return BITNET_OK;
+  return launch_pdl(bf16 ? pack_kernel<true> : pack_kernel<false>, dim3((int)blocks),
+                    dim3(kPackThreads), 0, st, W, N, K, ldw, (const float*)gamma, packed);
 }
 
 static int validate_tw2(const void* a, const void* b, int N, int K) {

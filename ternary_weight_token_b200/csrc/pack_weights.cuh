@@ -6,7 +6,8 @@
 // checkpoint stores them ternary, four to a byte, with a weight_scale.
 // "BitNet b1.58 2B4T", "Model Details": absmean quantisation.
 //
-// Three launches on the caller's stream:
+// Three launches on the caller's stream (with programmatic dependent launch:
+// each waits for its predecessor before touching global memory):
 //   1. absmean_partial: a fixed grid sums |W| in fp64, one partial per CTA in
 //      a fixed order (deterministic run to run);
 //   2. absmean_final: one CTA adds the partials in a fixed order and writes
@@ -29,33 +30,69 @@ __global__ void __launch_bounds__(kPackThreads) absmean_partial_kernel(const voi
                                                                        double* partials) {
   __shared__ double red[33];
   double acc = 0.0;
+  grid_launch_dependents();       // launched with programmatic dependent launch:
+  grid_dependency_wait();         // no global access before the preceding grid completed
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   if (BF16) {
+    // four independent 16-byte loads in flight per thread, four partial sums
+    // added in a fixed order
     const uint4* v8 = reinterpret_cast<const uint4*>(W);
     const long long nv = count / 8;
-    for (long long i = t0; i < nv; i += stride) {
+    double a4[4] = {0.0, 0.0, 0.0, 0.0};
+    long long i = t0;
+    for (; i + 3 * stride < nv; i += 4 * stride) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld_stream_v4(v8 + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          a4[u] += fabs((double)bf16_bits_to_f32(w[j] & 0xffffu));
+          a4[u] += fabs((double)bf16_bits_to_f32(w[j] >> 16));
+        }
+      }
+    }
+    for (; i < nv; i += stride) {
       uint4 v = v8[i];
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        acc += fabs((double)bf16_bits_to_f32(w[j] & 0xffffu));
-        acc += fabs((double)bf16_bits_to_f32(w[j] >> 16));
+        a4[0] += fabs((double)bf16_bits_to_f32(w[j] & 0xffffu));
+        a4[0] += fabs((double)bf16_bits_to_f32(w[j] >> 16));
       }
     }
+    acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
     const uint16_t* s = reinterpret_cast<const uint16_t*>(W);
     for (long long i = nv * 8 + t0; i < count; i += stride)
       acc += fabs((double)bf16_bits_to_f32(s[i]));
   } else {
     const float4* v4 = reinterpret_cast<const float4*>(W);
     const long long nv = count / 4;
-    for (long long i = t0; i < nv; i += stride) {
-      float4 v = v4[i];
-      acc += fabs((double)v.x);
-      acc += fabs((double)v.y);
-      acc += fabs((double)v.z);
-      acc += fabs((double)v.w);
+    double a4[4] = {0.0, 0.0, 0.0, 0.0};
+    long long i = t0;
+    for (; i + 3 * stride < nv; i += 4 * stride) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = ld_stream_v4(v4 + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a4[u] += fabs((double)__uint_as_float(v[u].x));
+        a4[u] += fabs((double)__uint_as_float(v[u].y));
+        a4[u] += fabs((double)__uint_as_float(v[u].z));
+        a4[u] += fabs((double)__uint_as_float(v[u].w));
+      }
     }
+    for (; i < nv; i += stride) {
+      float4 v = v4[i];
+      a4[0] += fabs((double)v.x);
+      a4[0] += fabs((double)v.y);
+      a4[0] += fabs((double)v.z);
+      a4[0] += fabs((double)v.w);
+    }
+    acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
     const float* s = reinterpret_cast<const float*>(W);
     for (long long i = nv * 4 + t0; i < count; i += stride) acc += fabs((double)s[i]);
   }
@@ -69,18 +106,26 @@ __global__ void __launch_bounds__(kPackThreads) absmean_final_kernel(const doubl
                                                                      float* gamma) {
   __shared__ double red[33];
   double acc = 0.0;
+  grid_launch_dependents();
+  grid_dependency_wait();
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) acc += partials[i];
   acc = block_sum_f64(acc, red);
   if (threadIdx.x == 0) *gamma = count > 0 ? (float)(acc / (double)count) : 0.0f;
 }
 
-__device__ __forceinline__ uint32_t ternary_code(float w, float g) {
-  if (g == 0.0f) return 1u;                         // t = 0
-  float r = __fdiv_rn(w, g);                        // IEEE fp32 division
-  r = fminf(fmaxf(r, -2.0f), 2.0f);                 // keep rint in range
-  float t = rintf(r);                               // half to even
-  t = fminf(fmaxf(t, -1.0f), 1.0f);
-  return (uint32_t)((int)t + 1);                    // stored code c = t + 1
+// t = clamp(rint(fl(w / g)), -1, 1) without the division.  t != 0 exactly
+// when |fl(w / g)| > 1/2; rounding is monotone and the tie 1/2 + 2^-25 rounds
+// to the even 1/2, so that holds exactly when |w| > g (1/2 + 2^-25) = T.  T
+// is exact in fp64 (a 24-bit significand times a 26-bit one), and for an
+// fp32 |w|, |w| > T exactly when |w| > T rounded down to fp32 (thr).  g = 0
+// gives t = 0 for every weight.
+__device__ __forceinline__ float ternary_threshold(float g) {
+  return __double2float_rd((double)g * (0.5 + 0x1p-25));
+}
+
+__device__ __forceinline__ uint32_t ternary_code(float w, float g, float thr) {
+  if (g == 0.0f || !(fabsf(w) > thr)) return 1u;   // t = 0
+  return w > 0.0f ? 2u : 0u;                        // stored code c = t + 1
 }
 
 // One thread per 32-bit word of the packed layout: word w of row n holds
@@ -91,7 +136,10 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
                                                             uint8_t* packed) {
   const int words_per_row = ldw / 4;
   const long long total = (long long)N * words_per_row;
+  grid_launch_dependents();
+  grid_dependency_wait();
   const float g = *gamma;
+  const float thr = ternary_threshold(g);
   for (long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
        idx += (long long)gridDim.x * blockDim.x) {
     const int n = (int)(idx / words_per_row);
@@ -103,7 +151,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
       if (BF16) {
         const uint4* src = reinterpret_cast<const uint4*>(
             reinterpret_cast<const uint16_t*>(W) + (size_t)n * K + k0);
-        uint4 a = src[0], b = src[1];
+        uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 1);
         const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -113,10 +161,13 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
       } else {
         const float4* src = reinterpret_cast<const float4*>(
             reinterpret_cast<const float*>(W) + (size_t)n * K + k0);
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(src + j);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float4 v = src[j];
-          w[4 * j] = v.x; w[4 * j + 1] = v.y; w[4 * j + 2] = v.z; w[4 * j + 3] = v.w;
+          w[4 * j] = __uint_as_float(v[j].x); w[4 * j + 1] = __uint_as_float(v[j].y);
+          w[4 * j + 2] = __uint_as_float(v[j].z); w[4 * j + 3] = __uint_as_float(v[j].w);
         }
       }
       word = 0;
@@ -124,7 +175,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          word |= ternary_code(w[4 * i + j], g) << (8 * j + 2 * i);
+          word |= ternary_code(w[4 * i + j], g, thr) << (8 * j + 2 * i);
     }
     reinterpret_cast<uint32_t*>(packed + (size_t)n * ldw)[wi] = word;
   }

@@ -158,6 +158,30 @@ def test_tw2_export_and_import(N, K):
     np.testing.assert_array_equal(back.cpu().numpy(), oracle.pack(t))
 
 
+def test_pack_threshold_boundary():
+    """Codes of weights within a few hundred fp32 ulps of 0.5 * gamma, on both
+    sides of the rounding boundary of fl(w / gamma): a ballast of +-1 entries
+    fixes gamma, 512 consecutive fp32 values around the expected 0.5 * gamma
+    straddle it.  Bit-exact against the oracle's IEEE division and rint."""
+    n_ball, n_cand = 65536, 512
+    c = 0.5 * n_ball / (n_ball + n_cand - n_cand / 2)      # gamma / 2 with the candidates in
+    cand = [np.float32(c)]
+    for _ in range(n_cand // 2):
+        cand.append(np.nextafter(cand[-1], np.float32(1), dtype=np.float32))
+        cand.insert(0, np.nextafter(cand[0], np.float32(0), dtype=np.float32))
+    cand = np.array(cand[:n_cand], dtype=np.float32)
+    sign = np.where(np.arange(n_cand) % 2 == 0, 1, -1).astype(np.float32)
+    ball = np.where(np.arange(n_ball) % 2 == 0, 1, -1).astype(np.float32)
+    W = np.concatenate([ball, cand * sign]).reshape(-1, 256)
+    g = oracle.absmean(W)
+    t = oracle.ternarize(W, g)
+    tc = t.ravel()[n_ball:]
+    assert (tc == 0).any() and (tc != 0).any()            # the boundary lies inside the run
+    packed, gamma = gpu_pack(W)
+    assert gamma == g
+    np.testing.assert_array_equal(packed, oracle.pack(t))
+
+
 def test_pack_is_deterministic():
     W = synthetic.weight(np.random.default_rng(12), 2560, 2560)
     a = gpu_pack(W)
