@@ -373,8 +373,17 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   }
   for (int i = lp.nseg; i <= kMaxSegments; ++i) p.seg_tile0[i] = tiles;
   for (int i = lp.nseg; i < kMaxSegments; ++i) maps.w[i] = maps.w[0];
+  // The cluster size S: at least one CTA per SM.  When the activation codes
+  // come from the preceding kernel (a programmatic dependent launch without
+  // LAUNCH_PDL_INPUTS), a CTA converts at most three weight chunks (its
+  // ring of TMEM slots) before they arrive, and every further chunk costs a
+  // round trip between the MMA and the converter warps after that.  For a
+  // few tokens, where the cross-CTA reduction is cheap, S then grows until a
+  // CTA's slice fits the ring (three chunks, six 64-input units).
+  const bool dependent = (lp.flags & LAUNCH_PDL) && !(lp.flags & LAUNCH_PDL_INPUTS);
+  const int units_fit = dependent && lp.M <= 8 ? 6 : 1 << 30;
   int S = s_min;
-  while (S < s_max && tiles * S < di.sms) ++S;
+  while (S < s_max && (tiles * S < di.sms || (units + S - 1) / S > units_fit)) ++S;
   CUtensorMap mx;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 kDecTokens, CU_TENSOR_MAP_SWIZZLE_128B))

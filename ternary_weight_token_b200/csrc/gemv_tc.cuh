@@ -41,11 +41,14 @@ constexpr int kDecTokens = 16;                  // MMA N (tokens, zero-padded)
 constexpr int kDecMaxChunks = 7;                // slice <= 896 inputs
 constexpr int kDecMaxCluster = 8;
 constexpr int kDecThreads = 192;                // warp 0 TMA+MMA, warp 1 alloc, warps 2-5 work
-// D in columns [0, 16), A chunks from column 32: 32 + 7 * 32 = 256.  Two
-// co-resident CTAs (this launch and the next one under programmatic
-// dependent launch) always fit in the 512 columns of an SM.
-constexpr int kDecTmemCols = 256;
-constexpr int kDecMinSmem = 80 * 1024;          // at most two CTAs per SM
+// D in columns [0, 16); converted weight chunks in a ring of three 32-column
+// slots at columns 32, 64, 96 (a slot is refilled once the MMAs that read it
+// have completed).  At most four CTAs share an SM (the shared-memory floor
+// below), and 4 x 128 columns fit the 512 of an SM, so a CTA of a dependent
+// launch can never hold the tensor memory its predecessor still needs.
+constexpr int kDecTmemCols = 128;
+constexpr int kDecASlots = 3;
+constexpr int kDecMinSmem = 46 * 1024;          // at most four CTAs per SM
 
 struct DecParams {
   int M, K;
@@ -74,14 +77,16 @@ struct DecSmem {
   static constexpr int X_CHUNK = kDecTokens * kDecChunkK;         // 2 KB
   static constexpr int OFF_X = 0;                                  // 1024-aligned chunks
   static constexpr int OFF_W = OFF_X + kDecMaxChunks * X_CHUNK;
-  static constexpr int OFF_PART = OFF_W + kDecMaxChunks * W_CHUNK; // [S][16][128] int32
-  static constexpr int PART_BYTES = kDecTokens * 128 * 4;          // 8 KB per CTA
-  static constexpr int OFF_BAR = OFF_PART + kDecMaxCluster * PART_BYTES;
-  // bars: wfull[chunks], xfull[chunks], aready, mma_done, reduce
-  static constexpr int NUM_BARS = 2 * kDecMaxChunks + 3;
+  // leader: the cluster's partial sums, [16 tokens][128 rows] int32, which
+  // every CTA of the cluster adds its own into (distributed shared memory)
+  static constexpr int OFF_PART = OFF_W + kDecMaxChunks * W_CHUNK;
+  static constexpr int PART_BYTES = kDecTokens * 128 * 4;          // 8 KB
+  static constexpr int OFF_BAR = OFF_PART + PART_BYTES;
+  // bars: wfull[chunks], xfull[chunks], afull[slots], aempty[slots], mma_done, reduce
+  static constexpr int NUM_BARS = 2 * kDecMaxChunks + 2 * kDecASlots + 2;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int BYTES = OFF_MISC + 16;
-  static constexpr int ALLOC = BYTES + 1024;
+  static constexpr int ALLOC = BYTES + 1024 > kDecMinSmem ? BYTES + 1024 : kDecMinSmem;
   static_assert(ALLOC <= 227 * 1024, "decode shared memory");
 };
 
@@ -120,8 +125,10 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_addr, uint32_t ran
   return r;
 }
 
-__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+// Atomic add into a (possibly peer CTA's) shared-memory word of the cluster.
+__device__ __forceinline__ void red_add_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("red.relaxed.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(addr), "r"(v)
+               : "memory");
 }
 
 __device__ __forceinline__ void mbar_arrive_remote_release(uint32_t remote_bar) {
@@ -170,7 +177,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)
       : "r"(taddr));
 }
 
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, 4)
     gemv_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
                    const __grid_constant__ DecMaps maps, DecParams p) {
   extern __shared__ uint8_t dec_smem_raw[];
@@ -181,8 +188,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + DecSmem::OFF_BAR);
   uint64_t* wfull = bars;                                 // [chunks] weight bytes landed
   uint64_t* xfull = bars + kDecMaxChunks;                 // [chunks] activation bytes landed
-  uint64_t* aready = bars + 2 * kDecMaxChunks;            // every chunk's codes in TMEM
-  uint64_t* mma_done = aready + 1;                        // accumulator complete
+  uint64_t* afull = bars + 2 * kDecMaxChunks;             // [slots] a chunk's codes in TMEM
+  uint64_t* aempty = afull + kDecASlots;                  // [slots] its MMAs completed
+  uint64_t* mma_done = aempty + kDecASlots;               // accumulator complete
   uint64_t* reduce_bar = mma_done + 1;                    // leader: all partials in
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + DecSmem::OFF_MISC);
 
@@ -209,7 +217,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mbar_init(&wfull[c], 1);
       mbar_init(&xfull[c], 1);
     }
-    mbar_init(aready, 4);
+    for (int a = 0; a < kDecASlots; ++a) {
+      mbar_init(&afull[a], 4);                // four converter warps
+      mbar_init(&aempty[a], 1);               // tcgen05.commit
+    }
     mbar_init(mma_done, 1);
     mbar_init(reduce_bar, csize * 4);        // 4 storing warps per CTA
     fence_barrier_init();
@@ -217,6 +228,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, kDecTmemCols);
     tmem_relinquish();
+  }
+  if (rank == 0) {                           // the partial sums start at zero
+    uint32_t* part = reinterpret_cast<uint32_t*>(smem + DecSmem::OFF_PART);
+    for (int i = threadIdx.x; i < kDecTokens * 128; i += kDecThreads) part[i] = 0u;
   }
   tc_fence_before();
   __syncthreads();
@@ -246,16 +261,16 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       const uint32_t idesc = make_idesc_i8(128, kDecTokens);
       const int steps = ks / 32;
       int s = 0;
-      bool ok = true;
-      ok = mbar_wait(aready, 0, nullptr);
-      for (int c = 0; c < chunks && ok; ++c) {
-        ok = mbar_wait(&xfull[c], 0, nullptr);
-        if (!ok) break;
+      for (int c = 0; c < chunks; ++c) {
+        const int slot = c % kDecASlots;
+        if (!mbar_wait(&afull[slot], (uint32_t)(c / kDecASlots) & 1u, nullptr)) break;
+        if (!mbar_wait(&xfull[c], 0, nullptr)) break;
         tc_fence_after();
         const uint32_t xaddr = smem_u32(sx + c * DecSmem::X_CHUNK);
         for (int j = 0; j < 4 && s < steps; ++j, ++s)
-          mma_i8_ts(tbase, tbase + a_col0 + 32u * c + 8u * j,
+          mma_i8_ts(tbase, tbase + a_col0 + 32u * slot + 8u * j,
                     make_sdesc_sw128(xaddr + 32u * j), idesc, s > 0 ? 1u : 0u);
+        tc_commit(&aempty[slot]);             // the slot is free once these complete
       }
       tc_commit(mma_done);
       // never leave bulk copies in flight
@@ -272,7 +287,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16);
     bool ok = true;
     for (int c = 0; c < chunks; ++c) {
+      const int slot = c % kDecASlots;
       if (!mbar_wait(&wfull[c], 0, nullptr)) { ok = false; break; }
+      if (c >= kDecASlots &&                  // the slot's previous chunk has been multiplied
+          !mbar_wait(&aempty[slot], (uint32_t)(c / kDecASlots - 1) & 1u, nullptr)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const uint4* src = reinterpret_cast<const uint4*>(sw + c * DecSmem::W_CHUNK + row * 32);
       const uint4 a = src[0], b = src[1];
@@ -285,14 +306,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       expand_codes(b.y, e[20], e[21], e[22], e[23]);
       expand_codes(b.z, e[24], e[25], e[26], e[27]);
       expand_codes(b.w, e[28], e[29], e[30], e[31]);
-      tmem_st_32x32b_x32(lane_base + a_col0 + 32u * c, e);
+      tmem_st_32x32b_x32(lane_base + a_col0 + 32u * slot, e);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&afull[slot]);
     }
-    // one wait for every chunk's stores, then one signal to the MMA thread
-    tmem_st_wait();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(aready);
-    // partial sums -> the leader's slot for this rank, as [token][row]
+    // partial sums -> the leader's [token][row] sums (valid tokens only)
     uint32_t d[16];
     if (ok && mbar_wait(mma_done, 0, nullptr)) {
       tc_fence_after();
@@ -302,12 +322,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int t = 0; t < 16; ++t) d[t] = 0u;
     }
-    cluster_wait();                          // the leader's barriers are initialised
-    const uint32_t part_local =
-        smem_u32(smem + DecSmem::OFF_PART + rank * DecSmem::PART_BYTES) + 4u * row;
-    const uint32_t part_remote = map_to_rank(part_local, 0);
+    cluster_wait();                          // the leader's barriers and zeroed sums exist
+    const uint32_t part_remote =
+        map_to_rank(smem_u32(smem + DecSmem::OFF_PART) + 4u * row, 0);
 #pragma unroll
-    for (int t = 0; t < 16; ++t) st_cluster_u32(part_remote + 4u * 128u * t, d[t]);
+    for (int t = 0; t < 16; ++t)
+      if (t < p.M) red_add_cluster_u32(part_remote + 4u * 128u * t, d[t]);
     __syncwarp();
     if (lane == 0) mbar_arrive_remote_release(map_to_rank(smem_u32(reduce_bar), 0));
 
@@ -333,11 +353,9 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
       for (int m = 0; m < kDecTokens; ++m) acc[m] = -__shfl_sync(0xffffffffu, rs_m, m);
       if (all_in) {
-        for (int r = 0; r < (int)csize; ++r) {
 #pragma unroll
-          for (int m = 0; m < kDecTokens; ++m)
-            if (m < p.M) acc[m] += part[(r * 16 + m) * 128 + row];
-        }
+        for (int m = 0; m < kDecTokens; ++m)
+          if (m < p.M) acc[m] += part[m * 128 + row];
       }
       float y[kDecTokens];
 #pragma unroll
