@@ -477,6 +477,57 @@ def bench_ffn(torch, bn, device, iters=20):
     return {"M": M, "H": H, "I": I, "us": dt * 1e6, "TOPS": ops / dt / 1e12}
 
 
+def bench_decode_ffn(torch, bn, device, reps=3):
+    """The W1.58A8 block FFN at decode sizes (M = 1, 4, 16 tokens of the
+    2560 -> 6912 -> 2560 FFN): back-to-back bitnet_ffn calls in a CUDA graph
+    over a pool of weight sets larger than twice the L2.  Four launches per
+    call (quant, gate + up, relu^2 * up with the sub-norm quant, down); GB/s
+    counts the three packed weight matrices, x (read twice) and y."""
+    cfg = synthetic.WORKLOADS["ffn"].dims
+    H, I = cfg["H"], cfg["I"]
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    inp = synthetic.ffn_inputs(max(DECODE_M), H, I, seed=5)
+    base = []
+    for k in ("Wg", "Wu", "Wd"):
+        W = torch.from_numpy(inp[k]).to(device)
+        P, g, ws = bn.alloc_packed(*W.shape, device)
+        bn.bitnet_pack_weights(W, P, g, ws)
+        base.append((P, g))
+    set_bytes = sum(P.numel() for P, _ in base)
+    pool = max(8, int(2 * l2 // set_bytes) + 2)
+    sets = [[(P.clone(), g) for P, g in base] for _ in range(pool)]
+    X_all = torch.from_numpy(inp["x_bf16"].view(np.int16)).to(device).view(torch.bfloat16)
+    out = []
+    for M in DECODE_M:
+        X = X_all[:M].contiguous()
+        Y = torch.empty((M, H), dtype=torch.bfloat16, device=device)
+        ws = bn.alloc_ffn_workspace(M, H, I, device=device)
+        step_bytes = set_bytes + 3 * 2 * M * H      # + x (twice: norm, residual) and y, bf16
+
+        def run(st, w):
+            bn.bitnet_ffn(X, w[0][0], w[0][1], w[1][0], w[1][1], w[2][0], w[2][1], Y, ws,
+                          variant=bn.BITNET_FFN_RELU2_GLU, eps=1e-5, stream=st)
+        run(None, sets[0])
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        stream = torch.cuda.Stream(device)
+        with torch.cuda.stream(stream):
+            graph.capture_begin(capture_error_mode="thread_local")
+            for w in sets:
+                run(stream, w)
+            graph.capture_end()
+        torch.cuda.synchronize()
+        graph.replay()
+        torch.cuda.synchronize()
+        best = min(time_loop(torch, graph.replay, 4) for _ in range(reps))
+        out.append({"M": M, "H": H, "I": I, "weight_sets_in_pool": pool,
+                    "us_per_ffn": best / (4 * pool) * 1e6,
+                    "GB_s": step_bytes * 4 * pool / best / 1e9})
+        del graph
+    del sets
+    return out
+
+
 def bench_hffn(torch, bn, device, iters=50):
     cfg = synthetic.WORKLOADS["hffn"].dims
     M, D, F = cfg["M"], cfg["D"], cfg["F"]
@@ -654,6 +705,7 @@ def run_b200(args, world, rank, local):
         line["workloads"] = {
             "decode": dec,
             "decode_qkv": bench_decode_qkv(torch, bn, device),
+            "decode_ffn": bench_decode_ffn(torch, bn, device),
             "decode_peak_source": f"{peaks['source']} HBM copy {peaks['hbm_gbs']} GB/s",
             "ffn": bench_ffn(torch, bn, device),
             "hffn": bench_hffn(torch, bn, device),
@@ -699,7 +751,8 @@ def run_only(args, local):
         out = decode_single(torch, bn, device, M, K, N, max(1, args.steps))
     else:
         fn = {"decode": bench_decode, "ffn": bench_ffn, "hffn": bench_hffn,
-              "tiny": bench_tiny, "qkv": bench_decode_qkv, "online": bench_online}[args.only]
+              "tiny": bench_tiny, "qkv": bench_decode_qkv, "online": bench_online,
+              "dffn": bench_decode_ffn}[args.only]
         out = fn(torch, bn, device)
     print(json.dumps({"only": args.only, "result": out}), flush=True)
     return 0
@@ -716,7 +769,7 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-step-seconds", type=float, default=None,
                     help="with --impl reference: target seconds of oracle work per step")
-    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny", "qkv", "online"),
+    ap.add_argument("--only", choices=("decode", "ffn", "hffn", "tiny", "qkv", "online", "dffn"),
                     default=None,
                     help="time one secondary workload and print its JSON (profiling aid)")
     ap.add_argument("--decode-shape", default=None,

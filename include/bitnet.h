@@ -225,6 +225,10 @@ BITNET_API size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant);
  *   Y = x + down_proj(RMSNorm(m; sub_norm_gain, eps))   (ffn_sub_norm)
  *   X, Y [M][H] of x_dtype / y_dtype (F32 or BF16); W_gate, W_up [I][H] and
  *   W_down [H][I] packed; gains may be NULL (all ones).
+ *   Decode (M <= 16): gate and up run as two projections of one decode
+ *   launch, and the sub-norm quantiser forms m from their fp32 outputs as it
+ *   loads them (the workspace is then larger by M * I * 4 bytes); larger M
+ *   runs the fused gate/up GEMM, whose epilogue forms m.
  * BITNET_FFN_HADAMARD_SILU ("bitnetv2-model" README, "Architecture
  * Overview"): Y = W2 . silu(W1 . x), each an H-BitLinear (FWHT prelude);
  *   W_gate = W1 [I][H], W_down = W2 [H][I], W_up / gamma_up must be NULL,

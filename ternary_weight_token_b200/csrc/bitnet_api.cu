@@ -196,7 +196,9 @@ int launch_quant_rows(const QuantParams& p, bool bf16, int prelude, cudaStream_t
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
   void (*kern)(QuantParams) = nullptr;
-  if (prelude == PRE_RMSNORM)
+  if (prelude == PRE_GLU_RMSNORM)
+    kern = quant_act_reg_kernel<NT, VPT, PRE_GLU_RMSNORM, false>;
+  else if (prelude == PRE_RMSNORM)
     kern = bf16 ? quant_act_reg_kernel<NT, VPT, PRE_RMSNORM, true>
                 : quant_act_reg_kernel<NT, VPT, PRE_RMSNORM, false>;
   else
@@ -206,12 +208,15 @@ int launch_quant_rows(const QuantParams& p, bool bf16, int prelude, cudaStream_t
   return launch_pdl(kern, dim3(grid), dim3(NT), 0, st, p);
 }
 
+// X2: the up projection when prelude is PRE_GLU_RMSNORM (X is then the gate
+// projection, both fp32), else null.
 int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const float* gain,
-                 float eps, int8_t* Xq, float* scale, int32_t* rowsum, cudaStream_t st) {
+                 float eps, int8_t* Xq, float* scale, int32_t* rowsum, cudaStream_t st,
+                 const float* X2 = nullptr) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
   QuantParams p;
-  p.X = X; p.M = M; p.K = K; p.gain = gain; p.eps = eps;
+  p.X = X; p.X2 = X2; p.M = M; p.K = K; p.gain = gain; p.eps = eps;
   p.fwht_c = (float)(1.0 / std::sqrt((double)K));
   p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
   if (prelude != PRE_FWHT) {
@@ -710,7 +715,9 @@ size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant) {
   total += align256(m * (size_t)I * 4);        // fp32 hidden activation
   total += align256(m * (size_t)I);            // codes of the hidden activation
   total += align256(m * 4) * 2;                // its scale and rowsum
-  (void)variant;
+  // decode (M <= 16) gate/up run as two projections of one launch: the up
+  // projection's fp32 output too
+  if (variant == BITNET_FFN_RELU2_GLU && M <= 16) total += align256(m * (size_t)I * 4);
   return total;
 }
 
@@ -765,7 +772,8 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   float* hid = reinterpret_cast<float*>(ws);             ws += align256(m * I * 4);
   int8_t* hq = reinterpret_cast<int8_t*>(ws);            ws += align256(m * I);
   float* hs = reinterpret_cast<float*>(ws);              ws += align256(m * 4);
-  int32_t* hrs = reinterpret_cast<int32_t*>(ws);
+  int32_t* hrs = reinterpret_cast<int32_t*>(ws);         ws += align256(m * 4);
+  float* hid_up = reinterpret_cast<float*>(ws);          // decode GLU only
   const bool xbf = x_dtype == BITNET_BF16;
 
   LinearParams p1;
@@ -779,6 +787,26 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   single_segment(p1);
   single_segment(p2);
 
+  if (variant == BITNET_FFN_RELU2_GLU && M <= 16) {
+    // Decode: gate and up as two projections of one decode launch (fp32
+    // outputs), relu(g)^2 * u formed by the sub-norm quantiser as it loads
+    // them, the down projection with the residual.  Each launch after the
+    // first streams its weights while its predecessor finishes (PDL).
+    if (int rc = launch_quant(X, xbf, M, H, PRE_RMSNORM, pre_norm_gain, eps, xq, xs, xrs, st))
+      return rc;
+    p1.N = 2 * I;                              // rows of both projections
+    p1.nseg = 2;
+    p1.seg_row0[0] = 0; p1.seg_row0[1] = I; p1.seg_row0[2] = 2 * I;
+    p1.seg_W[1] = W_up; p1.seg_gamma[1] = gamma_up; p1.seg_Y[1] = hid_up;
+    p1.flags = LAUNCH_PDL;
+    if (int rc = launch_linear(p1, st)) return rc;
+    if (int rc = launch_quant(hid, false, M, I, PRE_GLU_RMSNORM, sub_norm_gain, eps, hq, hs, hrs,
+                              st, hid_up))
+      return rc;
+    p2.flags = EPI_RESIDUAL | LAUNCH_PDL;
+    p2.resid = X;
+    return launch_linear(p2, st);
+  }
   if (variant == BITNET_FFN_RELU2_GLU) {
     if (int rc = launch_quant(X, xbf, M, H, PRE_RMSNORM, pre_norm_gain, eps, xq, xs, xrs, st))
       return rc;

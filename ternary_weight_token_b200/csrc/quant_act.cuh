@@ -24,10 +24,13 @@
 
 namespace bitnet {
 
-enum { PRE_NONE = 0, PRE_RMSNORM = 1, PRE_FWHT = 2 };
+// PRE_GLU_RMSNORM: the row is m = relu(g)^2 * u of two fp32 inputs (gate
+// X, up X2), as the fused gate/up epilogue forms it, then RMSNorm.
+enum { PRE_NONE = 0, PRE_RMSNORM = 1, PRE_FWHT = 2, PRE_GLU_RMSNORM = 3 };
 
 struct QuantParams {
   const void* X;
+  const float* X2;     // up projection for PRE_GLU_RMSNORM, else unused
   int M, K;
   const float* gain;   // [K] or null (RMSNorm only)
   float eps;           // RMSNorm epsilon
@@ -325,9 +328,10 @@ struct RowRed {
 template <int NT, int VPT, int PRE, bool BF16>
 __device__ __forceinline__ void quant_row(const QuantParams& p, int m, float4 (&v)[VPT],
                                           RowRed& red, int par) {
+  constexpr bool RMS = PRE == PRE_RMSNORM || PRE == PRE_GLU_RMSNORM;
   const int K = p.K;
   float r = 1.0f, amax = 0.0f;
-  if (PRE == PRE_RMSNORM) {
+  if (RMS) {
     double s0 = 0.0, s1 = 0.0;
     float xmax = 0.0f;
 #pragma unroll
@@ -374,7 +378,7 @@ __device__ __forceinline__ void quant_row(const QuantParams& p, int m, float4 (&
   if (zero_row) s = 1.0f;
   if (threadIdx.x == 0) p.scale[m] = s;
   // the RMS factor is applied here when no gain was (same two roundings)
-  const bool fold_r = PRE == PRE_RMSNORM && p.gain == nullptr;
+  const bool fold_r = RMS && p.gain == nullptr;
   int rsum = 0;
   uint8_t* dst = reinterpret_cast<uint8_t*>(p.Xq) + (size_t)m * K;
   auto codes = [&](const float4& x) -> uint32_t {
@@ -448,7 +452,9 @@ __device__ __forceinline__ void unpack_row(const uint4 (&u)[BF16 ? VPT / 2 : VPT
 // before the first reduction.
 template <int NT, int VPT, int PRE, bool BF16>
 __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
-  static_assert(PRE == PRE_NONE || PRE == PRE_RMSNORM, "FWHT uses the shared-memory kernel");
+  static_assert(PRE == PRE_NONE || PRE == PRE_RMSNORM || PRE == PRE_GLU_RMSNORM,
+                "FWHT uses the shared-memory kernel");
+  static_assert(PRE != PRE_GLU_RMSNORM || !BF16, "gate/up rows are fp32");
   static_assert(!BF16 || VPT % 2 == 0, "bf16 rows load 8 values per 16 bytes");
   constexpr int NU = BF16 ? VPT / 2 : VPT;
   __shared__ RowRed red;
@@ -469,6 +475,21 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
     }
     float4 v[VPT];
     unpack_row<NT, VPT, BF16>(u, v);
+    if (PRE == PRE_GLU_RMSNORM) {
+      // m = relu(g)^2 * u, fp32 products in the epilogue's order
+      const float4* up = reinterpret_cast<const float4*>(p.X2 + (size_t)m * K);
+      auto glu = [](float g, float x) { return __fmul_rn(g > 0.0f ? __fmul_rn(g, g) : 0.0f, x); };
+      uint4 w[VPT];
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int idx = (int)threadIdx.x + i * NT;
+        w[i] = idx < units ? ld_stream_v4(up + idx) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < VPT; ++i)
+        v[i] = make_float4(glu(v[i].x, __uint_as_float(w[i].x)), glu(v[i].y, __uint_as_float(w[i].y)),
+                           glu(v[i].z, __uint_as_float(w[i].z)), glu(v[i].w, __uint_as_float(w[i].w)));
+    }
     quant_row<NT, VPT, PRE, BF16>(p, m, v, red, par);
     __syncthreads();
     finish_rowsum(p, m, red);

@@ -64,7 +64,9 @@ def run_ffn_relu2(inp, rows=None, gains=False):
                   sub_norm_gain=None if sub is None else dev(sub), eps=1e-5)
     torch.cuda.synchronize()
     got = Y.float().cpu().numpy()
-    # the workspace holds the fp32 hidden activation m and its codes
+    # the workspace holds the fp32 hidden activation m and its codes; at
+    # decode sizes (M <= 16) the gate output g in m's place and the up output
+    # u after the codes' scale and sum, m = relu(g)^2 * u formed on loading
     ws_np = ws.cpu().numpy()
     off = 0
 
@@ -76,6 +78,10 @@ def run_ffn_relu2(inp, rows=None, gains=False):
     take(M * H), take(M * 4), take(M * 4)
     m_dev = take(M * I * 4).view(np.float32).reshape(M, I)
     qm_dev = take(M * I).view(np.int8).reshape(M, I)
+    if M <= 16:
+        take(M * 4), take(M * 4)
+        u_dev = take(M * I * 4).view(np.float32).reshape(M, I)
+        m_dev = oracle.relu2_glu(m_dev, u_dev)
     sel = np.arange(M) if rows is None else np.asarray(rows)
     go, To = {}, {}
     for k in ("Wg", "Wu", "Wd"):
@@ -87,8 +93,13 @@ def run_ffn_relu2(inp, rows=None, gains=False):
 
 
 @pytest.mark.parametrize("M,H,I,gains", [(64, 256, 512, False), (300, 512, 1024, True),
-                                         (9, 256, 512, False)])
+                                         (9, 256, 512, False), (1, 2560, 6912, True),
+                                         (2, 256, 512, True), (4, 2560, 6912, False),
+                                         (16, 512, 1024, True), (17, 256, 512, False)])
 def test_ffn_relu2_small(M, H, I, gains):
+    """M <= 16 runs gate and up as one decode launch (streaming kernel for
+    1-2 tokens, cluster tensor-core kernel for 3-16) and forms m in the
+    sub-norm quantiser; M = 17 on is the fused gate/up GEMM."""
     inp = synthetic.ffn_inputs(M, H, I, seed=M)
     got, want, m_dev, m, qm_dev, qm = run_ffn_relu2(inp, gains=gains)
     # gate/up epilogue: m = relu(g)^2 * u
