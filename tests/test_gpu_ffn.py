@@ -94,8 +94,10 @@ def run_ffn_relu2(inp, rows=None, gains=False):
 
 @pytest.mark.parametrize("M,H,I,gains", [(64, 256, 512, False), (300, 512, 1024, True),
                                          (9, 256, 512, False), (1, 2560, 6912, True),
-                                         (2, 256, 512, True), (4, 2560, 6912, False),
-                                         (16, 512, 1024, True), (17, 256, 512, False)])
+                                         (1, 2560, 6912, False), (2, 256, 512, True),
+                                         (2, 320, 448, False), (1, 208, 272, True),
+                                         (4, 2560, 6912, False), (16, 512, 1024, True),
+                                         (17, 256, 512, False)])
 def test_ffn_relu2_small(M, H, I, gains):
     """M <= 16 runs gate and up as one decode launch (streaming kernel for
     1-2 tokens, cluster tensor-core kernel for 3-16) and forms m in the
@@ -166,3 +168,40 @@ def test_hffn_decode_path():
     go2, T2, _ = oracle.quantize_weights(inp["W2"])
     want = oracle.hffn(inp["X"], T1, go1, T2, go2)
     assert _rel_l2(Y.cpu().numpy(), want) <= 1e-3
+
+
+@pytest.mark.parametrize("M", [1, 2, 5])
+def test_ffn_relu2_decode_fp32_io(M):
+    """The decode route with fp32 input and output (the residual then adds in
+    fp32) and a sub-norm gain, against the oracle block."""
+    H, I = 512, 1536
+    inp = synthetic.ffn_inputs(M, H, I, seed=40 + M)
+    Pg, gg = _pack_dev(inp["Wg"])
+    Pu, gu = _pack_dev(inp["Wu"])
+    Pd, gd = _pack_dev(inp["Wd"])
+    sub = np.random.default_rng(3).uniform(0.5, 1.5, I).astype(np.float32)
+    Y = torch.empty((M, H), device="cuda")
+    ws = bn.alloc_ffn_workspace(M, H, I)
+    bn.bitnet_ffn(dev(inp["x"]), Pg, gg, Pu, gu, Pd, gd, Y, ws, variant=bn.BITNET_FFN_RELU2_GLU,
+                  sub_norm_gain=dev(sub), eps=1e-5)
+    torch.cuda.synchronize()
+    assert bn.bitnet_check_device_error() == bn.BITNET_OK
+    go, To = {}, {}
+    for k in ("Wg", "Wu", "Wd"):
+        go[k], To[k], _ = oracle.quantize_weights(inp[k])
+    want, m, qm, sm = oracle.ffn_relu2(inp["x"], To["Wg"], go["Wg"], To["Wu"], go["Wu"], To["Wd"],
+                                       go["Wd"], sub_gain=sub, eps=1e-5, residual=True, keep=True)
+    ws_np = ws.cpu().numpy()
+    off = lambda n: (n + 255) // 256 * 256
+    base = off(M * H) + 2 * off(M * 4)
+    g_dev = ws_np[base:base + M * I * 4].view(np.float32).reshape(M, I)
+    qbase = base + off(M * I * 4)
+    qm_dev = ws_np[qbase:qbase + M * I].view(np.int8).reshape(M, I)
+    ubase = qbase + off(M * I) + 2 * off(M * 4)
+    u_dev = ws_np[ubase:ubase + M * I * 4].view(np.float32).reshape(M, I)
+    np.testing.assert_allclose(oracle.relu2_glu(g_dev, u_dev), m, rtol=1e-5, atol=0)
+    assert_codes_chain(qm_dev, qm, "decode codes")
+    got = Y.cpu().numpy()
+    if code_mismatch_stats(qm_dev, qm)[0] == 0:
+        np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-6 * np.abs(want).max())
+    assert _rel_l2(got, want) <= 1e-3
