@@ -81,6 +81,34 @@ def test_quant_rmsnorm(M, K, with_gain):
         np.testing.assert_allclose(s, so, rtol=1e-6)
 
 
+@pytest.mark.parametrize("M,K,bf16,prelude", [(2001, 2560, False, 0), (2001, 2560, True, 1),
+                                               (701, 6912, False, 1), (1500, 512, False, 0),
+                                               (3000, 16384, True, 0)])
+def test_quant_many_rows(M, K, bf16, prelude):
+    """Prefill-sized row counts on every row-kernel width (64 x 10, 128 x 14 and
+    256 x 16 threads x chunks), zero and one-hot rows among them."""
+    X = _acts(M, K, seed=M + K)
+    X[M // 2] = 0.0
+    X[M - 1] = 0.0
+    X[M - 1, K // 5] = 3.25
+    if bf16:
+        bits = synthetic.to_bf16_bits(X)
+        X = oracle.bf16_bits_to_f32(bits)
+    pre = (bn.BITNET_PRELUDE_RMSNORM, oracle.PRELUDE_RMSNORM) if prelude else (
+        bn.BITNET_PRELUDE_NONE, oracle.PRELUDE_NONE)
+    q, s, rs = gpu_quant(X, pre[0], eps=1e-5, x_dev=bf16_dev(bits) if bf16 else None)
+    qo, so, rso = oracle.quant_act(X, pre[1], eps=1e-5)
+    if prelude:
+        assert_codes_chain(q, qo, "rmsnorm codes")
+        if code_mismatch_stats(q, qo)[0] == 0:
+            np.testing.assert_array_equal(s, so)
+            np.testing.assert_array_equal(rs, rso)
+    else:
+        np.testing.assert_array_equal(q, qo)
+        np.testing.assert_array_equal(s, so)
+        np.testing.assert_array_equal(rs, rso)
+
+
 def test_quant_bf16_input():
     X = _acts(40, 2560, seed=5)
     bits = synthetic.to_bf16_bits(X)
