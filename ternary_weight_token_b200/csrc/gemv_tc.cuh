@@ -15,14 +15,19 @@
 //     128 bytes per chunk in the 128-byte swizzled layout), so the whole
 //     slice is in flight;
 //   - four converter warps expand each chunk's 2-bit codes to byte codes in
-//     tensor memory (one TMEM lane per weight row) as soon as it lands;
+//     tensor memory (one TMEM lane per weight row) as soon as it lands, into
+//     a ring of three 32-column slots; a slot is refilled once the
+//     tcgen05.commit of the MMAs that read it has arrived;
 //   - one thread issues tcgen05.mma kind::i8 (M = 128 weight rows, N = 16
 //     tokens, K = 32) per 32-k step into a 16-column int32 accumulator;
-//   - the four warps read the partial sums back (tcgen05.ld) and store them
-//     into the leader CTA's shared memory (distributed shared memory), then
-//     arrive on the leader's mbarrier with cluster-scope release;
-//   - the leader waits (bounded) for all S partials, adds them, subtracts the
-//     token's code sum, dequantises and writes the outputs.
+//   - the four warps read the partial sums back (tcgen05.ld) and add those of
+//     the valid tokens into one [16][128] buffer in the leader CTA's shared
+//     memory (red.add over distributed shared memory), then arrive on the
+//     leader's mbarrier with cluster-scope release;
+//   - the leader waits (bounded) for all S arrivals, subtracts the token's
+//     code sum, dequantises and writes the outputs.
+// 128 TMEM columns and about 51 KB of shared memory per CTA: four CTAs
+// (four consecutive calls) share an SM.
 // With programmatic dependent launch the weight loads and their expansion
 // start before the preceding kernel on the stream has finished; activation
 // codes, scales and outputs are touched only after griddepcontrol.wait.  When
