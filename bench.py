@@ -12,7 +12,8 @@ once (the pages' packed checkpoint stores them ternary, "offline").
 Prints ONE JSON line (rank 0).  `value` is int8 TOPS (2*M*N*K per projection,
 zero weights not skipped) over all ranks; `roofline` is the tcgen05 GEMM's
 achieved fraction of the int8 tensor peak; `e2e` is the same step through the
-C ABI with host buffers (pinned H2D of the activations, D2H of the outputs);
+C ABI with host buffers (pinned H2D of the activations, D2H of the outputs,
+pipelined over token chunks on two copy streams);
 `cpu_baseline` is the CPU oracle on a bounded sample of the same step;
 `workloads` adds the decode GEMV streaming bandwidth and the FFN / H-FFN /
 tiny configurations.
@@ -51,6 +52,10 @@ GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_tc_prefill_4096x2560x6912.md
 
 def prefill_ops():
     return sum(2 * PREFILL_M * N * K for K, N in PREFILL_KN)
+
+
+# token chunks of the end-to-end step's copy / compute / copy pipeline
+E2E_CHUNKS = 8
 
 
 def decode_bytes(M, K, N):
@@ -289,6 +294,7 @@ class Prefill:
                                 "rs": rs, "Y": Y, "X_host": None, "Y_host": None})
         torch.cuda.synchronize()
         self.launches_per_step = 2 * len(self.shapes)
+        self.copy_in = self.copy_out = None
 
     def step(self, gemm_events=None):
         bn = self.bn
@@ -307,15 +313,40 @@ class Prefill:
             if sh["X_host"] is None:
                 sh["X_host"] = sh["X"].cpu().pin_memory()
                 sh["Y_host"] = torch.empty(sh["Y"].shape, dtype=sh["Y"].dtype).pin_memory()
+        if self.copy_in is None:
+            self.copy_in, self.copy_out = torch.cuda.Stream(), torch.cuda.Stream()
 
     def e2e_step(self):
-        bn = self.bn
+        """One step through the public API from and to pinned host buffers,
+        pipelined over token chunks: the host-to-device copy of a chunk (copy-in
+        stream), its quantiser and projection (the current stream) and the
+        device-to-host copy of its outputs (copy-out stream) overlap those of
+        the neighbouring chunks, and PCIe carries both directions at once.  The
+        step starts after all earlier work on the current stream and ends, on
+        that stream, when the last outputs are on the host."""
+        torch, bn = self.torch, self.bn
+        main = torch.cuda.current_stream()
+        self.copy_in.wait_stream(main)
+        self.copy_out.wait_stream(main)
+        rows = PREFILL_M // E2E_CHUNKS
         for sh in self.shapes:
-            sh["X"].copy_(sh["X_host"], non_blocking=True)
-            bn.bitnet_quant_act(sh["X"], sh["q"], sh["s"], sh["rs"],
-                                prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
-            bn.bitnet_linear(sh["q"], sh["s"], sh["rs"], sh["P"], sh["g"], sh["K"], sh["Y"])
-            sh["Y_host"].copy_(sh["Y"], non_blocking=True)
+            for c in range(E2E_CHUNKS):
+                sl = slice(c * rows, (c + 1) * rows)
+                with torch.cuda.stream(self.copy_in):
+                    sh["X"][sl].copy_(sh["X_host"][sl], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(self.copy_in)
+                main.wait_event(landed)
+                bn.bitnet_quant_act(sh["X"][sl], sh["q"][sl], sh["s"][sl], sh["rs"][sl],
+                                    prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
+                bn.bitnet_linear(sh["q"][sl], sh["s"][sl], sh["rs"][sl], sh["P"], sh["g"],
+                                 sh["K"], sh["Y"][sl])
+                done = torch.cuda.Event()
+                done.record(main)
+                self.copy_out.wait_event(done)
+                with torch.cuda.stream(self.copy_out):
+                    sh["Y_host"][sl].copy_(sh["Y"][sl], non_blocking=True)
+        main.wait_stream(self.copy_out)
 
     def h2d_bytes(self):
         return sum(sh["X"].numel() * sh["X"].element_size() for sh in self.shapes)
