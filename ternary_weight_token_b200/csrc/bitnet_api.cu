@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -397,11 +398,16 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   p.xs = lp.xs; p.xrs = lp.xrs;
   p.resid = lp.resid; p.out_type = lp.out_type;
   p.flags = lp.flags & ~LAUNCH_PDL;     // keeps LAUNCH_PDL_INPUTS for the kernel
-  static bool attr_set = false;
-  if (!attr_set) {
+  // The shared-memory attribute belongs to each device's context: set it once
+  // per device (a bit per device ordinal; ordinals past 63 set it every call).
+  static std::atomic<uint64_t> attr_set{0};
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
+  if (bit == 0 || (attr_set.load(std::memory_order_acquire) & bit) == 0) {
     BN_CHECK_CUDA(cudaFuncSetAttribute(gemv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        DecSmem::ALLOC));
-    attr_set = true;
+    attr_set.fetch_or(bit, std::memory_order_release);
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(tiles * S), 1, 1);
