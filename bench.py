@@ -594,14 +594,32 @@ def bench_tiny(torch, bn, device, iters=200):
     q, s, rs = bn.alloc_quant(M, K, device)
     Y = torch.empty((M, N), device=device)
 
-    def run():
-        bn.bitnet_quant_act(X, q, s, rs)
-        bn.bitnet_linear(q, s, rs, P, g, K, Y)
+    def run(stream=None):
+        bn.bitnet_quant_act(X, q, s, rs, stream=stream)
+        bn.bitnet_linear(q, s, rs, P, g, K, Y, epilogue=bn.BITNET_F32 | bn.BITNET_LAUNCH_PDL,
+                         stream=stream)
     for _ in range(5):
         run()
     dt = time_loop(torch, run, iters) / iters
-    return {"M": M, "K": K, "N": N, "us_per_call": dt * 1e6,
-            "note": "quant + linear, launch-latency bound"}
+    # the same pairs replayed from a CUDA graph: device time without the
+    # Python and launch overhead of each call
+    reps = 20
+    graph = torch.cuda.CUDAGraph()
+    stream = torch.cuda.Stream(device)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        graph.capture_begin(capture_error_mode="thread_local")
+        for _ in range(reps):
+            run(stream)
+        graph.capture_end()
+    torch.cuda.synchronize()
+    graph.replay()
+    torch.cuda.synchronize()
+    dg = min(time_loop(torch, graph.replay, 10) for _ in range(3)) / (10 * reps)
+    del graph
+    return {"M": M, "K": K, "N": N, "us_per_call": dt * 1e6, "us_per_call_graph": dg * 1e6,
+            "note": "quant + linear: eager calls are bound by host launch overhead; the graph "
+                    "replay gives the device time of a dependent pair"}
 
 
 def bench_online(torch, bn, device, iters=20):
