@@ -287,9 +287,10 @@ BITNET_API int bitnet_check_device_error(bitnet_stream_t stream);
  * context usable.  Returns BITNET_OK if the launch succeeded. */
 BITNET_API int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t stream);
 
-/* Drop the host-side cache of TMA tensor descriptors (keyed by pointer and
- * shape).  Call after freeing buffers that were passed to bitnet_linear() if
- * their addresses may be reused with different shapes. */
+/* Empty the host-side cache of TMA tensor descriptors.  The cache is keyed
+ * by device, pointer, shape, box and swizzle, so it stays correct when an
+ * address is reused; it holds at most 16384 descriptors (it starts over when
+ * full).  This call only releases its memory. */
 BITNET_API void bitnet_release_cache(void);
 
 /* Library version string. */

@@ -123,6 +123,7 @@ struct MapKeyHash {
   }
 };
 
+constexpr size_t kMapCacheMax = 16384;   // descriptors (128 B each) kept at most
 std::mutex g_map_mu;
 std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_map_cache;
 
@@ -154,6 +155,9 @@ int tensor_map_2d(CUtensorMap& out, const void* ptr, CUtensorMapDataType dtype, 
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(BITNET_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   std::lock_guard<std::mutex> lock(g_map_mu);
+  // bounded: a caller that keeps passing new buffers starts the cache over
+  // instead of growing it without limit
+  if (g_map_cache.size() >= kMapCacheMax) g_map_cache.clear();
   g_map_cache[key] = out;
   return BITNET_OK;
 }
