@@ -180,6 +180,19 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def sources_sha():
+    """One hash over the kernel sources and the C header, identifying the
+    build a line was measured with."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ternary_weight_token_b200", "csrc")
+    names = sorted(n for n in os.listdir(csrc) if n.endswith((".cu", ".cuh", ".h")))
+    for name in names + ["../../include/bitnet.h"]:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def profiled_traffic():
     """DRAM bytes per GEMM launch from the committed ncu summary, or None when
     the summary is missing or the kernel source changed since the capture."""
@@ -684,10 +697,12 @@ def run_b200(args, world, rank, local):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
+    torch.cuda.nvtx.range_push(f"prefill: {args.steps} timed steps")
     start.record()
     for s in range(args.steps):
         pre.step(evs[s])
     end.record()
+    torch.cuda.nvtx.range_pop()
     end.synchronize()
     t_wall1 = time.time()
     elapsed = start.elapsed_time(end) / 1e3
@@ -709,7 +724,9 @@ def run_b200(args, world, rank, local):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
+    torch.cuda.nvtx.range_push(f"prefill e2e: {e2e_steps} steps from host buffers")
     e2e_elapsed = time_loop(torch, pre.e2e_step, e2e_steps)
+    torch.cuda.nvtx.range_pop()
     e2e_elapsed = max_over_ranks(e2e_elapsed, dist, device)
     e2e_value = world * prefill_ops() * e2e_steps / e2e_elapsed / 1e12
 
@@ -742,7 +759,8 @@ def run_b200(args, world, rank, local):
                     "h2d_bytes_per_step": pre.h2d_bytes(),
                     "d2h_bytes_per_step": pre.d2h_bytes(), "steps": e2e_steps},
             "gpu_launches": pre.launches_per_step * args.steps,
-            "clocks": clocks}
+            "clocks": clocks,
+            "source": {"csrc_sha256_16": sources_sha()}}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_prefill_sample(target_s=args.cpu_seconds)
