@@ -180,6 +180,21 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def nvtx_push(torch, name):
+    """Named range for profilers; a no-op where NVTX is unavailable."""
+    try:
+        torch.cuda.nvtx.range_push(name)
+    except Exception:             # noqa: BLE001
+        pass
+
+
+def nvtx_pop(torch):
+    try:
+        torch.cuda.nvtx.range_pop()
+    except Exception:             # noqa: BLE001
+        pass
+
+
 def sources_sha():
     """One hash over the kernel sources and the C header, identifying the
     build a line was measured with."""
@@ -697,12 +712,12 @@ def run_b200(args, world, rank, local):
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
-    torch.cuda.nvtx.range_push(f"prefill: {args.steps} timed steps")
+    nvtx_push(torch, f"prefill: {args.steps} timed steps")
     start.record()
     for s in range(args.steps):
         pre.step(evs[s])
     end.record()
-    torch.cuda.nvtx.range_pop()
+    nvtx_pop(torch)
     end.synchronize()
     t_wall1 = time.time()
     elapsed = start.elapsed_time(end) / 1e3
@@ -724,9 +739,9 @@ def run_b200(args, world, rank, local):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    torch.cuda.nvtx.range_push(f"prefill e2e: {e2e_steps} steps from host buffers")
+    nvtx_push(torch, f"prefill e2e: {e2e_steps} steps from host buffers")
     e2e_elapsed = time_loop(torch, pre.e2e_step, e2e_steps)
-    torch.cuda.nvtx.range_pop()
+    nvtx_pop(torch)
     e2e_elapsed = max_over_ranks(e2e_elapsed, dist, device)
     e2e_value = world * prefill_ops() * e2e_steps / e2e_elapsed / 1e12
 
