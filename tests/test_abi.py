@@ -51,6 +51,13 @@ def test_workspace_sizes():
     # codes of x, fp32 hidden activation and its codes, plus per-token vectors
     assert need >= 2048 * 2560 + 2048 * 6912 * 5
     assert bn.bitnet_ffn_workspace_size(-1, 2560, 6912) == 0
+    # decode sizes (M <= 16) also hold the up projection's fp32 output
+    for M in (1, 4, 16):
+        glu = bn.bitnet_ffn_workspace_size(M, 2560, 6912, bn.BITNET_FFN_RELU2_GLU)
+        had = bn.bitnet_ffn_workspace_size(M, 2560, 6912, bn.BITNET_FFN_HADAMARD_SILU)
+        assert glu >= had + M * 6912 * 4
+    assert (bn.bitnet_ffn_workspace_size(17, 2560, 6912, bn.BITNET_FFN_RELU2_GLU)
+            == bn.bitnet_ffn_workspace_size(17, 2560, 6912, bn.BITNET_FFN_HADAMARD_SILU))
 
 
 # Raw ctypes calls with fake, aligned pointers: validation must reject them
