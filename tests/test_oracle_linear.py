@@ -133,6 +133,127 @@ def test_silu_against_fp64_closed_form():
         assert v == np.float32(d / (1.0 + math.exp(-d))) or abs(v - d / (1 + math.exp(-d))) <= abs(v) * 6e-8
 
 
+# ---- SiLU pinned by the mathematics of y * sigmoid(y), not by its formula
+
+def _f(v):
+    return Fraction(float(v))
+
+
+def test_silu_odd_part_is_the_identity():
+    """silu(y) - silu(-y) = y for every y (sigmoid(y) + sigmoid(-y) = 1), up to
+    the two fp32 roundings of the oracle's outputs; checked in exact rationals.
+    A wrong factor or an added term breaks it."""
+    ys = np.concatenate([np.linspace(-30, 30, 6001), np.geomspace(1e-6, 80, 400)]).astype(np.float32)
+    pos, neg = oracle.silu(ys), oracle.silu(-ys)
+    for y, a, b in zip(ys, pos, neg):
+        half = (_f(np.spacing(np.abs(a))) + _f(np.spacing(np.abs(b)))) / 2
+        assert abs(_f(a) - _f(b) - _f(y)) <= half, (y, a, b)
+
+
+def test_silu_even_part_is_y_tanh_half_y():
+    """silu(y) + silu(-y) = y (sigmoid(y) - sigmoid(-y)) = y tanh(y / 2).  This
+    separates y * sigmoid(y) from y * sigmoid(-y) (an exp(+y) sign slip, which
+    has the same odd part but the opposite even part)."""
+    ys = np.linspace(-12, 12, 2401).astype(np.float32)
+    got = oracle.silu(ys).astype(np.float64) + oracle.silu(-ys).astype(np.float64)
+    want = np.array([float(y) * math.tanh(float(y) / 2) for y in ys])
+    tol = 2 * np.spacing(np.abs(oracle.silu(np.abs(ys)))).astype(np.float64) + 1e-300
+    assert np.all(np.abs(got - want) <= tol)
+    assert np.all(got[ys != 0] > 0)          # y tanh(y/2) > 0 away from 0
+
+
+def test_silu_limits():
+    """y >> 0: sigmoid(y) = 1 to fp32 precision, silu(y) == y.  y << 0:
+    silu(y) = y e^y (1 - e^y + ...) -> 0 from below.  y -> 0: silu(y) / y -> 1/2."""
+    big = np.linspace(20, 80, 61).astype(np.float32)
+    np.testing.assert_array_equal(oracle.silu(big), big)
+    for y in (-20.0, -30.0, -50.0, -80.0):
+        v = float(oracle.silu(np.array([y], np.float32))[0])
+        assert v < 0
+        assert abs(v / (y * math.exp(y)) - 1) <= 1e-6
+    for y in (1e-4, -1e-4, 1e-6):
+        v = float(oracle.silu(np.array([y], np.float32))[0])
+        assert abs(v / float(np.float32(y)) - 0.5) <= 1e-4
+
+
+def test_silu_minimum_is_at_minus_one_minus_lambert_w():
+    """silu has one minimum: silu'(y) = 0 gives (1 + y) e^-y = -1, so
+    y* = -1 - W(1/e) = -1.27846454... and silu(y*) = 1 + y* = -W(1/e)
+    (W = Lambert's W function, principal branch)."""
+    from scipy.special import lambertw
+    w = float(lambertw(1.0 / math.e).real)
+    y_star = -1.0 - w
+    ys = np.linspace(-1.6, -1.0, 60001).astype(np.float32)
+    v = oracle.silu(ys).astype(np.float64)
+    i = int(np.argmin(v))
+    assert abs(float(ys[i]) - y_star) <= 2e-3   # the minimum is flat: v - min ~ (y - y*)^2
+    assert abs(v[i] - (-w)) <= 2.0 ** -24 * w
+    assert np.all(np.diff(v[: i + 1]) <= 1e-7) and np.all(np.diff(v[i:]) >= -1e-7)
+
+
+# ---- H-BitLinear pinned through a Sylvester Hadamard weight
+
+def _sylvester(n):
+    from scipy.linalg import hadamard
+    return hadamard(n).astype(np.int8)
+
+
+def _x_with_exact_transform(n, seed, e=-3):
+    """x = (H v / sqrt(n)) 2^e for an integer v with max|v| = 127, n a power of
+    four (sqrt(n) a power of two): x is exact in fp32 and its normalised
+    transform is exactly v 2^e, so per-token quantisation returns v itself."""
+    rng = np.random.default_rng(seed)
+    v = rng.integers(-127, 128, size=n).astype(np.int64)
+    v[rng.integers(n)] = 127 * (1 if rng.random() < 0.5 else -1)
+    H = _sylvester(n).astype(np.int64)
+    x = (H @ v).astype(np.float64) / math.sqrt(n) * 2.0 ** e
+    assert np.all(np.float32(x) == x)
+    return x.astype(np.float32)[None, :], v
+
+
+@pytest.mark.parametrize("n", [16, 64, 256])
+def test_hbitlinear_with_a_hadamard_weight_returns_sqrt_n_x(n):
+    """An H-BitLinear whose ternary weight is the Sylvester matrix H (entries
+    +-1, so gamma = mean|W| = 1) computes H . dequant(quant(H x / sqrt(n))).
+    Since H H^T = n I that is sqrt(n) x, exactly when the quantiser's rounding
+    is exact (x built so that H x / sqrt(n) is an integer vector times 2^e)."""
+    H = _sylvester(n)
+    W = H.astype(np.float32) * np.float32(0.75)      # any |W| = c gives gamma = c, t = H
+    g, T, _ = oracle.quantize_weights(W)
+    assert g == np.float32(0.75)
+    np.testing.assert_array_equal(T, H)
+    x, v = _x_with_exact_transform(n, seed=n)
+    q, s, _ = oracle.quant_act(x, oracle.PRELUDE_FWHT)
+    np.testing.assert_array_equal(q[0].astype(np.int64), v)
+    y = oracle.bitlinear(x, T, np.float32(1.0), oracle.PRELUDE_FWHT)
+    np.testing.assert_array_equal(y, (np.float32(math.sqrt(n)) * x).astype(np.float32))
+    y = oracle.bitlinear(x, T, g, oracle.PRELUDE_FWHT)        # gamma scales the output
+    np.testing.assert_array_equal(y, (np.float32(0.75 * math.sqrt(n)) * x).astype(np.float32))
+
+
+@pytest.mark.parametrize("n", [64, 256])
+def test_hffn_with_hadamard_weights(n):
+    """The H-FFN W2 . silu(W1 . x) with both weights the Sylvester matrix
+    (gamma = 1): the first H-BitLinear returns sqrt(n) x exactly (previous
+    test), so the hidden activation is silu(sqrt(n) x); the second returns
+    H q / s with q / s the int8 rounding of H h / sqrt(n), i.e. sqrt(n) h plus
+    H e with |e| <= 1 / (2 s) per element: |out - sqrt(n) h| <= n / (2 s) +
+    fp32 error.  A dropped transform, a transposed stage order or a missing
+    activation breaks one of the two."""
+    H = _sylvester(n)
+    x, _ = _x_with_exact_transform(n, seed=3 * n, e=-5)
+    out, h = oracle.hffn(x, H, np.float32(1.0), H, np.float32(1.0), keep=True)
+    y1 = (np.float32(math.sqrt(n)) * x).astype(np.float32)
+    np.testing.assert_array_equal(h, oracle.silu(y1))
+    _, s2, _ = oracle.quant_act(h, oracle.PRELUDE_FWHT)
+    err = np.abs(out.astype(np.float64) - math.sqrt(n) * h.astype(np.float64))
+    bound = n / (2.0 * float(s2[0])) + 1e-5 * math.sqrt(n) * np.abs(h).max()
+    assert np.all(err <= bound), (err.max(), bound)
+    # and it is a real transform of h, not h itself: without the second
+    # Hadamard prelude the result would be H h, far from sqrt(n) h
+    assert np.abs(H.astype(np.float64) @ h[0] - math.sqrt(n) * h[0]).max() > 10 * bound
+
+
 def _ffn_case(M=6, H=64, I=128, seed=17):
     rng = np.random.default_rng(seed)
     Wg = (rng.standard_normal((I, H)) * 0.02).astype(np.float32)

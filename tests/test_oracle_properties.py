@@ -9,6 +9,8 @@ rounded operands), "The two checkpoints" (four codes to a byte); the
 "bitnetv2-model" README, "Special Features" (normalised Hadamard transform on
 power-of-two widths).
 """
+from fractions import Fraction
+
 import numpy as np
 import pytest
 
@@ -17,6 +19,7 @@ from hypothesis import given, settings, strategies as st  # noqa: E402
 from hypothesis.extra import numpy as hnp  # noqa: E402
 
 import oracle  # noqa: E402
+from tests.exact import nearest_f32  # noqa: E402
 
 SETTINGS = settings(max_examples=150, deadline=None)
 
@@ -79,6 +82,32 @@ def test_quant_codes_are_invariant_under_power_of_two_scaling(X, k):
 _w = st.floats(min_value=-4.0, max_value=4.0, allow_nan=False, allow_infinity=False, width=32)
 
 
+def assert_gamma_is_rounded_mean(W, g):
+    """gamma is the exact rational mean of |W| rounded to the nearest fp32
+    (subnormals included, where fp32 holds fewer than 24 significant bits):
+    within half an fp32 spacing at that mean, plus the few fp64 ulps the
+    accumulation of the sum may add (the mean is a real number; the oracle
+    sums in fp64 and rounds once)."""
+    exact = sum(Fraction(float(abs(v))) for v in W.ravel()) / W.size
+    near = nearest_f32(exact)
+    spacing = Fraction(float(np.spacing(np.float32(min(abs(near), np.float32(3.0e38))))))
+    bound = spacing / 2 + exact * Fraction(W.size + 2, 2 ** 52)
+    assert abs(Fraction(float(g)) - exact) <= bound, (float(g), float(exact))
+
+
+def test_gamma_of_a_single_subnormal_mean():
+    """Regression case: one weight at the smallest normal fp32 (2^-126), the
+    other eleven zero; the mean 2^-126 / 12 is subnormal in fp32, so gamma is
+    that value rounded at the subnormal spacing 2^-149."""
+    W = np.zeros((3, 4), np.float32)
+    W[0, 0] = np.float32(2.0 ** -126)
+    g, T, _ = oracle.quantize_weights(W)
+    assert g == nearest_f32(Fraction(2) ** -126 / 12)
+    assert_gamma_is_rounded_mean(W, g)
+    # |W[0,0]| / gamma = 12 > 1/2: code +1; the zeros stay 0
+    assert T[0, 0] == 1 and np.count_nonzero(T) == 1
+
+
 @SETTINGS
 @given(st.integers(1, 6).flatmap(lambda n: st.sampled_from([4, 8, 16]).flatmap(
     lambda k: hnp.arrays(np.float32, (n, k), elements=_w))))
@@ -86,8 +115,7 @@ def test_ternary_codes_follow_the_absmean_rule(W):
     """gamma is mean|W| (to fp32); t is in {-1, 0, 1}, never opposite to W,
     monotone in |W|, 0 well below gamma / 2 and +-1 well above it."""
     g, T, _ = oracle.quantize_weights(W)
-    mean = np.abs(W.astype(np.float64)).mean()
-    assert abs(float(g) - mean) <= 2.0 ** -23 * mean
+    assert_gamma_is_rounded_mean(W, g)
     assert set(np.unique(T)).issubset({-1, 0, 1})
     assert np.all(T.astype(np.int64) * np.sign(W) >= 0)
     if g == 0:
