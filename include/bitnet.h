@@ -256,7 +256,9 @@ BITNET_API int bitnet_ffn(const void *X, int x_dtype, int M, int H, int I,
  *              returns BITNET_ERR_WORKSPACE and launches nothing.
  *   Set-up     The first call on each device looks up the device address of
  *              the array (cudaGetSymbolAddress) with that device current; make
- *              that first call before any stream capture begins.
+ *              that first call before any stream capture begins.  The address
+ *              belongs to the device's context: after cudaDeviceReset call
+ *              bitnet_release_cache(), and the next call looks it up again.
  *   Sharing    All calls on a device share the one array and it keeps the last
  *              call's contents (nothing in it needs to start at zero).  Calls
  *              that can overlap on the GPU (different streams, no ordering
@@ -287,10 +289,14 @@ BITNET_API int bitnet_check_device_error(bitnet_stream_t stream);
  * context usable.  Returns BITNET_OK if the launch succeeded. */
 BITNET_API int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t stream);
 
-/* Empty the host-side cache of TMA tensor descriptors.  The cache is keyed
- * by device, pointer, shape, box and swizzle, so it stays correct when an
- * address is reused; it holds at most 16384 descriptors (it starts over when
- * full).  This call only releases its memory. */
+/* Empty the host-side cache of TMA tensor descriptors and forget the
+ * per-context state the library keeps: the device address of the
+ * no-allocation FFN scratch and which devices have the decode kernel's
+ * shared-memory attribute set.  The descriptor cache is keyed by device,
+ * pointer, shape, box and swizzle, so it stays correct when an address is
+ * reused; it holds at most 16384 descriptors (it starts over when full).
+ * After cudaDeviceReset (which ends the context those addresses and
+ * attributes belong to) call this before the next call into the library. */
 BITNET_API void bitnet_release_cache(void);
 
 /* Library version string. */

@@ -349,6 +349,11 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mw0, mw1, my, p);
 }
 
+// Devices whose context has the decode kernel's shared-memory attribute set
+// (a bit per device ordinal); cleared by bitnet_release_cache so that a
+// context created after cudaDeviceReset gets it again.
+std::atomic<uint64_t> g_dec_attr_set{0};
+
 using TcPlain = TcConfig<128, 256, 4, false>;
 using TcSilu = TcConfig<128, 256, 4, false, true>;
 using TcGlu = TcConfig<128, 256, 4, true>;
@@ -404,7 +409,7 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   p.flags = lp.flags & ~LAUNCH_PDL;     // keeps LAUNCH_PDL_INPUTS for the kernel
   // The shared-memory attribute belongs to each device's context: set it once
   // per device (a bit per device ordinal; ordinals past 63 set it every call).
-  static std::atomic<uint64_t> attr_set{0};
+  std::atomic<uint64_t>& attr_set = g_dec_attr_set;
   int dev = 0;
   BN_CHECK_CUDA(cudaGetDevice(&dev));
   const uint64_t bit = dev >= 0 && dev < 64 ? (uint64_t)1 << dev : 0;
@@ -536,6 +541,12 @@ int validate_linear(const int8_t* Xq, const float* xs, const int32_t* xrs, const
     return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   return BITNET_OK;
 }
+
+// Device address of the no-allocation FFN scratch (bitnet_ffn_noalloc), per
+// device ordinal, looked up once per context.
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
 
 }  // namespace
 }  // namespace bitnet
@@ -854,8 +865,16 @@ int bitnet_check_device_error(bitnet_stream_t stream) {
 }
 
 void bitnet_release_cache(void) {
-  std::lock_guard<std::mutex> lock(g_map_mu);
-  g_map_cache.clear();
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    g_map_cache.clear();
+  }
+  // per-context state: looked up / set again on the next call
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    for (int d = 0; d < kMaxDevices; ++d) g_noalloc_ptr[d] = nullptr;
+  }
+  g_dec_attr_set.store(0, std::memory_order_release);
 }
 
 const char* bitnet_version(void) { return "bitnet-b200 0.1.0 (sm_100a)"; }
@@ -901,9 +920,6 @@ extern "C" int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t st
 namespace bitnet {
 static __device__ __align__(256) uint8_t g_ffn_noalloc_scratch[BITNET_FFN_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
 
 int noalloc_scratch(void** out) {
   int dev = 0;

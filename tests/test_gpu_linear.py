@@ -45,6 +45,27 @@ def test_linear_int32_bit_exact(M, K, N):
     np.testing.assert_array_equal(got, oracle.contract(q, T))
 
 
+# Shapes with more 128 x 128 tiles than the 148 persistent CTAs: every CTA
+# runs two or more tiles, so each TMEM accumulator buffer is reused (the
+# epilogue's zeroing, the buffer-empty barrier's phase flip, the alternating
+# token-factor buffers); ragged last tiles in both directions.
+MULTI_TILE = [(2048, 2560, 1280), (2048, 256, 4096), (1500, 512, 2000)]
+
+
+@pytest.mark.parametrize("M,K,N", MULTI_TILE)
+def test_persistent_gemm_every_epilogue_bit_exact(M, K, N):
+    X, g, T, P, q, s, rs = _case(M, K, N, seed=M + 7 * N)
+    acc = oracle.contract(q, T)
+    np.testing.assert_array_equal(gpu_linear(q, s, rs, P, g, K, N, out=torch.int32), acc)
+    y = oracle.dequant(acc, s, g)
+    assert_f32_close(gpu_linear(q, s, rs, P, g, K, N, out=torch.float32), y, what="f32")
+    assert_bf16_matches(gpu_linear(q, s, rs, P, g, K, N, out=torch.bfloat16), y, what="bf16")
+    R = oracle.round_bf16(synthetic.activations(np.random.default_rng(M), M, N))
+    gotr = gpu_linear(q, s, rs, P, g, K, N, out=torch.bfloat16, flags=bn.BITNET_EPI_RESIDUAL,
+                      residual=dev(R).to(torch.bfloat16))
+    assert_bf16_matches(gotr, (R + y).astype(np.float32), what="bf16 residual")
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 2560, 2560), (16, 6912, 300), (300, 2560, 300),
                                    (200, 512, 2048)])
 def test_linear_f32_and_bf16(M, K, N):

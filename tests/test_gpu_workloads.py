@@ -75,6 +75,36 @@ def test_prefill_full_size_sampled(K, N):
                             what="prefill chain")
 
 
+@pytest.mark.parametrize("K,N", [(2560, 6912), (6912, 2560)])
+def test_prefill_full_size_int32_every_row(K, N):
+    """The persistent GEMM at the bench's size (4096 tokens, 1728 / 640 tiles
+    on 148 CTAs, so every CTA runs several tiles and reuses each accumulator
+    buffer): the int32 contraction of every token against the oracle's
+    integer matmul, bit for bit, on the device's own codes; the codes
+    themselves against the oracle's RMSNorm quantiser (chain tolerance); the
+    bf16 outputs of every row against the oracle's dequantisation."""
+    M = synthetic.WORKLOADS["prefill"].dims["M"]
+    seed = {(2560, 6912): 0, (6912, 2560): 1}[(K, N)]
+    inp = synthetic.linear_inputs(M, K, N, seed=seed)
+    P, g = _pack(inp["W"])
+    q, s, rs = bn.alloc_quant(M, K)
+    bn.bitnet_quant_act(dev(inp["X"]), q, s, rs, prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
+    Yi = torch.empty((M, N), dtype=torch.int32, device="cuda")
+    bn.bitnet_linear(q, s, rs, P, g, K, Yi, epilogue=bn.BITNET_I32)
+    Yb = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    bn.bitnet_linear(q, s, rs, P, g, K, Yb)
+    torch.cuda.synchronize()
+    go, T, _ = oracle.quantize_weights(inp["W"])
+    qd = q.cpu().numpy()
+    np.testing.assert_array_equal(rs.cpu().numpy(), qd.astype(np.int64).sum(axis=1))
+    qo, so, _ = oracle.quant_act(inp["X"], oracle.PRELUDE_RMSNORM, eps=1e-5)
+    assert_codes_chain(qd, qo, "prefill codes, every row")
+    acc = oracle.contract(qd, T)
+    np.testing.assert_array_equal(Yi.cpu().numpy(), acc)
+    assert_bf16_matches(Yb.float().cpu().numpy(), oracle.dequant(acc, s.cpu().numpy(), go),
+                        what="prefill bf16, every row")
+
+
 @pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 6912), (6912, 2560)])
 def test_decode_full_rows(K, N):
     inp = synthetic.linear_inputs(16, K, N, seed=K + N)
@@ -118,16 +148,17 @@ def test_ffn_block_full_size_sampled():
     bn.bitnet_ffn(bf16_dev(inp["x_bf16"]), packs[0][0], packs[0][1], packs[1][0], packs[1][1],
                   packs[2][0], packs[2][1], Y, ws, eps=1e-5)
     torch.cuda.synchronize()
-    rows = _rows(M, 12, seed=3)
+    # every row: the sub-norm codes (the GLU GEMM's m through the sub-norm
+    # quantiser) and the outputs
     T = {k: oracle.quantize_weights(inp[k]) for k in ("Wg", "Wu", "Wd")}
-    out, m, qm, sm = oracle.ffn_relu2(inp["x"][rows], T["Wg"][1], T["Wg"][0], T["Wu"][1],
+    out, m, qm, sm = oracle.ffn_relu2(inp["x"], T["Wg"][1], T["Wg"][0], T["Wu"][1],
                                       T["Wu"][0], T["Wd"][1], T["Wd"][0], eps=1e-5, keep=True)
     ws_np = ws.cpu().numpy()
     a256 = lambda n: (n + 255) // 256 * 256
     off = a256(M * H) + 2 * a256(M * 4) + a256(M * I * 4)
-    qm_dev = ws_np[off:off + M * I].view(np.int8).reshape(M, I)[rows]
-    assert_codes_chain(qm_dev, qm, "ffn sub-norm codes")
-    got = Y.float().cpu().numpy()[rows]
+    qm_dev = ws_np[off:off + M * I].view(np.int8).reshape(M, I)
+    assert_codes_chain(qm_dev, qm, "ffn sub-norm codes, every row")
+    got = Y.float().cpu().numpy()
     if code_mismatch_stats(qm_dev, qm)[0] == 0:
         assert_bf16_matches(got, out, what="ffn out")
     want = oracle.round_bf16(out).astype(np.float64)

@@ -52,6 +52,29 @@ def test_noalloc_ffn_matches_the_workspace_entry_point_twice():
     assert bn.bitnet_check_device_error() == bn.BITNET_OK
 
 
+@pytest.mark.parametrize("M", [1, 16])
+def test_noalloc_decode_ffn_matches_twice(M):
+    """At decode sizes (M <= 16) the GLU FFN runs gate and up as two
+    projections of one decode launch and keeps the up projection's fp32
+    output in a second piece of the scratch; that path too must match the
+    workspace entry point, twice in a row."""
+    H, I = 2560, 6912
+    inp = synthetic.ffn_inputs(M, H, I, seed=9)
+    (Pg, gg), (Pu, gu), (Pd, gd) = (_pack(inp[k]) for k in ("Wg", "Wu", "Wd"))
+    X = bf16_dev(inp["x_bf16"])
+    ref = torch.empty((M, H), dtype=torch.bfloat16, device="cuda")
+    ws = bn.alloc_ffn_workspace(M, H, I)
+    bn.bitnet_ffn(X, Pg, gg, Pu, gu, Pd, gd, ref, ws)
+    torch.cuda.synchronize()
+    ref_np = ref.float().cpu().numpy()
+    for call in range(2):
+        Y = torch.full((M, H), float("nan"), dtype=torch.bfloat16, device="cuda")
+        bn.bitnet_ffn_noalloc(X, Pg, gg, Pu, gu, Pd, gd, Y)
+        torch.cuda.synchronize()
+        assert_bf16_matches(Y.float().cpu().numpy(), ref_np, what=f"noalloc decode M={M} {call}")
+    assert bn.bitnet_check_device_error() == bn.BITNET_OK
+
+
 def test_noalloc_hadamard_ffn_matches_twice():
     M, D, F = 16, 512, 2048
     inp = synthetic.hffn_inputs(M, D, F, seed=6)
