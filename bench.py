@@ -252,6 +252,76 @@ def oracle_prefill_sample(target_s=12.0, max_tokens=PREFILL_M):
                       f"bf16 round), {dt:.1f} s on {threads} OpenMP threads"}
 
 
+def _timed(fn, min_s):
+    """Run fn until min_s seconds have passed (at least twice); seconds per run."""
+    fn()                                         # warm (page faults, thread pool)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s and n >= 2:
+            return dt / n
+
+
+def oracle_workload_baselines(per_case_s=0.6):
+    """The CPU oracle timed on this host for every secondary workload, on the
+    same synthetic inputs (seeds) as the GPU lines: the tiny linear and the
+    decode calls on one thread (a token or a few), the FFN block and the
+    H-FFN on all OpenMP threads over a bounded token sample, scaled to a full
+    call.  Reported baselines, not targets."""
+    import oracle
+    out = {}
+    prev = oracle.num_threads()
+    try:
+        oracle.set_threads(1)
+        d = synthetic.WORKLOADS["tiny"].dims
+        inp = synthetic.linear_inputs(d["M"], d["K"], d["N"], seed=0)
+        g, T, _ = oracle.quantize_weights(inp["W"])
+        dt = _timed(lambda: oracle.bitlinear(inp["X"], T, g), per_case_s)
+        out["tiny"] = {"us_per_call": dt * 1e6, "cores": 1, "kind": "oracle",
+                       "sample": "the whole call (quant + contraction + dequant), 1 thread"}
+        dec = []
+        for K, N in DECODE_KN:
+            inp = synthetic.linear_inputs(max(DECODE_M), K, N, seed=K + N)
+            g, T, _ = oracle.quantize_weights(inp["W"])
+            for M in DECODE_M:
+                q, s, _ = oracle.quant_act(inp["X"][:M])
+                dt = _timed(lambda: oracle.round_bf16(oracle.dequant(oracle.contract(q, T), s, g)),
+                            per_case_s / 3)
+                dec.append({"M": M, "K": K, "N": N, "us_per_call": dt * 1e6,
+                            "GB_s": decode_bytes(M, K, N) / dt / 1e9, "cores": 1,
+                            "kind": "oracle", "sample": "the whole call (contraction + dequant "
+                                                        "+ bf16 round of int8 codes), 1 thread"})
+        out["decode"] = dec
+        oracle.set_threads(prev)
+        d = synthetic.WORKLOADS["hffn"].dims
+        inp = synthetic.hffn_inputs(d["M"], d["D"], d["F"], seed=0)
+        g1, T1, _ = oracle.quantize_weights(inp["W1"])
+        g2, T2, _ = oracle.quantize_weights(inp["W2"])
+        rows = 128
+        dt = _timed(lambda: oracle.hffn(inp["X"][:rows], T1, g1, T2, g2), per_case_s)
+        full = dt * d["M"] / rows
+        out["hffn"] = {"us": full * 1e6, "TOPS": 2 * 2 * d["M"] * d["D"] * d["F"] / full / 1e12,
+                       "cores": prev, "kind": "oracle",
+                       "sample": f"{rows} of {d['M']} tokens, scaled to the full call"}
+        d = synthetic.WORKLOADS["ffn"].dims
+        inp = synthetic.ffn_inputs(d["M"], d["H"], d["I"], seed=0)
+        Tw = {k: oracle.quantize_weights(inp[k]) for k in ("Wg", "Wu", "Wd")}
+        rows = 32
+        dt = _timed(lambda: oracle.round_bf16(oracle.ffn_relu2(
+            inp["x"][:rows], Tw["Wg"][1], Tw["Wg"][0], Tw["Wu"][1], Tw["Wu"][0], Tw["Wd"][1],
+            Tw["Wd"][0], eps=1e-5)), per_case_s)
+        full = dt * d["M"] / rows
+        out["ffn"] = {"us": full * 1e6,
+                      "TOPS": (2 * 2 * d["M"] * d["H"] * d["I"] + 2 * d["M"] * d["I"] * d["H"])
+                      / full / 1e12, "cores": prev, "kind": "oracle",
+                      "sample": f"{rows} of {d['M']} tokens, scaled to the full block"}
+    finally:
+        oracle.set_threads(prev)
+    return out
+
+
 def run_reference(args, world, rank):
     """Reference arm: the CPU oracle as it stands, on this host's cores."""
     if rank != 0:
@@ -801,6 +871,20 @@ def run_b200(args, world, rank, local):
             "tiny": extra(bench_tiny),
             "online_ternarisation": extra(bench_online),
         }
+        if not args.no_cpu_baseline:
+            # the oracle beside every secondary workload (same inputs)
+            try:
+                base = oracle_workload_baselines()
+                w = line["workloads"]
+                for name in ("tiny", "hffn", "ffn"):
+                    if isinstance(w.get(name), dict):
+                        w[name]["cpu_baseline"] = base[name]
+                for rec in w["decode"]:
+                    for b in base["decode"]:
+                        if (b["M"], b["K"], b["N"]) == (rec["M"], rec["K"], rec["N"]):
+                            rec["cpu_baseline"] = b
+            except Exception as e:        # noqa: BLE001
+                line["workloads"]["cpu_baseline_error"] = f"{type(e).__name__}: {e}"
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

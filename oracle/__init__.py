@@ -63,6 +63,8 @@ def _load():
         "orc_ffn_relu2": (i32, [P, i32, i32, i32, P, f32, P, f32, P, f32, P, P, f32, i32,
                                 P, P, P, P]),
         "orc_hffn": (i32, [P, i32, i32, i32, P, f32, P, f32, P, P]),
+        "orc_set_threads": (None, [i32]),
+        "orc_get_threads": (i32, []),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -302,5 +304,12 @@ def f32_to_bf16_bits(x):
 
 def num_threads():
     """Threads the OpenMP parts of the oracle use."""
-    v = os.environ.get("OMP_NUM_THREADS")
-    return int(v) if v else (os.cpu_count() or 1)
+    return int(_load().orc_get_threads())
+
+
+def set_threads(n):
+    """Set the threads of the OpenMP parts of the oracle (plumbing, no
+    arithmetic); returns the previous count."""
+    prev = num_threads()
+    _load().orc_set_threads(int(n))
+    return prev

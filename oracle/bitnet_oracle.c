@@ -37,6 +37,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORC_OK 0
 #define ORC_ERR_OVERFLOW 1
@@ -416,4 +419,25 @@ int orc_fwht(const float *X, int M, int n, float *out)
         if (err) return err;
     }
     return ORC_OK;
+}
+
+/* ------------------------------------------------------ threading (plumbing) */
+
+/* Threads the OpenMP loops above use (1 when built without OpenMP). */
+void orc_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+int orc_get_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
 }
