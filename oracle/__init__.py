@@ -63,6 +63,8 @@ def _load():
         "orc_ffn_relu2": (i32, [P, i32, i32, i32, P, f32, P, f32, P, f32, P, P, f32, i32,
                                 P, P, P, P]),
         "orc_hffn": (i32, [P, i32, i32, i32, P, f32, P, f32, P, P]),
+        "orc_block_tail": (i32, [P, P, i32, i32, i32, P, f32, P, f32, P, f32, P, f32, P, P, P,
+                                 f32, P, P]),
         "orc_set_threads": (None, [i32]),
         "orc_get_threads": (i32, []),
     }
@@ -271,6 +273,25 @@ def ffn_relu2(x, Tg, gg, Tu, gu, Td, gd, pre_gain=None, sub_gain=None, eps=1e-5,
     if keep:
         return out, m, qm, sm
     return out
+
+
+def block_tail(a, x, To, go, Tg, gg, Tu, gu, Td, gd, attn_gain=None, post_gain=None,
+               sub_gain=None, eps=1e-5, keep=False):
+    """The block after attention: h = x + o_proj(attn_sub_norm(a)), then the
+    W1.58A8 FFN with residual on h.  Returns fp32 out (and h when ``keep``)."""
+    a, x = _f32(a), _f32(x)
+    M, H = x.shape
+    I = Tg.shape[0]
+    To, Tg, Tu, Td = _i8(To), _i8(Tg), _i8(Tu), _i8(Td)
+    gains = [None if g is None else _f32(g) for g in (attn_gain, post_gain, sub_gain)]
+    out = np.empty((M, H), dtype=np.float32)
+    h = np.empty((M, H), dtype=np.float32) if keep else None
+    f = ctypes.c_float
+    _check(_load().orc_block_tail(_p(a), _p(x), M, H, I, _p(To), f(float(go)), _p(Tg),
+                                  f(float(gg)), _p(Tu), f(float(gu)), _p(Td), f(float(gd)),
+                                  _p(gains[0]), _p(gains[1]), _p(gains[2]), f(eps), _p(h),
+                                  _p(out)), "block_tail")
+    return (out, h) if keep else out
 
 
 def hffn(x, T1, g1, T2, g2, keep=False):

@@ -367,6 +367,31 @@ int orc_ffn_relu2(const float *x, int M, int H, int I,
     return err;
 }
 
+/* The block after attention ([NN] "The block, in order"):
+ *   h   = x + o_proj(attn_sub_norm(a))          (a = attention output)
+ *   out = h + down_proj(ffn_sub_norm(relu(gate_proj(z))^2 * up_proj(z))),
+ *         z = post_attention_layernorm(h)
+ * a, x [M][H] fp32 (bf16 inputs widened exactly by the caller); To [H][H],
+ * Tg, Tu [I][H], Td [H][I] ternary codes; gains [H] / [I] or NULL; h is
+ * kept in fp32 (written to h_out when non-NULL); out [M][H] fp32. */
+int orc_block_tail(const float *a, const float *x, int M, int H, int I,
+                   const int8_t *To, float go, const int8_t *Tg, float gg,
+                   const int8_t *Tu, float gu, const int8_t *Td, float gd,
+                   const float *attn_gain, const float *post_gain, const float *sub_gain,
+                   float eps, float *h_out, float *out)
+{
+    int64_t MH = (int64_t)M * H;
+    float *h = (float *)malloc(sizeof(float) * (size_t)MH + 4);
+    int err = orc_bitlinear(a, M, H, ORC_PRELUDE_RMSNORM, attn_gain, eps, To, go, H, x, h);
+    if (!err) {
+        if (h_out) memcpy(h_out, h, sizeof(float) * (size_t)MH);
+        err = orc_ffn_relu2(h, M, H, I, Tg, gg, Tu, gu, Td, gd, post_gain, sub_gain, eps, 1,
+                            out, NULL, NULL, NULL);
+    }
+    free(h);
+    return err;
+}
+
 /* The H-BitLinear FFN ([H1] "H-BitLinear Feed-Forward Network: 512 -> 2048
  * -> 512", "Activation function: silu", "Hadamard transform-based linear
  * layers"): y = W2 . silu(W1 . x), each projection an H-BitLinear, i.e. a

@@ -320,3 +320,67 @@ def test_hffn_matches_its_written_out_steps():
     np.testing.assert_array_equal(h, H)
     q2, s2, _ = oracle.quant_act(oracle.fwht(H))
     np.testing.assert_array_equal(out, oracle.dequant(oracle.contract(q2, T2), s2, g2))
+
+
+# ---- the block after attention: o_proj with attn_sub_norm, residual, FFN
+
+def _tail_case(M=5, H=64, I=128, seed=31):
+    rng = np.random.default_rng(seed)
+    Ws = {k: (rng.standard_normal(shape) * 0.02).astype(np.float32)
+          for k, shape in (("Wo", (H, H)), ("Wg", (I, H)), ("Wu", (I, H)), ("Wd", (H, I)))}
+    q = {k: oracle.quantize_weights(W) for k, W in Ws.items()}
+    a = rng.standard_normal((M, H)).astype(np.float32)
+    x = rng.standard_normal((M, H)).astype(np.float32)
+    w = (q["Wo"][1], q["Wo"][0], q["Wg"][1], q["Wg"][0], q["Wu"][1], q["Wu"][0], q["Wd"][1],
+         q["Wd"][0])
+    gains = dict(attn_gain=rng.uniform(0.5, 1.5, H).astype(np.float32),
+                 post_gain=rng.uniform(0.5, 1.5, H).astype(np.float32),
+                 sub_gain=rng.uniform(0.5, 1.5, I).astype(np.float32))
+    return a, x, w, gains
+
+
+def test_block_tail_attn_sub_norm_undoes_scaling():
+    """nnterp "bitnet", "Scaling inside a sublayer is undone by the sub-norm":
+    scaling the attention output a by 2^k leaves the block's output bit for
+    bit unchanged when eps = 0 (RMSNorm(2^k a) = RMSNorm(a) exactly)."""
+    a, x, w, gains = _tail_case()
+    base = oracle.block_tail(a, x, *w, eps=0.0, **gains)
+    for k in (-3, 1, 5):
+        np.testing.assert_array_equal(
+            oracle.block_tail(a * np.float32(2.0 ** k), x, *w, eps=0.0, **gains), base)
+
+
+def test_block_tail_reduces_to_the_ffn_when_o_proj_is_zero():
+    """All-zero o_proj weights (gamma 0, every code 0) give o = 0 exactly, so
+    h = x and the block is the pinned FFN of x."""
+    a, x, w, gains = _tail_case(seed=32)
+    To0 = np.zeros_like(w[0])
+    got = oracle.block_tail(a, x, To0, np.float32(0.0), *w[2:], **gains)
+    want = oracle.ffn_relu2(x, *w[2:], pre_gain=gains["post_gain"], sub_gain=gains["sub_gain"])
+    np.testing.assert_array_equal(got, want)
+
+
+def test_block_tail_reduces_to_o_proj_when_the_ffn_is_zero():
+    """All-zero gate/up weights give m = 0, whose sub-norm codes are 0 (zero
+    row: q = 0, s = 1), so the FFN adds exactly 0 and the block is
+    x + BitLinear(RMSNorm(a)) (the pinned BitLinear with a residual)."""
+    a, x, w, gains = _tail_case(seed=33)
+    Z = np.zeros_like(w[2])
+    got, h = oracle.block_tail(a, x, w[0], w[1], Z, np.float32(0.0), Z, np.float32(0.0), w[6],
+                               w[7], keep=True, **gains)
+    want = oracle.bitlinear(a, w[0], w[1], oracle.PRELUDE_RMSNORM, gain=gains["attn_gain"],
+                            residual=x)
+    np.testing.assert_array_equal(h, want)
+    np.testing.assert_array_equal(got, want)
+
+
+
+def test_block_tail_ffn_residual_is_h():
+    """The FFN's residual is h (the stream after the attention residual), not
+    x: out = fl32(h + FFN_without_residual(h)) bit for bit."""
+    a, x, w, gains = _tail_case(seed=34)
+    out, h = oracle.block_tail(a, x, *w, keep=True, **gains)
+    d = oracle.ffn_relu2(h, *w[2:], pre_gain=gains["post_gain"], sub_gain=gains["sub_gain"],
+                         residual=False)
+    np.testing.assert_array_equal(out, (h + d).astype(np.float32))
+    assert not np.array_equal(out, (x + d).astype(np.float32))
