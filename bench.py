@@ -609,9 +609,10 @@ def bench_ffn(torch, bn, device, iters=20):
 def bench_decode_ffn(torch, bn, device, reps=3):
     """The W1.58A8 block FFN at decode sizes (M = 1, 4, 16 tokens of the
     2560 -> 6912 -> 2560 FFN): back-to-back bitnet_ffn calls in a CUDA graph
-    over a pool of weight sets larger than twice the L2.  Four launches per
-    call (quant, gate + up, relu^2 * up with the sub-norm quant, down); GB/s
-    counts the three packed weight matrices, x (read twice) and y."""
+    over a pool of weight sets larger than twice the L2, as the default
+    four-launch route (quant, gate + up, relu^2 * up with the sub-norm quant,
+    down) and as one persistent launch per FFN (BITNET_FFN_SINGLE_LAUNCH).  GB/s counts the three packed
+    weight matrices, x (read twice) and y."""
     cfg = synthetic.WORKLOADS["ffn"].dims
     H, I = cfg["H"], cfg["I"]
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
@@ -633,26 +634,31 @@ def bench_decode_ffn(torch, bn, device, reps=3):
         ws = bn.alloc_ffn_workspace(M, H, I, device=device)
         step_bytes = set_bytes + 3 * 2 * M * H      # + x (twice: norm, residual) and y, bf16
 
-        def run(st, w):
-            bn.bitnet_ffn(X, w[0][0], w[0][1], w[1][0], w[1][1], w[2][0], w[2][1], Y, ws,
-                          variant=bn.BITNET_FFN_RELU2_GLU, eps=1e-5, stream=st)
-        run(None, sets[0])
-        torch.cuda.synchronize()
-        graph = torch.cuda.CUDAGraph()
-        stream = torch.cuda.Stream(device)
-        with torch.cuda.stream(stream):
-            graph.capture_begin(capture_error_mode="thread_local")
-            for w in sets:
-                run(stream, w)
-            graph.capture_end()
-        torch.cuda.synchronize()
-        graph.replay()
-        torch.cuda.synchronize()
-        best = min(time_loop(torch, graph.replay, 4) for _ in range(reps))
-        out.append({"M": M, "H": H, "I": I, "weight_sets_in_pool": pool,
-                    "us_per_ffn": best / (4 * pool) * 1e6,
-                    "GB_s": step_bytes * 4 * pool / best / 1e9})
-        del graph
+        rec = {"M": M, "H": H, "I": I, "weight_sets_in_pool": pool}
+        # one persistent launch per FFN (the default), and the four-launch route
+        for key, variant in (("", bn.BITNET_FFN_RELU2_GLU),
+                             ("_single_launch",
+                              bn.BITNET_FFN_RELU2_GLU | bn.BITNET_FFN_SINGLE_LAUNCH)):
+            def run(st, w):
+                bn.bitnet_ffn(X, w[0][0], w[0][1], w[1][0], w[1][1], w[2][0], w[2][1], Y, ws,
+                              variant=variant, eps=1e-5, stream=st)
+            run(None, sets[0])
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            stream = torch.cuda.Stream(device)
+            with torch.cuda.stream(stream):
+                graph.capture_begin(capture_error_mode="thread_local")
+                for w in sets:
+                    run(stream, w)
+                graph.capture_end()
+            torch.cuda.synchronize()
+            graph.replay()
+            torch.cuda.synchronize()
+            best = min(time_loop(torch, graph.replay, 4) for _ in range(reps))
+            rec["us_per_ffn" + key] = best / (4 * pool) * 1e6
+            rec["GB_s" + key] = step_bytes * 4 * pool / best / 1e9
+            del graph
+        out.append(rec)
     del sets
     return out
 

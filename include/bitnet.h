@@ -112,6 +112,12 @@ extern "C" {
 /* ----------------------------------------------------------- FFN variants */
 #define BITNET_FFN_RELU2_GLU      0  /* x + down(subnorm(relu(gate(z))^2 * up(z))), z = RMSNorm(x) */
 #define BITNET_FFN_HADAMARD_SILU  1  /* W2 . silu(W1 . x), each projection an H-BitLinear          */
+/* Launch option, OR-ed into the variant: run the decode-size GLU FFN (M <= 16,
+ * H and I multiples of 128) as one persistent cooperative launch instead of
+ * four launches (see bitnet_ffn).  It needs every SM at once, so callers
+ * whose other kernels run concurrently should leave it off.  No effect on
+ * other sizes or on the results' tolerance. */
+#define BITNET_FFN_SINGLE_LAUNCH 0x200
 
 typedef void *bitnet_stream_t;       /* a cudaStream_t */
 
@@ -225,10 +231,19 @@ BITNET_API size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant);
  *   Y = x + down_proj(RMSNorm(m; sub_norm_gain, eps))   (ffn_sub_norm)
  *   X, Y [M][H] of x_dtype / y_dtype (F32 or BF16); W_gate, W_up [I][H] and
  *   W_down [H][I] packed; gains may be NULL (all ones).
- *   Decode (M <= 16): gate and up run as two projections of one decode
- *   launch, and the sub-norm quantiser forms m from their fp32 outputs as it
- *   loads them (the workspace is then larger by M * I * 4 bytes); larger M
- *   runs the fused gate/up GEMM, whose epilogue forms m.
+ *   Decode (M <= 16): four launches -- the RMSNorm quantiser, gate and up as
+ *   two projections of one decode launch (fp32 outputs), the sub-norm
+ *   quantiser forming m from them as it loads them (the workspace is then
+ *   larger by M * I * 4 bytes), down with the residual.  With
+ *   BITNET_FFN_SINGLE_LAUNCH (H and I multiples of 128) the whole FFN runs
+ *   as one persistent cooperative launch with one CTA per SM (weights of
+ *   every projection bulk-copied into shared memory at start, x quantised by
+ *   every CTA, gate and up on mma.sync, one grid-wide exchange of m's sums of
+ *   squares through the workspace, the sub-norm codes formed by every CTA,
+ *   down with the residual); the exchange uses a fresh 64-bit epoch per
+ *   launch, so the workspace needs no initialisation, and calls sharing a
+ *   workspace must not overlap on the GPU.  Larger M runs the fused gate/up
+ *   GEMM, whose epilogue forms m.
  * BITNET_FFN_HADAMARD_SILU ("bitnetv2-model" README, "Architecture
  * Overview"): Y = W2 . silu(W1 . x), each an H-BitLinear (FWHT prelude);
  *   W_gate = W1 [I][H], W_down = W2 [H][I], W_up / gamma_up must be NULL,
@@ -241,6 +256,37 @@ BITNET_API int bitnet_ffn(const void *X, int x_dtype, int M, int H, int I,
                const float *pre_norm_gain, const float *sub_norm_gain, float eps,
                int variant, void *Y, int y_dtype,
                void *workspace, size_t ws_bytes, bitnet_stream_t stream);
+
+/* Workspace bytes bitnet_block_tail() needs. */
+BITNET_API size_t bitnet_block_tail_workspace_size(int M, int H, int I);
+
+/* The part of a W1.58A8 block after attention, at decode sizes, in one
+ * persistent launch (nnterp "bitnet", "The block, in order"):
+ *   h = x + o_proj(attn_sub_norm(a))                       (h kept in fp32)
+ *   Y = h + down_proj(ffn_sub_norm(relu(gate_proj(z))^2 * up_proj(z))),
+ *       z = post_attention_layernorm(h)
+ * every norm an RMSNorm with eps and a gain (NULL for all ones), every
+ * projection a BitLinear ("The projections quantize their inputs and
+ * weights").  A (attention output) and X (residual stream), H_out and Y are
+ * [M][H] of `dtype` (F32 or BF16); W_o [H][H], W_gate, W_up [I][H], W_down
+ * [H][I] packed.  H_out receives h in `dtype` (NULL to skip).
+ * One cooperative launch, one CTA per SM, two bounded grid-wide exchanges
+ * through the workspace (epochs, as bitnet_ffn at decode sizes): o_proj rows,
+ * then gate/up features, then down rows split over the CTAs; the codes of a,
+ * h and m formed by every CTA.  Supported: 1 <= M <= 16, H and I multiples
+ * of 128, staged weights and codes within an SM's shared memory (for the 2B
+ * model's 2560 / 6912, M <= 8); otherwise BITNET_ERR_UNSUPPORTED before any
+ * launch -- compose bitnet_quant_act (RMSNorm), bitnet_linear (fp32 output
+ * with the residual) and bitnet_ffn instead.  Calls sharing a workspace must
+ * not overlap on the GPU.  Errors: INVALID_ARG, UNSUPPORTED, WORKSPACE, CUDA. */
+BITNET_API int bitnet_block_tail(const void *A, const void *X, int dtype, int M, int H, int I,
+                                 const uint8_t *W_o, const float *gamma_o,
+                                 const uint8_t *W_gate, const float *gamma_gate,
+                                 const uint8_t *W_up, const float *gamma_up,
+                                 const uint8_t *W_down, const float *gamma_down,
+                                 const float *attn_norm_gain, const float *post_norm_gain,
+                                 const float *sub_norm_gain, float eps, void *H_out, void *Y,
+                                 void *workspace, size_t ws_bytes, bitnet_stream_t stream);
 
 /* bitnet_ffn without a workspace argument, for callers that cannot allocate
  * device memory: code running inside a CUDA stream capture whose mode forbids

@@ -20,6 +20,7 @@ from ._binding import (  # noqa: F401
     BITNET_EPI_RESIDUAL,
     BITNET_EPI_SILU,
     BITNET_EPI_TYPE_MASK,
+    BITNET_FFN_SINGLE_LAUNCH,
     BITNET_ERR_CUDA,
     BITNET_ERR_INVALID_ARG,
     BITNET_ERR_TIMEOUT,
@@ -36,9 +37,12 @@ from ._binding import (  # noqa: F401
     BITNET_PRELUDE_NONE,
     BITNET_PRELUDE_RMSNORM,
     BitnetError,
+    alloc_block_tail_workspace,
     alloc_ffn_workspace,
     alloc_packed,
     alloc_quant,
+    bitnet_block_tail,
+    bitnet_block_tail_workspace_size,
     bitnet_check_device_error,
     bitnet_debug_wait_timeout,
     bitnet_export_tw2,

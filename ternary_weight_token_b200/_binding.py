@@ -22,6 +22,7 @@ BITNET_EPI_SILU = 0x20
 BITNET_LAUNCH_PDL = 0x100
 BITNET_LAUNCH_PDL_INPUTS = 0x200
 BITNET_FFN_RELU2_GLU, BITNET_FFN_HADAMARD_SILU = 0, 1
+BITNET_FFN_SINGLE_LAUNCH = 0x200
 
 _DTYPE_CODE = {torch.float32: BITNET_F32, torch.bfloat16: BITNET_BF16, torch.int32: BITNET_I32}
 
@@ -62,6 +63,9 @@ def library():
         "bitnet_ffn_workspace_size": (S, [I, I, I, I]),
         "bitnet_ffn": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P, S, P]),
         "bitnet_ffn_noalloc": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P]),
+        "bitnet_block_tail_workspace_size": (S, [I, I, I]),
+        "bitnet_block_tail": (I, [P, P, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P, F, P, P, P,
+                                  S, P]),
         "bitnet_last_error": (ctypes.c_char_p, []),
         "bitnet_check_device_error": (I, [P]),
         "bitnet_debug_wait_timeout": (I, [U, P]),
@@ -200,6 +204,29 @@ def bitnet_ffn(X, W_gate, gamma_gate, W_up, gamma_up, W_down, gamma_down, Y, wor
                                 _ptr(pre_norm_gain), _ptr(sub_norm_gain), float(eps), int(variant),
                                 _ptr(Y), _dtype(Y), _ptr(workspace),
                                 workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def bitnet_block_tail_workspace_size(M, H, I):
+    return int(library().bitnet_block_tail_workspace_size(int(M), int(H), int(I)))
+
+
+def bitnet_block_tail(A, X, W_o, gamma_o, W_gate, gamma_gate, W_up, gamma_up, W_down,
+                      gamma_down, Y, workspace, H_out=None, attn_norm_gain=None,
+                      post_norm_gain=None, sub_norm_gain=None, eps=1e-5, stream=None):
+    """The block after attention at decode sizes, one launch (include/bitnet.h)."""
+    M, H = X.shape
+    I = W_gate.shape[0]
+    _check(library().bitnet_block_tail(
+        _ptr(A), _ptr(X), _dtype(X), M, H, I, _ptr(W_o), _ptr(gamma_o), _ptr(W_gate),
+        _ptr(gamma_gate), _ptr(W_up), _ptr(gamma_up), _ptr(W_down), _ptr(gamma_down),
+        _ptr(attn_norm_gain), _ptr(post_norm_gain), _ptr(sub_norm_gain), float(eps),
+        _ptr(H_out), _ptr(Y), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+
+
+def alloc_block_tail_workspace(M, H, I, device="cuda"):
+    return torch.empty(max(1, bitnet_block_tail_workspace_size(M, H, I)), dtype=torch.uint8,
+                       device=device)
 
 
 BITNET_FFN_NOALLOC_SCRATCH_BYTES = 8 << 20

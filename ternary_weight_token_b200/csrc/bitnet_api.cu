@@ -11,14 +11,18 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <chrono>
 #include <mutex>
+#include <random>
 #include <string>
 #include <unordered_map>
 
 #include "../../include/bitnet.h"
 #include "common.cuh"
+#include "ffn_decode.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_mma.cuh"
 #include "gemv_tc.cuh"
 #include "pack_weights.cuh"
 #include "quant_act.cuh"
@@ -45,6 +49,8 @@ int fail(int code, const char* fmt, ...) {
   } while (0)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align128(size_t x) { return (x + 127) & ~size_t(127); }
 
 constexpr int kMaxK = 16384;
 
@@ -224,7 +230,7 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   p.X = X; p.X2 = X2; p.M = M; p.K = K; p.gain = gain; p.eps = eps;
   p.fwht_c = (float)(1.0 / std::sqrt((double)K));
   p.Xq = Xq; p.scale = scale; p.rowsum = rowsum;
-  if (prelude != PRE_FWHT) {
+  if (!is_fwht(prelude)) {
     // NT threads x VPT 16-byte chunks must cover the row (K / 4 fp32 chunks,
     // K / 8 bf16 units of two chunks)
     const int k4 = K / 4;
@@ -236,14 +242,25 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   }
   // FWHT rows of 128 (fp32) / 256 (bf16) up to 2048 inputs: one warp per row
   // in registers; other widths: the row staged in shared memory
-  if (K <= 2048 && K >= (bf16 ? 256 : 128)) {
+  const bool silu = prelude == PRE_SILU_FWHT;
+  if (K <= 2048 && K >= (bf16 ? 256 : 128) && !(silu && bf16)) {
     void (*kw)(QuantParams) = nullptr;
-    switch (K) {
-      case 128: kw = quant_fwht_warp_kernel<128, false>; break;
-      case 256: kw = bf16 ? quant_fwht_warp_kernel<256, true> : quant_fwht_warp_kernel<256, false>; break;
-      case 512: kw = bf16 ? quant_fwht_warp_kernel<512, true> : quant_fwht_warp_kernel<512, false>; break;
-      case 1024: kw = bf16 ? quant_fwht_warp_kernel<1024, true> : quant_fwht_warp_kernel<1024, false>; break;
-      default: kw = bf16 ? quant_fwht_warp_kernel<2048, true> : quant_fwht_warp_kernel<2048, false>; break;
+    if (silu) {                    // fp32 hidden rows of the H-BitLinear FFN
+      switch (K) {
+        case 128: kw = quant_fwht_warp_kernel<128, false, true>; break;
+        case 256: kw = quant_fwht_warp_kernel<256, false, true>; break;
+        case 512: kw = quant_fwht_warp_kernel<512, false, true>; break;
+        case 1024: kw = quant_fwht_warp_kernel<1024, false, true>; break;
+        default: kw = quant_fwht_warp_kernel<2048, false, true>; break;
+      }
+    } else {
+      switch (K) {
+        case 128: kw = quant_fwht_warp_kernel<128, false>; break;
+        case 256: kw = bf16 ? quant_fwht_warp_kernel<256, true> : quant_fwht_warp_kernel<256, false>; break;
+        case 512: kw = bf16 ? quant_fwht_warp_kernel<512, true> : quant_fwht_warp_kernel<512, false>; break;
+        case 1024: kw = bf16 ? quant_fwht_warp_kernel<1024, true> : quant_fwht_warp_kernel<1024, false>; break;
+        default: kw = bf16 ? quant_fwht_warp_kernel<2048, true> : quant_fwht_warp_kernel<2048, false>; break;
+      }
     }
     const int rows_per_cta = 4;
     const int need = (M + rows_per_cta - 1) / rows_per_cta;
@@ -253,7 +270,9 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   const int threads = K >= 2048 ? 256 : 128;
   const size_t smem = (size_t)K * sizeof(float);
   const int grid = M < di.sms * 16 ? M : di.sms * 16;
-  void (*kern)(QuantParams) = bf16 ? quant_act_kernel<PRE_FWHT, true> : quant_act_kernel<PRE_FWHT, false>;
+  void (*kern)(QuantParams) =
+      silu ? (bf16 ? quant_act_kernel<PRE_SILU_FWHT, true> : quant_act_kernel<PRE_SILU_FWHT, false>)
+           : (bf16 ? quant_act_kernel<PRE_FWHT, true> : quant_act_kernel<PRE_FWHT, false>);
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
   return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, p);
 }
@@ -287,15 +306,41 @@ int launch_gemv(const LinearParams& p, cudaStream_t st) {
   return BITNET_OK;
 }
 
+// Schedule of the persistent GEMM: whole waves of full tiles, then the
+// remaining tiles (the last, partial wave) cut into `split` units of fewer
+// tokens each.  A unit costs about max(1 / split, kTailUnitFloor) of a full
+// tile (the weight tile is converted whole whatever the token count, and the
+// pipeline fill and epilogue do not shrink with it); the split minimises the
+// tail's rounds x unit cost, the smaller split on a tie.
+constexpr double kTailUnitFloor = 0.35;
+
+void tail_schedule(int num_tiles, int sms, int bn, int& full_units, int& split) {
+  full_units = (num_tiles / sms) * sms;
+  const int rest = num_tiles - full_units;
+  split = 1;
+  if (rest == 0) return;
+  double best = 1e30;
+  for (int f = 1; f <= 4; f *= 2) {
+    if (bn / f < kXBoxRows) break;
+    const int rounds = (rest * f + sms - 1) / sms;
+    const double cost = rounds * std::max(1.0 / f, kTailUnitFloor);
+    if (cost < best - 1e-9) {
+      best = cost;
+      split = f;
+    }
+  }
+}
+
 template <class C>
 int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1,
                   cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
-  CUtensorMap mx, mw0, mw1;
+  CUtensorMap mx, mxs, mw0, mw1;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return rc;
+  mxs = mx;
   // packed weight rows of BK/4 bytes, swizzled at that width (conflict-free
   // 16-byte loads in the converter)
   const CUtensorMapSwizzle wswz =
@@ -335,6 +380,13 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   p.tiles_n = (lp.N + C::TILE_N - 1) / C::TILE_N;
   const int tiles_m = (lp.M + C::BN - 1) / C::BN;
   p.num_tiles = p.tiles_n * tiles_m;
+  tail_schedule(p.num_tiles, di.sms, C::BN, p.full_units, p.tail_split);
+  p.num_units = p.full_units + (p.num_tiles - p.full_units) * p.tail_split;
+  if (p.tail_split > 1) {        // 32-row boxes for the split tail units
+    if (int rc = tensor_map_2d_u8(mxs, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
+                                  kXBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
+      return rc;
+  }
   p.xs = lp.xs; p.xrs = lp.xrs; p.gamma0 = lp.gamma; p.gamma1 = gamma1;
   p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type; p.flags = lp.flags;
   // One CTA per SM: request enough shared memory that two never co-reside
@@ -345,8 +397,8 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   if (smem > (size_t)di.max_smem_optin) smem = di.max_smem_optin;
   auto kern = gemm_tc_kernel<C>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
-  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mw0, mw1, my, p);
+  const int grid = p.num_units < di.sms ? p.num_units : di.sms;
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mxs, mw0, mw1, my, p);
 }
 
 // Devices whose context has the decode kernel's shared-memory attribute set
@@ -475,6 +527,45 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
 }
 
+// Decode for 1..16 tokens on short-lived CTAs (gemv_mma.cuh): 16 * RT weight
+// rows per CTA, RT chosen so the grid covers the SMs about twice.  Returns
+// BITNET_ERR_UNSUPPORTED when K is not a multiple of 32 or the staged rows
+// do not fit shared memory.
+template <int RT, int NTILE>
+int launch_gemv_mma_rt(const LinearParams& p, cudaStream_t st, const DeviceInfo& di) {
+  GmParams gp;
+  gp.lp = p;
+  gp.lp.flags &= ~LAUNCH_PDL;                  // keeps LAUNCH_PDL_INPUTS for the kernel
+  gp.rows_per_cta = 16 * RT;
+  gp.sw = p.ldw + kGmRowPad;
+  gp.sx = p.K + kGmRowPad;
+  gp.off_x = (int)align128((size_t)16 * RT * gp.sw);
+  const size_t smem = (size_t)gp.off_x + (size_t)p.M * gp.sx + 128;
+  if (smem > (size_t)di.max_smem_optin - 4096) return BITNET_ERR_UNSUPPORTED;
+  auto kern = gemv_mma_kernel<RT, NTILE>;
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  const int grid = (p.N + 16 * RT - 1) / (16 * RT);
+  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(kGmThreads), smem, st,
+                       gp);
+}
+
+int launch_gemv_mma(const LinearParams& p, cudaStream_t st) {
+  if (p.M < 1 || p.M > 16 || p.K % 32 != 0) return BITNET_ERR_UNSUPPORTED;
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const int tiles = (p.N + 15) / 16;
+  int rt = 1;
+  while (rt < 4 && (tiles + 2 * rt - 1) / (2 * rt) >= 2 * di.sms) rt *= 2;
+  if (p.M <= 8) {
+    if (rt == 1) return launch_gemv_mma_rt<1, 1>(p, st, di);
+    if (rt == 2) return launch_gemv_mma_rt<2, 1>(p, st, di);
+    return launch_gemv_mma_rt<4, 1>(p, st, di);
+  }
+  if (rt == 1) return launch_gemv_mma_rt<1, 2>(p, st, di);
+  if (rt == 2) return launch_gemv_mma_rt<2, 2>(p, st, di);
+  return launch_gemv_mma_rt<4, 2>(p, st, di);
+}
+
 // Projection i of a call as a call of its own.
 LinearParams segment_params(const LinearParams& p, int i) {
   LinearParams q = p;
@@ -515,6 +606,66 @@ int launch_linear(const LinearParams& p, cudaStream_t st) {
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Epochs of the grid-wide exchanges (persistent decode FFN, one-launch pack): a per-process
+// 64-bit counter started at a random value, so no launch reuses an epoch and
+// a workspace's initial contents match one with negligible probability.
+uint64_t next_epoch() {
+  static std::atomic<uint64_t> counter{[] {
+    std::random_device rd;
+    uint64_t v = ((uint64_t)rd() << 32) ^ (uint64_t)rd() ^
+                 (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
+    return v | 1u;
+  }()};
+  uint64_t e = counter.fetch_add(1, std::memory_order_relaxed);
+  return e == 0 ? counter.fetch_add(1, std::memory_order_relaxed) : e;
+}
+
+// The decode FFN in one cooperative launch (ffn_decode.cuh).  Returns
+// BITNET_ERR_UNSUPPORTED (nothing launched) when the shape does not fit it:
+// widths not multiples of 128, more than 64 features per CTA, or staged
+// weights and codes beyond the shared memory of an SM.
+int launch_ffn_decode(FfnDecodeParams p, cudaStream_t st, bool tail = false) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  if (p.M < 1 || p.M > 16 || p.H % 128 != 0 || p.I % 128 != 0) return BITNET_ERR_UNSUPPORTED;
+  int G = std::min(std::min(di.sms, kFdMaxGrid), (p.I + 7) / 8);
+  p.nf_per = (p.I + G - 1) / G;
+  p.groups = (p.nf_per + 7) / 8;
+  if (p.groups > kFdMaxGroups) return BITNET_ERR_UNSUPPORTED;
+  p.nr_per = (p.H + G - 1) / G;
+  if (p.nr_per > 32) return BITNET_ERR_UNSUPPORTED;
+  p.mpad = p.M <= 8 ? 8 : 16;
+  p.sw_h = p.ldwH + kFdRowPad;
+  p.sw_i = p.ldwI + kFdRowPad;
+  p.sx_h = p.H + kFdRowPad;
+  p.sx_i = p.I + kFdRowPad;
+  p.off_gu = 0;
+  p.off_d = (int)align128((size_t)p.groups * 16 * p.sw_h);
+  p.off_o = (int)align128((size_t)p.off_d + (size_t)p.nr_per * p.sw_i);
+  p.off_act = (int)align128((size_t)p.off_o + (tail ? (size_t)p.nr_per * p.sw_h : 0));
+  const size_t smem =
+      (size_t)p.off_act + (size_t)p.mpad * (size_t)std::max(p.sx_h, p.sx_i) + 128;
+  if (smem + sizeof(FfnDecodeShared) + 1024 > (size_t)di.max_smem_optin) return BITNET_ERR_UNSUPPORTED;
+  void (*kern)(FfnDecodeParams) = tail ? ffn_decode_kernel<true> : ffn_decode_kernel<false>;
+  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  int per_sm = 0;
+  BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFdThreads, smem));
+  if (per_sm < 1) return BITNET_ERR_UNSUPPORTED;
+  p.epoch = next_epoch();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)G);
+  cfg.blockDim = dim3(kFdThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;     // every CTA resident: the exchange waits on all
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kern, p));
+  return BITNET_OK;
+}
 
 int validate_linear(const int8_t* Xq, const float* xs, const int32_t* xrs, const uint8_t* W,
                     const float* gamma, int M, int N, int K, const void* Y, int epilogue,
@@ -563,7 +714,10 @@ size_t bitnet_packed_row_bytes(int K) {
 size_t bitnet_pack_workspace_size(int N, int K) {
   (void)N;
   (void)K;
-  return (size_t)kPackPartialBlocks * sizeof(double);
+  // one-launch path: partials and exchange flags; three-launch path: partials
+  const size_t fused = (size_t)kPackMaxGrid * (sizeof(double) + sizeof(unsigned long long));
+  const size_t split = (size_t)kPackPartialBlocks * sizeof(double);
+  return fused > split ? fused : split;
 }
 
 int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packed, float* gamma,
@@ -584,6 +738,34 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
   const bool bf16 = w_dtype == BITNET_BF16;
   const long long count = (long long)N * K;
   double* partials = reinterpret_cast<double*>(workspace);
+  if (N > 0) {
+    // one cooperative launch: two CTAs of 512 threads per SM
+    DeviceInfo di;
+    if (int rc = device_info(di)) return rc;
+    void (*kf)(const void*, int, int, int, long long, double*, unsigned long long*,
+               unsigned long long, float*, uint8_t*) =
+        bf16 ? pack_fused_kernel<true> : pack_fused_kernel<false>;
+    int per_sm = 0;
+    BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kPackFusedThreads, 0));
+    const int G = std::min(std::min(per_sm, 2) * di.sms, kPackMaxGrid);
+    if (G >= di.sms) {
+      unsigned long long* flags = reinterpret_cast<unsigned long long*>(partials + kPackMaxGrid);
+      const int ldw = (int)bitnet_packed_row_bytes(K);
+      const unsigned long long epoch = next_epoch();
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)G);
+      cfg.blockDim = dim3(kPackFusedThreads);
+      cfg.stream = st;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeCooperative;
+      attr[0].val.cooperative = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kf, W, N, K, ldw, count, partials, flags, epoch,
+                                       gamma, packed));
+      return BITNET_OK;
+    }
+  }
   if (int rc = launch_pdl(bf16 ? absmean_partial_kernel<true> : absmean_partial_kernel<false>,
                           dim3(kPackPartialBlocks), dim3(kPackThreads), 0, st, W, count,
                           partials))
@@ -736,9 +918,13 @@ size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant) {
   total += align256(m * (size_t)I * 4);        // fp32 hidden activation
   total += align256(m * (size_t)I);            // codes of the hidden activation
   total += align256(m * 4) * 2;                // its scale and rowsum
-  // decode (M <= 16) gate/up run as two projections of one launch: the up
-  // projection's fp32 output too
-  if (variant == BITNET_FFN_RELU2_GLU && M <= 16) total += align256(m * (size_t)I * 4);
+  // decode (M <= 16): the up projection's fp32 output (four-launch route),
+  // and the persistent launch's per-CTA partial sums and exchange flags
+  if ((variant & ~BITNET_FFN_SINGLE_LAUNCH) == BITNET_FFN_RELU2_GLU && M <= 16) {
+    total += align256(m * (size_t)I * 4);
+    total += align256((size_t)kFdMaxGrid * 16 * sizeof(double));
+    total += align256((size_t)kFdMaxGrid * sizeof(unsigned long long));
+  }
   return total;
 }
 
@@ -755,8 +941,11 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
     return fail(BITNET_ERR_INVALID_ARG, "x dtype must be F32 or BF16");
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16)
     return fail(BITNET_ERR_INVALID_ARG, "y dtype must be F32 or BF16");
+  const bool single = (variant & BITNET_FFN_SINGLE_LAUNCH) != 0;
+  const int variant_flags = variant;
+  variant &= ~BITNET_FFN_SINGLE_LAUNCH;
   if (variant != BITNET_FFN_RELU2_GLU && variant != BITNET_FFN_HADAMARD_SILU)
-    return fail(BITNET_ERR_INVALID_ARG, "unknown FFN variant %d", variant);
+    return fail(BITNET_ERR_INVALID_ARG, "unknown FFN variant %d", variant_flags);
   if (variant == BITNET_FFN_RELU2_GLU) {
     if (x_dtype != y_dtype)
       return fail(BITNET_ERR_UNSUPPORTED, "the residual FFN needs x and y of one dtype");
@@ -795,6 +984,10 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   float* hs = reinterpret_cast<float*>(ws);              ws += align256(m * 4);
   int32_t* hrs = reinterpret_cast<int32_t*>(ws);         ws += align256(m * 4);
   float* hid_up = reinterpret_cast<float*>(ws);          // decode GLU only
+  ws += align256(m * I * 4);
+  double* fd_partials = reinterpret_cast<double*>(ws);
+  ws += align256((size_t)kFdMaxGrid * 16 * sizeof(double));
+  unsigned long long* fd_flags = reinterpret_cast<unsigned long long*>(ws);
   const bool xbf = x_dtype == BITNET_BF16;
 
   LinearParams p1;
@@ -808,6 +1001,20 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   single_segment(p1);
   single_segment(p2);
 
+  if (variant == BITNET_FFN_RELU2_GLU && M <= 16 && single) {
+    // Decode: the whole FFN in one persistent launch when the shape fits it
+    FfnDecodeParams fp = {};
+    fp.X = X; fp.x_bf16 = xbf ? 1 : 0; fp.M = M; fp.H = H; fp.I = I;
+    fp.Wg = W_gate; fp.Wu = W_up; fp.Wd = W_down;
+    fp.gamma_g = gamma_gate; fp.gamma_u = gamma_up; fp.gamma_d = gamma_down;
+    fp.pre_gain = pre_norm_gain; fp.sub_gain = sub_norm_gain; fp.eps = eps;
+    fp.Y = Y; fp.y_bf16 = y_dtype == BITNET_BF16 ? 1 : 0;
+    fp.hid = hid; fp.hq = hq; fp.hs = hs; fp.hrs = hrs;
+    fp.partials = fd_partials; fp.flags = fd_flags;
+    fp.ldwH = (int)bitnet_packed_row_bytes(H); fp.ldwI = (int)bitnet_packed_row_bytes(I);
+    const int rc = launch_ffn_decode(fp, st);
+    if (rc != BITNET_ERR_UNSUPPORTED) return rc;
+  }
   if (variant == BITNET_FFN_RELU2_GLU && M <= 16) {
     // Decode: gate and up as two projections of one decode launch (fp32
     // outputs), relu(g)^2 * u formed by the sub-norm quantiser as it loads
@@ -839,13 +1046,84 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
     p2.resid = X;
     return launch_linear(p2, st);
   }
+  // H-BitLinear FFN: W1 writes its plain fp32 output; the second
+  // quantiser applies the SiLU as it loads the hidden rows (the same fp32
+  // operations the GEMM epilogue would apply, so the same values), then the
+  // transform.
   if (int rc = launch_quant(X, xbf, M, H, PRE_FWHT, nullptr, 0.0f, xq, xs, xrs, st)) return rc;
-  p1.flags = EPI_SILU;
+  p1.flags = 0;
   if (int rc = launch_linear(p1, st)) return rc;
-  if (int rc = launch_quant(hid, false, M, I, PRE_FWHT, nullptr, 0.0f, hq, hs, hrs, st)) return rc;
+  if (int rc = launch_quant(hid, false, M, I, PRE_SILU_FWHT, nullptr, 0.0f, hq, hs, hrs, st))
+    return rc;
   p2.flags = 0;
   p2.resid = nullptr;
   return launch_linear(p2, st);
+}
+
+size_t bitnet_block_tail_workspace_size(int M, int H, int I) {
+  if (M < 0 || H <= 0 || I <= 0) return 0;
+  const size_t m = (size_t)M;
+  return align256(m * (size_t)I * 4) + align256(m * (size_t)I) + 2 * align256(m * 4) +
+         align256((size_t)kFdMaxGrid * 16 * sizeof(double)) +
+         2 * align256((size_t)kFdMaxGrid * sizeof(unsigned long long)) +
+         align256(m * (size_t)H * 4);
+}
+
+int bitnet_block_tail(const void* A, const void* X, int dtype, int M, int H, int I,
+                      const uint8_t* W_o, const float* gamma_o, const uint8_t* W_gate,
+                      const float* gamma_gate, const uint8_t* W_up, const float* gamma_up,
+                      const uint8_t* W_down, const float* gamma_down, const float* attn_norm_gain,
+                      const float* post_norm_gain, const float* sub_norm_gain, float eps,
+                      void* H_out, void* Y, void* workspace, size_t ws_bytes,
+                      bitnet_stream_t stream) {
+  g_last_error.clear();
+  if (M < 0) return fail(BITNET_ERR_INVALID_ARG, "M=%d must be >= 0", M);
+  if (int rc = check_k(H)) return rc;
+  if (int rc = check_k(I)) return rc;
+  if (dtype != BITNET_F32 && dtype != BITNET_BF16)
+    return fail(BITNET_ERR_INVALID_ARG, "dtype must be F32 or BF16");
+  if (!(eps >= 0.0f && std::isfinite(eps)))
+    return fail(BITNET_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (M == 0) return BITNET_OK;
+  if (!A || !X || !W_o || !gamma_o || !W_gate || !gamma_gate || !W_up || !gamma_up || !W_down ||
+      !gamma_down || !Y)
+    return fail(BITNET_ERR_INVALID_ARG, "null pointer argument");
+  const void* ptrs[] = {A, X, W_o, gamma_o, W_gate, gamma_gate, W_up, gamma_up, W_down,
+                        gamma_down, Y, H_out, attn_norm_gain, post_norm_gain, sub_norm_gain};
+  for (const void* q : ptrs)
+    if (q && !aligned16(q)) return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (M > 16 || H % 128 != 0 || I % 128 != 0)
+    return fail(BITNET_ERR_UNSUPPORTED,
+                "the fused block tail runs at decode sizes (M <= 16, H and I multiples of 128); "
+                "compose bitnet_quant_act, bitnet_linear and bitnet_ffn otherwise");
+  const size_t need = bitnet_block_tail_workspace_size(M, H, I);
+  if (workspace == nullptr || ws_bytes < need)
+    return fail(BITNET_ERR_WORKSPACE, "workspace of %zu bytes needed", need);
+  if (!aligned16(workspace)) return fail(BITNET_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  const size_t m = (size_t)M;
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  FfnDecodeParams fp = {};
+  fp.hid = reinterpret_cast<float*>(ws);                  ws += align256(m * I * 4);
+  fp.hq = reinterpret_cast<int8_t*>(ws);                  ws += align256(m * I);
+  fp.hs = reinterpret_cast<float*>(ws);                   ws += align256(m * 4);
+  fp.hrs = reinterpret_cast<int32_t*>(ws);                ws += align256(m * 4);
+  fp.partials = reinterpret_cast<double*>(ws);            ws += align256((size_t)kFdMaxGrid * 16 * 8);
+  fp.flags = reinterpret_cast<unsigned long long*>(ws);   ws += align256((size_t)kFdMaxGrid * 8);
+  fp.flags_a = reinterpret_cast<unsigned long long*>(ws); ws += align256((size_t)kFdMaxGrid * 8);
+  fp.hbuf = reinterpret_cast<float*>(ws);
+  fp.X = X; fp.A = A; fp.x_bf16 = dtype == BITNET_BF16 ? 1 : 0;
+  fp.M = M; fp.H = H; fp.I = I;
+  fp.Wo = W_o; fp.gamma_o = gamma_o;
+  fp.Wg = W_gate; fp.Wu = W_up; fp.Wd = W_down;
+  fp.gamma_g = gamma_gate; fp.gamma_u = gamma_up; fp.gamma_d = gamma_down;
+  fp.attn_gain = attn_norm_gain; fp.pre_gain = post_norm_gain; fp.sub_gain = sub_norm_gain;
+  fp.eps = eps; fp.Y = Y; fp.H_out = H_out; fp.y_bf16 = fp.x_bf16;
+  fp.ldwH = (int)bitnet_packed_row_bytes(H); fp.ldwI = (int)bitnet_packed_row_bytes(I);
+  const int rc = launch_ffn_decode(fp, reinterpret_cast<cudaStream_t>(stream), true);
+  if (rc == BITNET_ERR_UNSUPPORTED)
+    return fail(BITNET_ERR_UNSUPPORTED, "staged weights and codes exceed shared memory "
+                "(M=%d, H=%d, I=%d)", M, H, I);
+  return rc;
 }
 
 const char* bitnet_last_error(void) { return g_last_error.c_str(); }

@@ -303,6 +303,55 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ------------------------------------------------- grid-wide exchange
+// For a cooperative launch (every CTA resident): each CTA publishes the
+// launch's 64-bit epoch in its own flag once its global writes are done, and
+// waits until every CTA's flag holds the epoch.  Epochs are never reused (the
+// host draws a fresh one per launch from a counter started at a random
+// value), so the flags need no reset and no zeroing.  Every thread of the CTA
+// calls it; warp 0 polls, bounded by kWaitLimitNs.  Returns false (device
+// error recorded) if the wait gave up.
+__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool grid_exchange(unsigned long long* flags, unsigned long long epoch,
+                                              int* ok_smem) {
+  __syncthreads();                               // this CTA's global writes are issued
+  if (threadIdx.x == 0) {
+    __threadfence();
+    st_release_u64(flags + blockIdx.x, epoch);
+    *ok_smem = 1;
+  }
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const unsigned long long t0 = global_timer_ns();
+    bool done = false;
+    for (uint32_t it = 0;; ++it) {
+      bool mine = true;
+      for (int i = lane; i < (int)gridDim.x; i += 32)
+        mine = mine && (ld_acquire_u64(flags + i) == epoch);
+      done = __all_sync(0xffffffffu, mine);
+      if (done) break;
+      if ((it & 7u) == 7u && global_timer_ns() - t0 > kWaitLimitNs) break;
+      __nanosleep(64);
+    }
+    if (!done && lane == 0) {
+      record_device_error(DEV_ERR_TIMEOUT);
+      *ok_smem = 0;
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
 // ------------------------------------------- programmatic dependent launch
 // Wait until the grids this one depends on have completed and their memory
 // is visible (returns at once for a launch without the PDL attribute).
@@ -317,6 +366,15 @@ __device__ __forceinline__ void grid_launch_dependents() {
 }
 
 // --------------------------------------------------------------- misc ALU
+// SiLU y / (1 + e^-y) in fp32 ("bitnetv2-model" README, "Architecture
+// Overview"): CUDA's expf (the full-precision function, not the fast
+// intrinsic) and IEEE fp32 add and division, a few fp32 ulp from the exact
+// value.  One definition for every kernel that applies it, so the GEMM
+// epilogue and the quantiser prelude give the same value.
+__device__ __forceinline__ float silu_f32(float y) {
+  return __fdiv_rn(y, __fadd_rn(1.0f, expf(-y)));
+}
+
 // Four unsigned bytes of `a` times four signed bytes of `b`, summed into c.
 __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   int d;

@@ -82,8 +82,14 @@ struct TcConfig {
 
 struct TcParams {
   int M, N, K;
-  int num_kb;                 // k stages = ceil(K / 128)
+  int num_kb;                 // k stages = ceil(K / BK)
   int tiles_n, num_tiles;
+  // Work units: tiles [0, full_units) are whole BN-token tiles (the full
+  // waves); each tile after them (the last, partial wave) is cut into
+  // tail_split units of BN / tail_split tokens, so the last wave's work is
+  // spread over more SMs.  num_units = full_units + (num_tiles - full_units)
+  // * tail_split.
+  int num_units, full_units, tail_split;
   const float* xs;            // [M] activation scales
   const int32_t* xrs;         // [M] sum of activation codes
   const float* gamma0;        // weight scale (gate weights for GLU)
@@ -97,9 +103,34 @@ struct TcParams {
 
 __device__ __forceinline__ int out_elem_bytes(int out_type) { return out_type == OUT_BF16 ? 2 : 4; }
 
+// Activation rows per TMA box of a tail unit: a unit of bn < BN tokens is
+// loaded as bn / 32 boxes (a second tensor map), each landing on a 1024-byte
+// boundary of the 128-byte-swizzled sub-tile; whole tiles load one box of BN
+// rows per 128-k sub-tile.
+constexpr int kXBoxRows = 32;
+
+// One work unit: weight tile tn, tokens [m0, m0 + bn).
+struct TcUnit {
+  int tn, m0, bn;
+};
+
+template <class C>
+__device__ __forceinline__ TcUnit tc_unit(const TcParams& p, int u) {
+  int tile = u, sub = 0, split = 1;
+  if (u >= p.full_units) {
+    const int v = u - p.full_units;
+    split = p.tail_split;
+    tile = p.full_units + v / split;
+    sub = v - (v / split) * split;
+  }
+  const int bn = C::BN / split;
+  return TcUnit{tile % p.tiles_n, (tile / p.tiles_n) * C::BN + sub * bn, bn};
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
+                   const __grid_constant__ CUtensorMap tm_xs,
                    const __grid_constant__ CUtensorMap tm_w0,
                    const __grid_constant__ CUtensorMap tm_w1,
                    const __grid_constant__ CUtensorMap tm_y, TcParams p) {
@@ -151,6 +182,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
+    if (p.tail_split > 1) tma_prefetch_desc(&tm_xs);
     tma_prefetch_desc(&tm_w0);
     if (C::GLU) tma_prefetch_desc(&tm_w1);
     if (p.tma_out) tma_prefetch_desc(&tm_y);
@@ -173,16 +205,25 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
-        const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
+      for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
+        const TcUnit t = tc_unit<C>(p, u);
+        const int tn = t.tn;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) goto producer_done;
-          mbar_arrive_expect_tx(&full[st], C::TX_BYTES);
+          mbar_arrive_expect_tx(&full[st], (uint32_t)(t.bn * C::BK + C::NW * C::W_STAGE));
+          if (t.bn == C::BN) {                // a whole tile: one box per 128-k sub-tile
 #pragma unroll
-          for (int xs = 0; xs < C::BK / 128; ++xs)
-            tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
-                        kb * C::BK + 128 * xs, tm * C::BN);
+            for (int xs = 0; xs < C::BK / 128; ++xs)
+              tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
+                          kb * C::BK + 128 * xs, t.m0);
+          } else {                            // a tail unit: bn / 32 boxes of 32 rows
+#pragma unroll
+            for (int xs = 0; xs < C::BK / 128; ++xs)
+              for (int r = 0; r < t.bn; r += kXBoxRows)
+                tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB + r * 128, &tm_xs, &full[st],
+                            kb * C::BK + 128 * xs, t.m0 + r);
+          }
           if (C::GLU) {                       // rows 0-63 gate, 64-127 up
             tma_load_2d(sw + st * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
                         tn * C::TILE_N);
@@ -209,9 +250,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // accumulator buffer after reading it, before handing it back.
     if (lane == 0) {
       const uint32_t me = warp == 1 ? 0u : 1u;
-      const uint32_t idesc = make_idesc_i8(C::BM, C::BN);
       uint32_t it = 0, tcount = 0;
-      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++tcount) {
+        const uint32_t idesc = make_idesc_i8(C::BM, tc_unit<C>(p, u).bn);
         const uint32_t ab = tcount & 1u, use = tcount >> 1;
         if (!mbar_wait(&accempty[ab], use & 1u, abort_flag)) break;
         tc_fence_after();
@@ -245,7 +286,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     const int q = warp & 3;
     const int row = 32 * q + lane;               // weight row within the tile = TMEM lane
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16) + a_col0;
-    const uint32_t total = (uint32_t)((p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) /
+    const uint32_t total = (uint32_t)((p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) /
                                       (int)gridDim.x) * (uint32_t)p.num_kb;
     for (uint32_t it = group; it < total; it += C::CONV_GROUPS) {
       const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
@@ -301,9 +342,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_arrive(&accempty[1]);
     }
     uint32_t tcount = 0, chunk_count = 0, xcount = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
-      const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
-      const int m0 = tm * C::BN;
+    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++tcount) {
+      const TcUnit unit = tc_unit<C>(p, u);
+      const int tn = unit.tn;
+      const int m0 = unit.m0;
       // first output feature of this warp (GLU: warps 0-1 hold gate rows,
       // warps 2-3 the up rows of the same features)
       const int nq0 = tn * C::TILE_N + 32 * (C::GLU ? (q & 1) : q);
@@ -312,7 +354,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       int* tok_rs = s_tok_rs[ab];
       // This buffer was last read for tile tcount - 2; every warp has since
       // arrived on the other buffer's barrier, so no warp still reads it.
-      for (int j = 32 * q + lane; j < C::BN; j += 128) {
+      for (int j = 32 * q + lane; j < unit.bn; j += 128) {
         const int m = m0 + j;
         float2 f0 = make_float2(0.0f, 0.0f), f1 = make_float2(0.0f, 0.0f);
         int rs = 0;
@@ -334,7 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int n = nq0 + lane;
       const bool n_ok = n < p.N;
 #pragma unroll 1
-      for (int c = 0; c < C::BN / 32; ++c, ++chunk_count) {
+      for (int c = 0; c < unit.bn / 32; ++c, ++chunk_count) {
         const int mc = m0 + 32 * c;              // first token of this chunk
         if (mc >= p.M) {                         // past the last token: only re-zero
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);

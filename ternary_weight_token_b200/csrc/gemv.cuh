@@ -94,14 +94,6 @@ __device__ __forceinline__ void dequant_factor(float gamma, float s, float& f_hi
   f_lo = __fdiv_rn(r, s);
 }
 
-// SiLU y / (1 + e^-y) in fp32 ("bitnetv2-model" README, "Architecture
-// Overview"): CUDA's expf (the full-precision function, not the fast
-// intrinsic) and IEEE fp32 add and division, a few fp32 ulp from the exact
-// value.
-__device__ __forceinline__ float silu_f32(float y) {
-  return __fdiv_rn(y, __fadd_rn(1.0f, expf(-y)));
-}
-
 // Epilogue tail shared by the decode and prefill kernels: fp32 value ->
 // optional SiLU / residual -> stored element.
 __device__ __forceinline__ void store_value(void* Y, const void* resid, size_t idx, float y,

@@ -6,8 +6,10 @@
 // checkpoint stores them ternary, four to a byte, with a weight_scale.
 // "BitNet b1.58 2B4T", "Model Details": absmean quantisation.
 //
-// Three launches on the caller's stream (with programmatic dependent launch:
-// each waits for its predecessor before touching global memory):
+// One cooperative launch (pack_fused_kernel, below) when the device can hold
+// its grid at once; otherwise three launches on the caller's stream (with
+// programmatic dependent launch: each waits for its predecessor before
+// touching global memory):
 //   1. absmean_partial: a fixed grid sums |W| in fp64, one partial per CTA in
 //      a fixed order (deterministic run to run);
 //   2. absmean_final: one CTA adds the partials in a fixed order and writes
@@ -152,6 +154,151 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
         const uint4* src = reinterpret_cast<const uint4*>(
             reinterpret_cast<const uint16_t*>(W) + (size_t)n * K + k0);
         uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 1);
+        const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          w[2 * j] = bf16_bits_to_f32(u[j] & 0xffffu);
+          w[2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+        }
+      } else {
+        const float4* src = reinterpret_cast<const float4*>(
+            reinterpret_cast<const float*>(W) + (size_t)n * K + k0);
+        uint4 v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(src + j);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          w[4 * j] = __uint_as_float(v[j].x); w[4 * j + 1] = __uint_as_float(v[j].y);
+          w[4 * j + 2] = __uint_as_float(v[j].z); w[4 * j + 3] = __uint_as_float(v[j].w);
+        }
+      }
+      word = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          word |= ternary_code(w[4 * i + j], g, thr) << (8 * j + 2 * i);
+    }
+    reinterpret_cast<uint32_t*>(packed + (size_t)n * ldw)[wi] = word;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Both passes in one cooperative launch (every CTA resident): each CTA adds
+// |W| over its grid-stride share in fp64 (the same loop as
+// absmean_partial_kernel, so the per-CTA order is fixed), publishes its
+// partial and the launch's epoch, waits (bounded) for every CTA's epoch, then
+// adds all partials in a fixed order -- the same gamma in every CTA, written
+// once by CTA 0 -- and packs its share of the codes.  The second read of W
+// mostly hits L2: the pass that read it just finished and the matrix is
+// smaller than L2.
+constexpr int kPackFusedThreads = 512;
+constexpr int kPackMaxGrid = 1024;        // partial / flag slots in the workspace
+
+template <bool BF16>
+__global__ void __launch_bounds__(kPackFusedThreads) pack_fused_kernel(
+    const void* W, int N, int K, int ldw, long long count, double* partials,
+    unsigned long long* flags, unsigned long long epoch, float* gamma_out, uint8_t* packed) {
+  __shared__ double red[33];
+  __shared__ int xok;
+  __shared__ float s_gamma;
+  // pass 1: this CTA's partial sum of |W|
+  double acc = 0.0;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  const long long t0 = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (BF16) {
+    const uint4* v8 = reinterpret_cast<const uint4*>(W);
+    const long long nv = count / 8;
+    double a4[4] = {0.0, 0.0, 0.0, 0.0};
+    long long i = t0;
+    for (; i + 3 * stride < nv; i += 4 * stride) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldcg(v8 + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          a4[u] += fabs((double)bf16_bits_to_f32(w[j] & 0xffffu));
+          a4[u] += fabs((double)bf16_bits_to_f32(w[j] >> 16));
+        }
+      }
+    }
+    for (; i < nv; i += stride) {
+      const uint4 v = __ldcg(v8 + i);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a4[0] += fabs((double)bf16_bits_to_f32(w[j] & 0xffffu));
+        a4[0] += fabs((double)bf16_bits_to_f32(w[j] >> 16));
+      }
+    }
+    acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    const uint16_t* sv = reinterpret_cast<const uint16_t*>(W);
+    for (long long j = nv * 8 + t0; j < count; j += stride) acc += fabs((double)bf16_bits_to_f32(sv[j]));
+  } else {
+    const uint4* v4 = reinterpret_cast<const uint4*>(W);
+    const long long nv = count / 4;
+    double a4[4] = {0.0, 0.0, 0.0, 0.0};
+    long long i = t0;
+    for (; i + 3 * stride < nv; i += 4 * stride) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = __ldcg(v4 + i + u * stride);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        a4[u] += fabs((double)__uint_as_float(v[u].x));
+        a4[u] += fabs((double)__uint_as_float(v[u].y));
+        a4[u] += fabs((double)__uint_as_float(v[u].z));
+        a4[u] += fabs((double)__uint_as_float(v[u].w));
+      }
+    }
+    for (; i < nv; i += stride) {
+      const uint4 v = __ldcg(v4 + i);
+      a4[0] += fabs((double)__uint_as_float(v.x));
+      a4[0] += fabs((double)__uint_as_float(v.y));
+      a4[0] += fabs((double)__uint_as_float(v.z));
+      a4[0] += fabs((double)__uint_as_float(v.w));
+    }
+    acc = (a4[0] + a4[1]) + (a4[2] + a4[3]);
+    const float* sv = reinterpret_cast<const float*>(W);
+    for (long long j = nv * 4 + t0; j < count; j += stride) acc += fabs((double)sv[j]);
+  }
+  acc = block_sum_f64(acc, red);
+  if (threadIdx.x == 0) partials[blockIdx.x] = acc;
+  // exchange, then gamma from every partial in a fixed order (warp 0: lane l
+  // adds partials l, l + 32, ... in turn, then a fixed xor tree)
+  const bool ok = grid_exchange(flags, epoch, &xok);
+  if (threadIdx.x < 32) {
+    double v = 0.0;
+    for (int i = threadIdx.x; i < (int)gridDim.x; i += 32) v += __ldcg(partials + i);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) {
+      const float g = count > 0 ? (float)(v / (double)count) : 0.0f;
+      s_gamma = g;
+      if (blockIdx.x == 0 && ok) *gamma_out = g;
+    }
+  }
+  __syncthreads();
+  if (!ok) return;
+  // pass 2: codes, one thread per 32-bit word of the packed layout
+  const float g = s_gamma;
+  const float thr = ternary_threshold(g);
+  const int words_per_row = ldw / 4;
+  const long long total = (long long)N * words_per_row;
+  for (long long idx = t0; idx < total; idx += stride) {
+    const int n = (int)(idx / words_per_row);
+    const int wi = (int)(idx % words_per_row);
+    const int k0 = 16 * wi;
+    uint32_t word = 0x55555555u;                    // padding: code 1 everywhere
+    if (k0 < K) {
+      float w[16];
+      if (BF16) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            reinterpret_cast<const uint16_t*>(W) + (size_t)n * K + k0);
+        const uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 1);
         const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {

@@ -26,7 +26,13 @@ namespace bitnet {
 
 // PRE_GLU_RMSNORM: the row is m = relu(g)^2 * u of two fp32 inputs (gate
 // X, up X2), as the fused gate/up epilogue forms it, then RMSNorm.
-enum { PRE_NONE = 0, PRE_RMSNORM = 1, PRE_FWHT = 2, PRE_GLU_RMSNORM = 3 };
+// PRE_SILU_FWHT: the row is silu(x) of the loaded values, then the FWHT (the
+// H-BitLinear FFN's hidden activation: the first projection stores its plain
+// dequantised output and the second projection's quantiser applies the SiLU
+// as it loads it).
+enum { PRE_NONE = 0, PRE_RMSNORM = 1, PRE_FWHT = 2, PRE_GLU_RMSNORM = 3, PRE_SILU_FWHT = 4 };
+
+__host__ __device__ constexpr bool is_fwht(int pre) { return pre == PRE_FWHT || pre == PRE_SILU_FWHT; }
 
 struct QuantParams {
   const void* X;
@@ -129,7 +135,7 @@ __device__ __forceinline__ float prelude_value(float v, int k, float r, const fl
   if (PRE == PRE_RMSNORM) {
     float t = __fmul_rn(v, r);
     return gain ? __fmul_rn(t, __ldg(gain + k)) : t;
-  } else if (PRE == PRE_FWHT) {
+  } else if (is_fwht(PRE)) {
     return __fmul_rn(v, c);
   }
   return v;
@@ -160,6 +166,10 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
         f[2] = bf16_bits_to_f32(v.y & 0xffffu); f[3] = bf16_bits_to_f32(v.y >> 16);
         f[4] = bf16_bits_to_f32(v.z & 0xffffu); f[5] = bf16_bits_to_f32(v.z >> 16);
         f[6] = bf16_bits_to_f32(v.w & 0xffffu); f[7] = bf16_bits_to_f32(v.w >> 16);
+        if (PRE == PRE_SILU_FWHT) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = silu_f32(f[j]);
+        }
         reinterpret_cast<float4*>(row)[2 * i] = make_float4(f[0], f[1], f[2], f[3]);
         reinterpret_cast<float4*>(row)[2 * i + 1] = make_float4(f[4], f[5], f[6], f[7]);
         if (PRE == PRE_RMSNORM) {
@@ -172,6 +182,9 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
                                                           (size_t)m * K);
       for (int i = tid; i < K / 4; i += nt) {
         float4 v = src[i];
+        if (PRE == PRE_SILU_FWHT) {
+          v.x = silu_f32(v.x); v.y = silu_f32(v.y); v.z = silu_f32(v.z); v.w = silu_f32(v.w);
+        }
         reinterpret_cast<float4*>(row)[i] = v;
         if (PRE == PRE_RMSNORM) {
           ss += (double)v.x * (double)v.x;
@@ -190,7 +203,7 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
     } else {
       __syncthreads();
     }
-    if (PRE == PRE_FWHT) {
+    if (is_fwht(PRE)) {
       for (int h = 1; h < K; h <<= 1) {
         for (int b = tid; b < K / 2; b += nt) {
           const int j = (b / h) * 2 * h + (b % h);
@@ -504,7 +517,7 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
 // between lanes (shuffle with lane ^ (h / VEC); the lower partner keeps a + b,
 // the upper a - b, the same fp32 operations as the staged kernel), h >= 32 VEC
 // between a lane's own vectors.  No block barrier anywhere.
-template <int K, bool BF16>
+template <int K, bool BF16, bool SILU = false>
 __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
   constexpr int VEC = BF16 ? 8 : 4;
   constexpr int J = K / (32 * VEC);
@@ -538,6 +551,12 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
         v[j][0] = __uint_as_float(u.x); v[j][1] = __uint_as_float(u.y);
         v[j][2] = __uint_as_float(u.z); v[j][3] = __uint_as_float(u.w);
       }
+    }
+    if (SILU) {                    // PRE_SILU_FWHT: the row is silu of the loaded values
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) v[j][e] = silu_f32(v[j][e]);
     }
     // h < VEC: inside each vector
 #pragma unroll

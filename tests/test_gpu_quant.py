@@ -218,6 +218,31 @@ def test_pack_is_deterministic():
     np.testing.assert_array_equal(a[0], b[0])
 
 
+@pytest.mark.parametrize("fill", [0x00, 0xFF, "random"])
+def test_pack_one_launch_workspace_needs_no_initialisation(fill):
+    """The one-launch pack exchanges its partial sums through flags in the
+    workspace tagged with a fresh epoch per launch: whatever the workspace
+    holds before (zeros, ones, random bytes, a previous call's flags), the
+    result is the same, call after call."""
+    W = synthetic.weight(np.random.default_rng(21), 2560, 6912)
+    Wd = dev(W).to(torch.bfloat16)
+    Ww = Wd.float().cpu().numpy()
+    go = oracle.absmean(Ww)
+    want = oracle.pack(oracle.ternarize(Ww, go))
+    packed, gamma, ws = bn.alloc_packed(2560, 6912)
+    if fill == "random":
+        ws.copy_(torch.randint(0, 256, ws.shape, dtype=torch.uint8, device="cuda"))
+    else:
+        ws.fill_(fill)
+    for _ in range(3):
+        packed.fill_(0)
+        bn.bitnet_pack_weights(Wd, packed, gamma, ws)
+        torch.cuda.synchronize()
+        assert gamma.item() == go
+        np.testing.assert_array_equal(packed.cpu().numpy(), want)
+    assert bn.bitnet_check_device_error() == bn.BITNET_OK
+
+
 def test_quant_rmsnorm_zero_row_with_zero_eps():
     """mean square 0 and eps 0 give r = inf; the all-zero row must still come
     out as q = 0, s = 1 (the oracle's 0 * inf products never exceed 0)."""
