@@ -306,41 +306,15 @@ int launch_gemv(const LinearParams& p, cudaStream_t st) {
   return BITNET_OK;
 }
 
-// Schedule of the persistent GEMM: whole waves of full tiles, then the
-// remaining tiles (the last, partial wave) cut into `split` units of fewer
-// tokens each.  A unit costs about max(1 / split, kTailUnitFloor) of a full
-// tile (the weight tile is converted whole whatever the token count, and the
-// pipeline fill and epilogue do not shrink with it); the split minimises the
-// tail's rounds x unit cost, the smaller split on a tie.
-constexpr double kTailUnitFloor = 0.35;
-
-void tail_schedule(int num_tiles, int sms, int bn, int& full_units, int& split) {
-  full_units = (num_tiles / sms) * sms;
-  const int rest = num_tiles - full_units;
-  split = 1;
-  if (rest == 0) return;
-  double best = 1e30;
-  for (int f = 1; f <= 4; f *= 2) {
-    if (bn / f < kXBoxRows) break;
-    const int rounds = (rest * f + sms - 1) / sms;
-    const double cost = rounds * std::max(1.0 / f, kTailUnitFloor);
-    if (cost < best - 1e-9) {
-      best = cost;
-      split = f;
-    }
-  }
-}
-
 template <class C>
 int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1,
                   cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
-  CUtensorMap mx, mxs, mw0, mw1;
+  CUtensorMap mx, mw0, mw1;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 C::BN, CU_TENSOR_MAP_SWIZZLE_128B))
     return rc;
-  mxs = mx;
   // packed weight rows of BK/4 bytes, swizzled at that width (conflict-free
   // 16-byte loads in the converter)
   const CUtensorMapSwizzle wswz =
@@ -368,25 +342,32 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
     // the bf16 fragment epilogue (no GLU) stages 64-byte rows with the
     // 64-byte swizzle, so its transposing stores are bank-conflict free
     const bool frag = !C::GLU && lp.out_type == OUT_BF16;
+    // GLU: each epilogue warp stores 16 features x 32 tokens (fp32 m)
     if (int rc = tensor_map_2d(my, lp.Y, dt, (uint64_t)lp.N, (uint64_t)lp.M,
-                               (uint64_t)lp.N * esz, 32, 32,
+                               (uint64_t)lp.N * esz, C::GLU ? 16 : 32, 32,
                                frag ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_NONE))
+      return rc;
+  }
+  // bf16 residual of the fragment epilogue through TMA (the same box and
+  // swizzle as the output staging)
+  CUtensorMap mr = my;
+  const bool tma_res = tma_out && !C::GLU && lp.out_type == OUT_BF16 && lp.resid != nullptr &&
+                       (lp.flags & EPI_RESIDUAL);
+  if (tma_res) {
+    if (int rc = tensor_map_2d(mr, lp.resid, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (uint64_t)lp.N,
+                               (uint64_t)lp.M, (uint64_t)lp.N * 2, 32, 32,
+                               CU_TENSOR_MAP_SWIZZLE_64B))
       return rc;
   }
   TcParams p;
   p.tma_out = tma_out ? 1 : 0;
+  p.tma_res = tma_res ? 1 : 0;
   p.M = lp.M; p.N = lp.N; p.K = lp.K;
   p.num_kb = (lp.K + C::BK - 1) / C::BK;
   p.tiles_n = (lp.N + C::TILE_N - 1) / C::TILE_N;
   const int tiles_m = (lp.M + C::BN - 1) / C::BN;
   p.num_tiles = p.tiles_n * tiles_m;
-  tail_schedule(p.num_tiles, di.sms, C::BN, p.full_units, p.tail_split);
-  p.num_units = p.full_units + (p.num_tiles - p.full_units) * p.tail_split;
-  if (p.tail_split > 1) {        // 32-row boxes for the split tail units
-    if (int rc = tensor_map_2d_u8(mxs, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
-                                  kXBoxRows, CU_TENSOR_MAP_SWIZZLE_128B))
-      return rc;
-  }
+
   p.xs = lp.xs; p.xrs = lp.xrs; p.gamma0 = lp.gamma; p.gamma1 = gamma1;
   p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type; p.flags = lp.flags;
   // One CTA per SM: request enough shared memory that two never co-reside
@@ -397,8 +378,8 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   if (smem > (size_t)di.max_smem_optin) smem = di.max_smem_optin;
   auto kern = gemm_tc_kernel<C>;
   BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int grid = p.num_units < di.sms ? p.num_units : di.sms;
-  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mxs, mw0, mw1, my, p);
+  const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
+  return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mw0, mw1, my, mr, p);
 }
 
 // Devices whose context has the decode kernel's shared-memory attribute set
@@ -537,8 +518,8 @@ int launch_gemv_mma_rt(const LinearParams& p, cudaStream_t st, const DeviceInfo&
   gp.lp = p;
   gp.lp.flags &= ~LAUNCH_PDL;                  // keeps LAUNCH_PDL_INPUTS for the kernel
   gp.rows_per_cta = 16 * RT;
-  gp.sw = p.ldw + kGmRowPad;
-  gp.sx = p.K + kGmRowPad;
+  gp.sw = p.ldw;
+  gp.sx = p.K;
   gp.off_x = (int)align128((size_t)16 * RT * gp.sw);
   const size_t smem = (size_t)gp.off_x + (size_t)p.M * gp.sx + 128;
   if (smem > (size_t)di.max_smem_optin - 4096) return BITNET_ERR_UNSUPPORTED;
@@ -636,14 +617,12 @@ int launch_ffn_decode(FfnDecodeParams p, cudaStream_t st, bool tail = false) {
   p.nr_per = (p.H + G - 1) / G;
   if (p.nr_per > 32) return BITNET_ERR_UNSUPPORTED;
   p.mpad = p.M <= 8 ? 8 : 16;
-  p.sw_h = p.ldwH + kFdRowPad;
-  p.sw_i = p.ldwI + kFdRowPad;
   p.sx_h = p.H + kFdRowPad;
   p.sx_i = p.I + kFdRowPad;
   p.off_gu = 0;
-  p.off_d = (int)align128((size_t)p.groups * 16 * p.sw_h);
-  p.off_o = (int)align128((size_t)p.off_d + (size_t)p.nr_per * p.sw_i);
-  p.off_act = (int)align128((size_t)p.off_o + (tail ? (size_t)p.nr_per * p.sw_h : 0));
+  p.off_d = (int)align128((size_t)2 * p.nf_per * p.ldwH);
+  p.off_o = (int)align128((size_t)p.off_d + (size_t)p.nr_per * p.ldwI);
+  p.off_act = (int)align128((size_t)p.off_o + (tail ? (size_t)p.nr_per * p.ldwH : 0));
   const size_t smem =
       (size_t)p.off_act + (size_t)p.mpad * (size_t)std::max(p.sx_h, p.sx_i) + 128;
   if (smem + sizeof(FfnDecodeShared) + 1024 > (size_t)di.max_smem_optin) return BITNET_ERR_UNSUPPORTED;

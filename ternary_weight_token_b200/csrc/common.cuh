@@ -262,6 +262,17 @@ __device__ __forceinline__ void stmatrix_x4_trans(uint32_t addr, uint32_t r0, ui
                : "memory");
 }
 
+// Inverse of stmatrix_x4_trans: four 8x8 matrices of 16-bit values loaded
+// transposed; thread 8i + r gives the address of row r of matrix i, and
+// register i of thread t receives elements (t/4, 2(t%4) + {0, 1}) of matrix i.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t& r0, uint32_t& r1,
+                                                  uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr)
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -309,15 +320,16 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 // waits until every CTA's flag holds the epoch.  Epochs are never reused (the
 // host draws a fresh one per launch from a counter started at a random
 // value), so the flags need no reset and no zeroing.  Every thread of the CTA
-// calls it; warp 0 polls, bounded by kWaitLimitNs.  Returns false (device
-// error recorded) if the wait gave up.
+// calls it; warp 0 polls (relaxed loads, then an acquire fence once every
+// flag matched), bounded by kWaitLimitNs.  Returns false (device error
+// recorded) if the wait gave up.
 __device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
   asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
   unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
 }
 
@@ -330,23 +342,23 @@ __device__ __forceinline__ bool grid_exchange(unsigned long long* flags, unsigne
     *ok_smem = 1;
   }
   if (threadIdx.x < 32) {
+    // every flag of a lane is loaded before any is compared (independent
+    // relaxed loads in flight together), then one acquire fence
     const int lane = threadIdx.x;
     const unsigned long long t0 = global_timer_ns();
     bool done = false;
     for (uint32_t it = 0;; ++it) {
-      bool mine = true;
-      for (int i = lane; i < (int)gridDim.x; i += 32)
-        mine = mine && (ld_acquire_u64(flags + i) == epoch);
-      done = __all_sync(0xffffffffu, mine);
+      int missing = 0;
+      for (int i = lane; i < (int)gridDim.x; i += 32) missing += ld_relaxed_u64(flags + i) != epoch;
+      done = __all_sync(0xffffffffu, missing == 0);
       if (done) break;
       if ((it & 7u) == 7u && global_timer_ns() - t0 > kWaitLimitNs) break;
-      __nanosleep(64);
     }
     if (!done && lane == 0) {
       record_device_error(DEV_ERR_TIMEOUT);
       *ok_smem = 0;
     }
-    __threadfence();
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
   }
   __syncthreads();
   return *ok_smem != 0;

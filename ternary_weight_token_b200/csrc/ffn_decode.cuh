@@ -14,11 +14,11 @@
 // arithmetic; run as four launches it pays four grid ramps and completions.
 // Here one cooperative grid (one CTA per SM) does it with a single grid-wide
 // exchange:
-//   P0  warp 0 of every CTA bulk-copies its weight rows into shared memory
-//       at once: 8-feature groups of gate rows and the matching up rows, and
-//       its slice of down rows (one copy per row, spread over the 32 lanes;
-//       rows padded by 16 bytes so the fragment loads below are bank-conflict
-//       free);
+//   P0  thread 0 of every CTA bulk-copies its weight rows into shared memory
+//       at once, one copy per block of contiguous rows: its gate rows, the
+//       matching up rows and its slice of down rows (the fragment loads of 8
+//       rows of one 16-byte-multiple stride share banks; a copy per padded
+//       row was measured far slower, the copy engine taking ~0.1 us a copy);
 //   P1  every CTA quantises all tokens of x itself (RMSNorm prelude; a row is
 //       spread over several warps, its loads all in flight): x is a few KB,
 //       so the redundant work costs less than an exchange;
@@ -90,7 +90,7 @@ struct FfnDecodeParams {
   int mpad;                    // tokens rounded up to 8
   // shared-memory carve-up (bytes from the 128-aligned base)
   int off_gu, off_d, off_act;
-  int sw_h, sw_i, sx_h, sx_i;  // row strides: weights (ldw + 16), activations (K + 16)
+  int sx_h, sx_i;              // staged code row strides (K + 16: conflict-free fragments)
 };
 
 struct FfnDecodeShared {
@@ -378,9 +378,10 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   __shared__ FfnDecodeShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(fd_smem_raw) + 127) & ~uintptr_t(127));
-  uint8_t* s_gu = smem + p.off_gu;          // [groups][16 rows][sw_h]
-  uint8_t* s_d = smem + p.off_d;            // [nr][sw_i]
-  uint8_t* s_o = smem + p.off_o;            // [nr][sw_h] (TAIL)
+  uint8_t* s_g = smem + p.off_gu;           // [nf_per][ldwH] gate rows
+  uint8_t* s_u = s_g + (size_t)p.nf_per * p.ldwH;   // [nf_per][ldwH] up rows
+  uint8_t* s_d = smem + p.off_d;            // [nr][ldwI]
+  uint8_t* s_o = smem + p.off_o;            // [nr][ldwH] (TAIL)
   int8_t* s_act = reinterpret_cast<int8_t*>(smem + p.off_act);   // [mpad][sx_h or sx_i]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -404,29 +405,22 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     sh.ok = 1;
   }
   __syncthreads();
-  // the 32 lanes of warp 0 issue the copies between them (lane 0 first sets
-  // each barrier's expected bytes, so no phase can complete early)
-  if (warp == 0) {
-    if (lane == 0) {
-      if (TAIL) mbar_arrive_expect_tx(&sh.bar_o, (uint32_t)(nr * p.ldwH));
-      mbar_arrive_expect_tx(&sh.bar_gu, (uint32_t)(2 * nf * p.ldwH));
-      mbar_arrive_expect_tx(&sh.bar_d, (uint32_t)(nr * p.ldwI));
-    }
-    __syncwarp();
+  // one bulk copy per block of contiguous rows (many small copies keep the
+  // copy engine busy for longer than the bytes take)
+  if (threadIdx.x == 0) {
     if (TAIL) {                                       // needed first
-      for (int r = lane; r < nr; r += 32)
-        bulk_copy_g2s(s_o + (size_t)r * p.sw_h, p.Wo + (size_t)(n0 + r) * p.ldwH,
-                      (uint32_t)p.ldwH, &sh.bar_o);
+      mbar_arrive_expect_tx(&sh.bar_o, (uint32_t)(nr * p.ldwH));
+      if (nr > 0)
+        bulk_copy_g2s(s_o, p.Wo + (size_t)n0 * p.ldwH, (uint32_t)(nr * p.ldwH), &sh.bar_o);
     }
-    for (int f = lane; f < nf; f += 32) {
-      uint8_t* row = s_gu + (size_t)((f >> 3) * 16 + (f & 7)) * p.sw_h;
-      bulk_copy_g2s(row, p.Wg + (size_t)(f0 + f) * p.ldwH, (uint32_t)p.ldwH, &sh.bar_gu);
-      bulk_copy_g2s(row + 8 * p.sw_h, p.Wu + (size_t)(f0 + f) * p.ldwH, (uint32_t)p.ldwH,
-                    &sh.bar_gu);
+    mbar_arrive_expect_tx(&sh.bar_gu, (uint32_t)(2 * nf * p.ldwH));
+    if (nf > 0) {
+      bulk_copy_g2s(s_g, p.Wg + (size_t)f0 * p.ldwH, (uint32_t)(nf * p.ldwH), &sh.bar_gu);
+      bulk_copy_g2s(s_u, p.Wu + (size_t)f0 * p.ldwH, (uint32_t)(nf * p.ldwH), &sh.bar_gu);
     }
-    for (int r = lane; r < nr; r += 32)
-      bulk_copy_g2s(s_d + (size_t)r * p.sw_i, p.Wd + (size_t)(n0 + r) * p.ldwI, (uint32_t)p.ldwI,
-                    &sh.bar_d);
+    mbar_arrive_expect_tx(&sh.bar_d, (uint32_t)(nr * p.ldwI));
+    if (nr > 0)
+      bulk_copy_g2s(s_d, p.Wd + (size_t)n0 * p.ldwI, (uint32_t)(nr * p.ldwI), &sh.bar_d);
   }
 
   // ---- TAIL: h = x + o_proj(attn_sub_norm(A)) for this CTA's rows, then
@@ -441,7 +435,7 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     if (threadIdx.x < M) dequant_factor(__ldg(p.gamma_o), sh.s_x[threadIdx.x],
                                         sh.fo_hi[threadIdx.x], sh.fo_lo[threadIdx.x]);
     if (!mbar_wait(&sh.bar_o, 0, nullptr) && lane == 0) sh.ok = 0;
-    fd_contract_rows(s_o, p.sw_h, nr, s_act, p.sx_h, p.H, ntile, sh.red);
+    fd_contract_rows(s_o, p.ldwH, nr, s_act, p.sx_h, p.H, ntile, sh.red);
     __syncthreads();
     if (threadIdx.x < 2 * 2 * 32) {
       const int idx = threadIdx.x;
@@ -495,6 +489,7 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   {
     const bool landed = mbar_wait(&sh.bar_gu, 0, nullptr);
     if (!landed && lane == 0) sh.ok = 0;
+    const int flast = nf > 0 ? nf - 1 : 0;
     const int steps = p.H / 32;
     const int s_lo = warp * steps / 8, s_hi = (warp + 1) * steps / 8;
     int acc[kFdMaxGroups][2][4];
@@ -517,9 +512,11 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
 #pragma unroll
       for (int j = 0; j < kFdMaxGroups; ++j) {
         if (j < p.groups) {
-          const uint8_t* r0 = s_gu + (size_t)(j * 16 + g8) * p.sw_h + 8 * s;
-          const uint2 lo = *reinterpret_cast<const uint2*>(r0);              // gate row
-          const uint2 hi = *reinterpret_cast<const uint2*>(r0 + 8 * p.sw_h);  // up row
+          // fragment rows g8 (gate) and 8 + g8 (up) of feature 8 j + g8;
+          // features past nf read a valid row (results discarded)
+          const size_t off = (size_t)min(8 * j + g8, flast) * p.ldwH + 8 * s;
+          const uint2 lo = *reinterpret_cast<const uint2*>(s_g + off);       // gate row
+          const uint2 hi = *reinterpret_cast<const uint2*>(s_u + off);       // up row
           const uint32_t a0 = (lo.x >> (2 * c4)) & 0x03030303u;
           const uint32_t a2 = (lo.y >> (2 * c4)) & 0x03030303u;
           const uint32_t a1 = (hi.x >> (2 * c4)) & 0x03030303u;
@@ -616,7 +613,7 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
 
   // ---- P5: down rows of this CTA (warps split K), residual, store
   if (!mbar_wait(&sh.bar_d, 0, nullptr) && lane == 0) sh.ok = 0;
-  fd_contract_rows(s_d, p.sw_i, nr, s_act, p.sx_i, p.I, ntile, sh.red);
+  fd_contract_rows(s_d, p.ldwI, nr, s_act, p.sx_i, p.I, ntile, sh.red);
   __syncthreads();
   if (threadIdx.x < 2 * 2 * 32) {
     // thread (row tile i, token tile t, lane): rows 16 i + g and 16 i + 8 + g,

@@ -31,7 +31,11 @@
 //   warps 4..     converters (CONV_GROUPS groups of 4 warps alternate stages)
 //   last 4 warps  epilogue: tcgen05.ld -> dequant -> fused op -> a 32 x 32
 //                 tile staged in shared memory and written by a TMA store
-//                 (plain stores when the output rows are not 16-byte multiples)
+//                 (plain stores when the output rows are not 16-byte multiples);
+//                 bf16 outputs take the residual through a TMA load of the
+//                 same 32 x 32 tile; GLU: each warp's TMEM quarter holds the
+//                 gate rows and the up rows of the same 16 features (placed so
+//                 by the converters), so m = relu(g)^2 * u forms in-thread
 // Every wait is bounded; a wait that gives up records a device error, raises a
 // CTA-wide abort flag, and the CTA drains its tensor-core work and bulk
 // copies, frees tensor memory and exits.
@@ -73,7 +77,7 @@ struct TcConfig {
   static constexpr int OFF_W = OFF_X + STAGES * X_STAGE;
   static constexpr int OFF_OUT = OFF_W + STAGES * NW * W_STAGE;  // 4 warps x 2 buffers
   static constexpr int OFF_BAR = OFF_OUT + 4 * 2 * STAGE_OUT_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 11;
+  static constexpr int NUM_BARS = 3 * STAGES + 7 + 8;    // + residual chunks (4 warps x 2)
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-B alignment
@@ -84,12 +88,6 @@ struct TcParams {
   int M, N, K;
   int num_kb;                 // k stages = ceil(K / BK)
   int tiles_n, num_tiles;
-  // Work units: tiles [0, full_units) are whole BN-token tiles (the full
-  // waves); each tile after them (the last, partial wave) is cut into
-  // tail_split units of BN / tail_split tokens, so the last wave's work is
-  // spread over more SMs.  num_units = full_units + (num_tiles - full_units)
-  // * tail_split.
-  int num_units, full_units, tail_split;
   const float* xs;            // [M] activation scales
   const int32_t* xrs;         // [M] sum of activation codes
   const float* gamma0;        // weight scale (gate weights for GLU)
@@ -99,41 +97,18 @@ struct TcParams {
   int out_type;
   int flags;
   int tma_out;                // 1: output written through the TMA map tm_y
+  int tma_res;                // 1: bf16 residual read through the TMA map tm_r
 };
 
 __device__ __forceinline__ int out_elem_bytes(int out_type) { return out_type == OUT_BF16 ? 2 : 4; }
 
-// Activation rows per TMA box of a tail unit: a unit of bn < BN tokens is
-// loaded as bn / 32 boxes (a second tensor map), each landing on a 1024-byte
-// boundary of the 128-byte-swizzled sub-tile; whole tiles load one box of BN
-// rows per 128-k sub-tile.
-constexpr int kXBoxRows = 32;
-
-// One work unit: weight tile tn, tokens [m0, m0 + bn).
-struct TcUnit {
-  int tn, m0, bn;
-};
-
-template <class C>
-__device__ __forceinline__ TcUnit tc_unit(const TcParams& p, int u) {
-  int tile = u, sub = 0, split = 1;
-  if (u >= p.full_units) {
-    const int v = u - p.full_units;
-    split = p.tail_split;
-    tile = p.full_units + v / split;
-    sub = v - (v / split) * split;
-  }
-  const int bn = C::BN / split;
-  return TcUnit{tile % p.tiles_n, (tile / p.tiles_n) * C::BN + sub * bn, bn};
-}
-
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tm_x,
-                   const __grid_constant__ CUtensorMap tm_xs,
                    const __grid_constant__ CUtensorMap tm_w0,
                    const __grid_constant__ CUtensorMap tm_w1,
-                   const __grid_constant__ CUtensorMap tm_y, TcParams p) {
+                   const __grid_constant__ CUtensorMap tm_y,
+                   const __grid_constant__ CUtensorMap tm_r, TcParams p) {
   extern __shared__ uint8_t tc_smem_raw[];
   // per-token dequant factors (fp32 head, tail) and code sums of a tile,
   // computed once by the four epilogue warps; two buffers alternate between
@@ -153,8 +128,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   uint64_t* accempty = accfull + 2;            // accumulator drained    (4 epilogue warps)
   uint64_t* drain = accempty + 2;              // teardown drain
   uint64_t* tokbar = drain + 1;                // tile's token factors written (4 warps)
-  uint64_t* upready = tokbar + 2;              // GLU: up values of a chunk staged (2 warps)
-  uint64_t* upfree = upready + 2;              // GLU: staged up values consumed (2 warps)
+  uint64_t* rbar = tokbar + 2;                 // [warp q][buffer] residual chunk landed (TMA)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
@@ -173,19 +147,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(drain, 2);
     mbar_init(&tokbar[0], 4);
     mbar_init(&tokbar[1], 4);
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&upready[b], 2);
-      mbar_init(&upfree[b], 2);
-    }
+    for (int b = 0; b < 8; ++b) mbar_init(&rbar[b], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_x);
-    if (p.tail_split > 1) tma_prefetch_desc(&tm_xs);
     tma_prefetch_desc(&tm_w0);
     if (C::GLU) tma_prefetch_desc(&tm_w1);
     if (p.tma_out) tma_prefetch_desc(&tm_y);
+    if (p.tma_res) tma_prefetch_desc(&tm_r);
   }
   if (warp == 2) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
@@ -205,25 +176,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
-      for (int u = blockIdx.x; u < p.num_units; u += gridDim.x) {
-        const TcUnit t = tc_unit<C>(p, u);
-        const int tn = t.tn;
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
+        const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) goto producer_done;
-          mbar_arrive_expect_tx(&full[st], (uint32_t)(t.bn * C::BK + C::NW * C::W_STAGE));
-          if (t.bn == C::BN) {                // a whole tile: one box per 128-k sub-tile
+          mbar_arrive_expect_tx(&full[st], C::TX_BYTES);
 #pragma unroll
-            for (int xs = 0; xs < C::BK / 128; ++xs)
-              tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
-                          kb * C::BK + 128 * xs, t.m0);
-          } else {                            // a tail unit: bn / 32 boxes of 32 rows
-#pragma unroll
-            for (int xs = 0; xs < C::BK / 128; ++xs)
-              for (int r = 0; r < t.bn; r += kXBoxRows)
-                tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB + r * 128, &tm_xs, &full[st],
-                            kb * C::BK + 128 * xs, t.m0 + r);
-          }
+          for (int xs = 0; xs < C::BK / 128; ++xs)
+            tma_load_2d(sx + st * C::X_STAGE + xs * C::XSUB, &tm_x, &full[st],
+                        kb * C::BK + 128 * xs, tm * C::BN);
           if (C::GLU) {                       // rows 0-63 gate, 64-127 up
             tma_load_2d(sw + st * C::W_STAGE, &tm_w0, &full[st], kb * (C::BK / 4),
                         tn * C::TILE_N);
@@ -250,9 +212,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // accumulator buffer after reading it, before handing it back.
     if (lane == 0) {
       const uint32_t me = warp == 1 ? 0u : 1u;
+      const uint32_t idesc = make_idesc_i8(C::BM, C::BN);
       uint32_t it = 0, tcount = 0;
-      for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++tcount) {
-        const uint32_t idesc = make_idesc_i8(C::BM, tc_unit<C>(p, u).bn);
+      for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
         const uint32_t ab = tcount & 1u, use = tcount >> 1;
         if (!mbar_wait(&accempty[ab], use & 1u, abort_flag)) break;
         tc_fence_after();
@@ -284,9 +246,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------- converters
     const uint32_t group = (uint32_t)(warp - 4) >> 2;   // stages with it % groups == group
     const int q = warp & 3;
-    const int row = 32 * q + lane;               // weight row within the tile = TMEM lane
+    // TMEM lane 32 q + lane holds weight row `row` of the stage: the row
+    // itself, or for GLU the gate row 16 q + lane (lane < 16) and the up row
+    // 64 + 16 q + lane - 16, so each epilogue warp's quarter holds the gate
+    // and up rows of the same 16 features
+    const int row = C::GLU ? (lane < 16 ? 16 * q + lane : 48 + 16 * q + lane) : 32 * q + lane;
     const uint32_t lane_base = tbase + ((uint32_t)(32 * q) << 16) + a_col0;
-    const uint32_t total = (uint32_t)((p.num_units - (int)blockIdx.x + (int)gridDim.x - 1) /
+    const uint32_t total = (uint32_t)((p.num_tiles - (int)blockIdx.x + (int)gridDim.x - 1) /
                                       (int)gridDim.x) * (uint32_t)p.num_kb;
     for (uint32_t it = group; it < total; it += C::CONV_GROUPS) {
       const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
@@ -341,20 +307,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_arrive(&accempty[0]);
       mbar_arrive(&accempty[1]);
     }
-    uint32_t tcount = 0, chunk_count = 0, xcount = 0;
-    for (int u = blockIdx.x; u < p.num_units; u += gridDim.x, ++tcount) {
-      const TcUnit unit = tc_unit<C>(p, u);
-      const int tn = unit.tn;
-      const int m0 = unit.m0;
+    uint32_t tcount = 0, chunk_count = 0;
+    uint32_t rphase = 0;                         // bit b: parity of this warp's rbar[b]
+    // bf16 residual of a 32 x 32 output chunk: one TMA load into the upper
+    // half of the chunk's staging buffer (64-byte swizzled like the output
+    // staging), issued a chunk ahead, read back with ldmatrix.trans
+    const bool res_tma = frag_path && p.tma_res && (p.flags & EPI_RESIDUAL);
+    auto res_load = [&](uint32_t cc, int nq, int mrow) {
+      const uint32_t b = cc & 1u;
+      const uint32_t dst = out_base + b * C::STAGE_OUT_BYTES + 2048u;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&rbar[2 * q + b], 2048u);
+        tma_load_2d(smem + (dst - smem_u32(smem)), &tm_r, &rbar[2 * q + b], nq, mrow);
+      }
+    };
+    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
+      const int m0 = tm * C::BN;
       // first output feature of this warp (GLU: warps 0-1 hold gate rows,
       // warps 2-3 the up rows of the same features)
       const int nq0 = tn * C::TILE_N + 32 * (C::GLU ? (q & 1) : q);
+      if (res_tma && nq0 < p.N && m0 < p.M) res_load(chunk_count, nq0, m0);
       const uint32_t ab = tcount & 1u, aph = (tcount >> 1) & 1u;
       float2* tok_f = s_tok_f[ab];               // [NW][BN]
       int* tok_rs = s_tok_rs[ab];
       // This buffer was last read for tile tcount - 2; every warp has since
       // arrived on the other buffer's barrier, so no warp still reads it.
-      for (int j = 32 * q + lane; j < unit.bn; j += 128) {
+      for (int j = 32 * q + lane; j < C::BN; j += 128) {
         const int m = m0 + j;
         float2 f0 = make_float2(0.0f, 0.0f), f1 = make_float2(0.0f, 0.0f);
         int rs = 0;
@@ -376,7 +355,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       const int n = nq0 + lane;
       const bool n_ok = n < p.N;
 #pragma unroll 1
-      for (int c = 0; c < unit.bn / 32; ++c, ++chunk_count) {
+      for (int c = 0; c < C::BN / 32; ++c, ++chunk_count) {
         const int mc = m0 + 32 * c;              // first token of this chunk
         if (mc >= p.M) {                         // past the last token: only re-zero
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
@@ -390,9 +369,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             tmem_ld_16x256b_x4(lane_base + ab * C::ACC_COLS + 32u * c, v);
             tmem_ld_16x256b_x4(lane_base + (16u << 16) + ab * C::ACC_COLS + 32u * c, v + 16);
             const int tq = 2 * (lane & 3);       // this thread's even token offset
+            // the next chunk's residual goes in flight before this one is used
+            if (res_tma && c + 1 < C::BN / 32 && mc + 32 < p.M && nq0 < p.N)
+              res_load(chunk_count + 1, nq0, mc + 32);
             // residual (bf16) of the same elements, two per register
             uint32_t rpk[16];
-            if (p.flags & EPI_RESIDUAL) {
+            if ((p.flags & EPI_RESIDUAL) && !res_tma) {
               const uint16_t* rp = reinterpret_cast<const uint16_t*>(p.resid);
 #pragma unroll
               for (int i = 0; i < 32; i += 2) {
@@ -412,6 +394,22 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             if (lane == 0) bulk_wait_group_read<1>();
             __syncwarp();
             const int mi = lane >> 3, rr8 = lane & 7;
+            if (res_tma && nq0 < p.N) {
+              const uint32_t b = chunk_count & 1u;
+              if (!mbar_wait(&rbar[2 * q + b], (rphase >> b) & 1u, abort_flag)) break;
+              rphase ^= 1u << b;
+              const uint32_t rb = buf + 2048u;
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int jp = 0; jp < 2; ++jp) {
+                  const int row = 8 * (2 * jp + (mi >> 1)) + rr8;
+                  const int chunk = (2 * h + (mi & 1)) ^ ((row >> 1) & 3);
+                  ldmatrix_x4_trans(rb + (uint32_t)(row * 64 + chunk * 16), rpk[8 * h + 4 * jp + 0],
+                                    rpk[8 * h + 4 * jp + 1], rpk[8 * h + 4 * jp + 2],
+                                    rpk[8 * h + 4 * jp + 3]);
+                }
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {        // weight rows nq0 + 16h .. + 15
               uint32_t pk[8];                    // bf16x2 of matrix (j, s): pk[2j + s]
@@ -430,8 +428,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     y1 = silu_f32(y1);
                   }
                   if (p.flags & EPI_RESIDUAL) {
-                    y0 = __fadd_rn(__uint_as_float(rpk[i >> 1] << 16), y0);
-                    y1 = __fadd_rn(__uint_as_float(rpk[i >> 1] & 0xffff0000u), y1);
+                    // TMA path: residual pair of matrix (j, s2) of half h
+                    const uint32_t rr2 = res_tma ? rpk[8 * h + 2 * j + s2] : rpk[i >> 1];
+                    y0 = __fadd_rn(__uint_as_float(rr2 << 16), y0);
+                    y1 = __fadd_rn(__uint_as_float(rr2 & 0xffff0000u), y1);
                   }
                   const __nv_bfloat162 b2 = __floats2bfloat162_rn(y0, y1);
                   pk[2 * j + s2] = *reinterpret_cast<const uint32_t*>(&b2);
@@ -456,45 +456,66 @@ __global__ void __launch_bounds__(C::THREADS, 1)
             continue;
           }
         }
+        if constexpr (C::GLU) {
+          // lanes 32 q .. + 15 hold gate rows, 32 q + 16 .. + 31 the up rows
+          // of the same 16 features: v[4j + k] (gate) and v[16 + 4j + k] (up)
+          // are feature fq0 + 8 (k / 2) + lane / 4, token mc + 8 j +
+          // 2 (lane % 4) + k % 2, so m = relu(g)^2 * u forms in the thread
+          uint32_t v[32];
+          tmem_ld_16x256b_x4(lane_base + ab * C::ACC_COLS + 32u * c, v);
+          tmem_ld_16x256b_x4(lane_base + (16u << 16) + ab * C::ACC_COLS + 32u * c, v + 16);
+          tmem_ld_wait();
+          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
+          const int tq = 2 * (lane & 3);
+          const int fq0 = tn * C::TILE_N + 16 * q;   // first feature of this warp
+          float mv[16];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int t = 32 * c + 8 * j + tq;
+            const float4 fg = *reinterpret_cast<const float4*>(&tok_f[t]);
+            const float4 fu = *reinterpret_cast<const float4*>(&tok_f[C::BN + t]);
+            const int2 rr = *reinterpret_cast<const int2*>(&tok_rs[t]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = 4 * j + k;
+              const bool odd = (k & 1) != 0;
+              const int rs = odd ? rr.y : rr.x;
+              const float g = dequant_dw((int)v[i] - rs, odd ? fg.z : fg.x, odd ? fg.w : fg.y);
+              const float u = dequant_dw((int)v[16 + i] - rs, odd ? fu.z : fu.x, odd ? fu.w : fu.y);
+              mv[i] = __fmul_rn(g > 0.0f ? __fmul_rn(g, g) : 0.0f, u);
+            }
+          }
+          if (p.tma_out) {
+            // 32 tokens x 16 features fp32 staged as 64-byte token rows
+            const uint32_t buf = out_base + (chunk_count & 1u) * C::STAGE_OUT_BYTES;
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int trel = 8 * (i >> 2) + tq + (i & 1);
+              const int frel = 8 * ((i >> 1) & 1) + (lane >> 2);
+              st_shared_u32(buf + (uint32_t)(trel * 64 + frel * 4), __float_as_uint(mv[i]));
+            }
+            fence_proxy_async_shared();
+            __syncwarp();
+            if (lane == 0 && fq0 < p.N) {
+              tma_store_2d(&tm_y, smem + (buf - smem_u32(smem)), fq0, mc);
+              bulk_commit_group();
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int m = mc + 8 * (i >> 2) + tq + (i & 1);
+              const int n = fq0 + 8 * ((i >> 1) & 1) + (lane >> 2);
+              if (m < p.M && n < p.N) reinterpret_cast<float*>(p.Y)[(size_t)m * p.N + n] = mv[i];
+            }
+          }
+          continue;
+        }
         uint32_t v[32];
         float y[32];
         tmem_ld_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c, v);
-        if (C::GLU) {
-          // up warps dequantise their rows and stage them token-major in the
-          // exchange buffer (the up warps' own output staging area); gate
-          // warps combine relu(g)^2 * u and store
-          tmem_ld_wait();
-          tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
-          const uint32_t xb = (uint32_t)(xcount & 1u), xuse = xcount >> 1;
-          ++xcount;
-          float* xbuf = reinterpret_cast<float*>(smem + C::OFF_OUT + 2 * 2 * C::STAGE_OUT_BYTES +
-                                                 xb * (C::BM / 2) * 32 * 4);
-          const int xrow = 32 * (q & 1) + lane;   // feature within the tile
-          if (q >= 2) {
-            if (!mbar_wait(&upfree[xb], (xuse & 1u) ^ 1u, abort_flag)) break;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const int t = 32 * c + j;
-              const float2 fb = tok_f[C::BN + t];
-              xbuf[j * (C::BM / 2) + xrow] = dequant_dw((int)v[j] - tok_rs[t], fb.x, fb.y);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&upready[xb]);
-            continue;                            // up warps store nothing
-          }
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int t = 32 * c + j;
-            const float2 fa = tok_f[t];
-            const float g = dequant_dw((int)v[j] - tok_rs[t], fa.x, fa.y);
-            y[j] = g > 0.0f ? __fmul_rn(g, g) : 0.0f;
-          }
-          if (!mbar_wait(&upready[xb], xuse & 1u, abort_flag)) break;
-#pragma unroll
-          for (int j = 0; j < 32; ++j) y[j] = __fmul_rn(y[j], xbuf[j * (C::BM / 2) + xrow]);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&upfree[xb]);
-        } else {
+        {
           tmem_ld_wait();
           tmem_zero_32x32b_x32(lane_base + ab * C::ACC_COLS + 32u * c);
           if (p.out_type == OUT_I32) {

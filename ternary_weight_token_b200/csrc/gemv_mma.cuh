@@ -10,10 +10,11 @@
 //
 // One CTA per 16 * RT weight rows (the rows of the call's projections,
 // concatenated), every input of those rows:
-//   - the lanes of warp 0 issue one bulk copy per weight row into shared
-//     memory (rows padded by 16 bytes: the fragment loads below hit distinct
-//     banks) and, once the preceding grid has completed (or at once when the
-//     caller states it writes none of the inputs), one per activation row;
+//   - thread 0 issues one bulk copy per run of contiguous weight rows into
+//     shared memory and, once the preceding grid has completed (or at once
+//     when the caller states it writes none of the inputs), one for all the
+//     activation rows (dense rows: the fragment loads of 8 rows share banks,
+//     which costs less than the copy engine's time per extra copy);
 //   - the 8 warps split the K steps of 32; each thread takes its A fragment
 //     words straight from the packed rows (two 16-weight words per step, its
 //     4-weight group picked by a shift and mask) and its B fragment words
@@ -32,7 +33,6 @@
 namespace bitnet {
 
 constexpr int kGmThreads = 256;
-constexpr int kGmRowPad = 16;
 
 struct GmParams {
   LinearParams lp;
@@ -85,25 +85,22 @@ __global__ void __launch_bounds__(kGmThreads) gemv_mma_kernel(GmParams gp) {
   }
   for (int i = threadIdx.x; i < RT * NTILE * 32 * 4; i += kGmThreads) red[i] = 0;
   __syncthreads();                                       // barriers initialised, red zeroed
-  if (warp == 0) {
-    // the 32 lanes issue the row copies between them; lane 0 first sets the
-    // expected bytes, so no phase can complete before every copy is counted
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&bar_w, (uint32_t)(nrows * p.ldw));
-      mbar_arrive_expect_tx(&bar_x, (uint32_t)(p.M * p.K));
-    }
-    __syncwarp();
-    // weight rows: the preceding work does not write them (LAUNCH_PDL)
-    for (int r = lane; r < nrows; r += 32) {
+  if (threadIdx.x == 0) {
+    // one bulk copy per run of rows within one projection (a CTA's rows span
+    // at most the end of one projection and the start of the next): the
+    // preceding work does not write the weights (LAUNCH_PDL)
+    mbar_arrive_expect_tx(&bar_w, (uint32_t)(nrows * p.ldw));
+    for (int r = 0; r < nrows;) {
       int nl;
       const int sg = segment_of(p, row0 + r, nl);
-      gm_bulk_g2s(s_w + (size_t)r * gp.sw, p.seg_W[sg] + (size_t)nl * p.ldw, (uint32_t)p.ldw,
-                  &bar_w);
+      const int run = min(nrows - r, p.seg_row0[sg + 1] - (row0 + r));
+      gm_bulk_g2s(s_w + (size_t)r * gp.sw, p.seg_W[sg] + (size_t)nl * p.ldw,
+                  (uint32_t)(run * p.ldw), &bar_w);
+      r += run;
     }
     if (!inputs_ready) grid_dependency_wait();
-    for (int m = lane; m < p.M; m += 32)
-      gm_bulk_g2s(smem + gp.off_x + (size_t)m * gp.sx, p.Xq + (size_t)m * p.K, (uint32_t)p.K,
-                  &bar_x);
+    mbar_arrive_expect_tx(&bar_x, (uint32_t)(p.M * p.K));
+    gm_bulk_g2s(smem + gp.off_x, p.Xq, (uint32_t)(p.M * p.K), &bar_x);   // all M rows at once
   }
 
   // per-token scale and code sum, read while the copies are in flight
