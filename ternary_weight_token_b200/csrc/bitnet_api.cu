@@ -240,29 +240,39 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
     if (k4 <= 128 * 14) return launch_quant_rows<128, 14>(p, bf16, prelude, st);
     return launch_quant_rows<256, 16>(p, bf16, prelude, st);   // K <= 16384
   }
-  // FWHT rows of 128 (fp32) / 256 (bf16) up to 2048 inputs: one warp per row
-  // in registers; other widths: the row staged in shared memory
+  // FWHT rows of 128 (fp32) / 256 (bf16) up to 2048 inputs: the row in
+  // registers, one warp per row up to 256 inputs, two up to 1024, four at
+  // 2048; other widths: the row staged in shared memory
   const bool silu = prelude == PRE_SILU_FWHT;
   if (K <= 2048 && K >= (bf16 ? 256 : 128) && !(silu && bf16)) {
     void (*kw)(QuantParams) = nullptr;
     if (silu) {                    // fp32 hidden rows of the H-BitLinear FFN
       switch (K) {
-        case 128: kw = quant_fwht_warp_kernel<128, false, true>; break;
-        case 256: kw = quant_fwht_warp_kernel<256, false, true>; break;
-        case 512: kw = quant_fwht_warp_kernel<512, false, true>; break;
-        case 1024: kw = quant_fwht_warp_kernel<1024, false, true>; break;
-        default: kw = quant_fwht_warp_kernel<2048, false, true>; break;
+        case 128: kw = quant_fwht_warp_kernel<128, false, true, 1>; break;
+        case 256: kw = quant_fwht_warp_kernel<256, false, true, 1>; break;
+        case 512: kw = quant_fwht_warp_kernel<512, false, true, 2>; break;
+        case 1024: kw = quant_fwht_warp_kernel<1024, false, true, 2>; break;
+        default: kw = quant_fwht_warp_kernel<2048, false, true, 4>; break;
       }
     } else {
       switch (K) {
-        case 128: kw = quant_fwht_warp_kernel<128, false>; break;
-        case 256: kw = bf16 ? quant_fwht_warp_kernel<256, true> : quant_fwht_warp_kernel<256, false>; break;
-        case 512: kw = bf16 ? quant_fwht_warp_kernel<512, true> : quant_fwht_warp_kernel<512, false>; break;
-        case 1024: kw = bf16 ? quant_fwht_warp_kernel<1024, true> : quant_fwht_warp_kernel<1024, false>; break;
-        default: kw = bf16 ? quant_fwht_warp_kernel<2048, true> : quant_fwht_warp_kernel<2048, false>; break;
+        case 128: kw = quant_fwht_warp_kernel<128, false, false, 1>; break;
+        case 256:
+          kw = bf16 ? quant_fwht_warp_kernel<256, true, false, 1> : quant_fwht_warp_kernel<256, false, false, 1>;
+          break;
+        case 512:
+          kw = bf16 ? quant_fwht_warp_kernel<512, true, false, 2> : quant_fwht_warp_kernel<512, false, false, 2>;
+          break;
+        case 1024:
+          kw = bf16 ? quant_fwht_warp_kernel<1024, true, false, 2> : quant_fwht_warp_kernel<1024, false, false, 2>;
+          break;
+        default:
+          kw = bf16 ? quant_fwht_warp_kernel<2048, true, false, 4> : quant_fwht_warp_kernel<2048, false, false, 4>;
+          break;
       }
     }
-    const int rows_per_cta = 4;
+    const int wpr = K >= 2048 ? 4 : K >= 512 ? 2 : 1;
+    const int rows_per_cta = 4 / wpr;
     const int need = (M + rows_per_cta - 1) / rows_per_cta;
     const int cap = di.sms * 16;
     return launch_pdl(kw, dim3(need < cap ? need : cap), dim3(128), 0, st, p);
@@ -612,17 +622,21 @@ int launch_ffn_decode(FfnDecodeParams p, cudaStream_t st, bool tail = false) {
   if (p.M < 1 || p.M > 16 || p.H % 128 != 0 || p.I % 128 != 0) return BITNET_ERR_UNSUPPORTED;
   int G = std::min(std::min(di.sms, kFdMaxGrid), (p.I + 7) / 8);
   p.nf_per = (p.I + G - 1) / G;
-  p.groups = (p.nf_per + 7) / 8;
-  if (p.groups > kFdMaxGroups) return BITNET_ERR_UNSUPPORTED;
+  p.slots = (p.nf_per + 7) / 8;
+  if (p.slots > kFdMaxSlots) return BITNET_ERR_UNSUPPORTED;
   p.nr_per = (p.H + G - 1) / G;
   if (p.nr_per > 32) return BITNET_ERR_UNSUPPORTED;
   p.mpad = p.M <= 8 ? 8 : 16;
   p.sx_h = p.H + kFdRowPad;
   p.sx_i = p.I + kFdRowPad;
-  p.off_gu = 0;
-  p.off_d = (int)align128((size_t)2 * p.nf_per * p.ldwH);
-  p.off_o = (int)align128((size_t)p.off_d + (size_t)p.nr_per * p.ldwI);
-  p.off_act = (int)align128((size_t)p.off_o + (tail ? (size_t)p.nr_per * p.ldwH : 0));
+  // gate and up sub-blocks, then down (TAIL: o_proj rows first, in the same
+  // place), then the staged codes
+  const size_t gu = align128((size_t)sb_bytes(p.nf_per, p.ldwH));
+  p.off_u = (int)gu;
+  p.off_d = (int)(2 * gu);
+  const size_t dn = std::max((size_t)sb_bytes(p.nr_per, p.ldwI),
+                             tail ? (size_t)sb_bytes(p.nr_per, p.ldwH) : (size_t)0);
+  p.off_act = (int)align128((size_t)p.off_d + dn);
   const size_t smem =
       (size_t)p.off_act + (size_t)p.mpad * (size_t)std::max(p.sx_h, p.sx_i) + 128;
   if (smem + sizeof(FfnDecodeShared) + 1024 > (size_t)di.max_smem_optin) return BITNET_ERR_UNSUPPORTED;
@@ -901,8 +915,7 @@ size_t bitnet_ffn_workspace_size(int M, int H, int I, int variant) {
   // and the persistent launch's per-CTA partial sums and exchange flags
   if ((variant & ~BITNET_FFN_SINGLE_LAUNCH) == BITNET_FFN_RELU2_GLU && M <= 16) {
     total += align256(m * (size_t)I * 4);
-    total += align256((size_t)kFdMaxGrid * 16 * sizeof(double));
-    total += align256((size_t)kFdMaxGrid * sizeof(unsigned long long));
+    total += align256(sizeof(FdControl));
   }
   return total;
 }
@@ -964,9 +977,7 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   int32_t* hrs = reinterpret_cast<int32_t*>(ws);         ws += align256(m * 4);
   float* hid_up = reinterpret_cast<float*>(ws);          // decode GLU only
   ws += align256(m * I * 4);
-  double* fd_partials = reinterpret_cast<double*>(ws);
-  ws += align256((size_t)kFdMaxGrid * 16 * sizeof(double));
-  unsigned long long* fd_flags = reinterpret_cast<unsigned long long*>(ws);
+  FdControl* fd_ctl = reinterpret_cast<FdControl*>(ws);  // decode GLU only
   const bool xbf = x_dtype == BITNET_BF16;
 
   LinearParams p1;
@@ -989,7 +1000,7 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
     fp.pre_gain = pre_norm_gain; fp.sub_gain = sub_norm_gain; fp.eps = eps;
     fp.Y = Y; fp.y_bf16 = y_dtype == BITNET_BF16 ? 1 : 0;
     fp.hid = hid; fp.hq = hq; fp.hs = hs; fp.hrs = hrs;
-    fp.partials = fd_partials; fp.flags = fd_flags;
+    fp.ctl = fd_ctl;
     fp.ldwH = (int)bitnet_packed_row_bytes(H); fp.ldwI = (int)bitnet_packed_row_bytes(I);
     const int rc = launch_ffn_decode(fp, st);
     if (rc != BITNET_ERR_UNSUPPORTED) return rc;
@@ -1043,9 +1054,7 @@ size_t bitnet_block_tail_workspace_size(int M, int H, int I) {
   if (M < 0 || H <= 0 || I <= 0) return 0;
   const size_t m = (size_t)M;
   return align256(m * (size_t)I * 4) + align256(m * (size_t)I) + 2 * align256(m * 4) +
-         align256((size_t)kFdMaxGrid * 16 * sizeof(double)) +
-         2 * align256((size_t)kFdMaxGrid * sizeof(unsigned long long)) +
-         align256(m * (size_t)H * 4);
+         align256(sizeof(FdControl)) + align256(m * (size_t)H * 4);
 }
 
 int bitnet_block_tail(const void* A, const void* X, int dtype, int M, int H, int I,
@@ -1086,9 +1095,7 @@ int bitnet_block_tail(const void* A, const void* X, int dtype, int M, int H, int
   fp.hq = reinterpret_cast<int8_t*>(ws);                  ws += align256(m * I);
   fp.hs = reinterpret_cast<float*>(ws);                   ws += align256(m * 4);
   fp.hrs = reinterpret_cast<int32_t*>(ws);                ws += align256(m * 4);
-  fp.partials = reinterpret_cast<double*>(ws);            ws += align256((size_t)kFdMaxGrid * 16 * 8);
-  fp.flags = reinterpret_cast<unsigned long long*>(ws);   ws += align256((size_t)kFdMaxGrid * 8);
-  fp.flags_a = reinterpret_cast<unsigned long long*>(ws); ws += align256((size_t)kFdMaxGrid * 8);
+  fp.ctl = reinterpret_cast<FdControl*>(ws);              ws += align256(sizeof(FdControl));
   fp.hbuf = reinterpret_cast<float*>(ws);
   fp.X = X; fp.A = A; fp.x_bf16 = dtype == BITNET_BF16 ? 1 : 0;
   fp.M = M; fp.H = H; fp.I = I;

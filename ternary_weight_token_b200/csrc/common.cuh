@@ -333,10 +333,16 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
   return v;
 }
 
+// `zero` / `nzero`: counters CTA 0 sets to 0 before it publishes its flag,
+// so that no CTA can reach them (a later grid_count_exchange) before they
+// are reset.
 __device__ __forceinline__ bool grid_exchange(unsigned long long* flags, unsigned long long epoch,
-                                              int* ok_smem) {
+                                              int* ok_smem, unsigned int* zero = nullptr,
+                                              int nzero = 0) {
   __syncthreads();                               // this CTA's global writes are issued
   if (threadIdx.x == 0) {
+    if (blockIdx.x == 0)
+      for (int i = 0; i < nzero; ++i) zero[i] = 0u;
     __threadfence();
     st_release_u64(flags + blockIdx.x, epoch);
     *ok_smem = 1;
@@ -358,6 +364,38 @@ __device__ __forceinline__ bool grid_exchange(unsigned long long* flags, unsigne
       record_device_error(DEV_ERR_TIMEOUT);
       *ok_smem = 0;
     }
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  }
+  __syncthreads();
+  return *ok_smem != 0;
+}
+
+// Grid-wide exchange on an arrival counter that was reset to 0 within this
+// launch (by a grid_exchange before it): thread 0 of each CTA makes the CTA's
+// global writes visible (fence), adds 1, and polls the one counter word until
+// all `expected` CTAs have arrived, bounded by kWaitLimitNs; then an acquire
+// fence.  Polling one word costs about a third of polling every CTA's flag
+// (measured on B200 with a 148-CTA cooperative grid: ~1.1 us against ~3 us
+// per exchange).  Returns false (device error recorded) if the wait gave up.
+__device__ __forceinline__ bool grid_count_exchange(unsigned int* ctr, unsigned int expected,
+                                                    int* ok_smem) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const unsigned long long t0 = global_timer_ns();
+    bool done = false;
+    for (uint32_t it = 0;; ++it) {
+      unsigned int v;
+      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+      if (v >= expected) {
+        done = true;
+        break;
+      }
+      if ((it & 15u) == 15u && global_timer_ns() - t0 > kWaitLimitNs) break;
+    }
+    if (!done) record_device_error(DEV_ERR_TIMEOUT);
+    *ok_smem = done ? 1 : 0;
     asm volatile("fence.acq_rel.gpu;" ::: "memory");
   }
   __syncthreads();

@@ -1,5 +1,6 @@
 // ffn_decode.cuh -- the W1.58A8 FFN of one block at decode sizes (1..16
-// tokens) in ONE persistent launch.
+// tokens) in ONE persistent launch, optionally preceded by the attention
+// output projection and its residual (the block after attention).
 //
 // nnterp encyclopedia "bitnet", "The block, in order" and "The MLP gates with
 // a squared ReLU":
@@ -12,13 +13,12 @@
 //
 // For a few tokens the FFN streams 13 MB of packed weights and does little
 // arithmetic; run as four launches it pays four grid ramps and completions.
-// Here one cooperative grid (one CTA per SM) does it with a single grid-wide
-// exchange:
-//   P0  thread 0 of every CTA bulk-copies its weight rows into shared memory
-//       at once, one copy per block of contiguous rows: its gate rows, the
-//       matching up rows and its slice of down rows (the fragment loads of 8
-//       rows of one 16-byte-multiple stride share banks; a copy per padded
-//       row was measured far slower, the copy engine taking ~0.1 us a copy);
+// Here one cooperative grid (one CTA per SM) does it:
+//   P0  warp 0 bulk-copies the CTA's weight rows into shared memory at once:
+//       its gate rows, the matching up rows and its slice of down rows, each
+//       as 8 sub-blocks of consecutive rows whose shared-memory starts differ
+//       by 16 bytes mod 128, so the 8 rows an mma fragment load touches (one
+//       per sub-block, same column) fall in 8 different bank quads;
 //   P1  every CTA quantises all tokens of x itself (RMSNorm prelude; a row is
 //       spread over several warps, its loads all in flight): x is a few KB,
 //       so the redundant work costs less than an exchange;
@@ -27,18 +27,21 @@
 //       fragment holds 8 gate rows over the same 8 up rows, so one thread
 //       holds the gate and up sums of a feature and forms m = relu(g)^2 * u
 //       (fp32, the fused epilogue's operations) directly; the warps split K
-//       and add their sums with shared-memory atomics (exact in int32); m goes
-//       to the workspace and each CTA's fp64 partial sums of m^2 per token to
-//       a partials array;
-//   P3  grid-wide exchange: each CTA publishes a 64-bit epoch in its flag
-//       (release) and waits, bounded, until every flag holds the epoch;
-//   P4  every CTA adds the partials in a fixed order (the same fp32 mean
-//       square in every CTA), then forms the sub-norm codes of all of m in
-//       shared memory (m read back from L2);
+//       and add their sums with shared-memory atomics (exact in int32);
+//   X1  each CTA publishes its fp64 sums of m^2 per token; exchange;
+//   P3  every CTA adds the G partial sums in one fixed order (the same fp32
+//       mean square, hence the same r, in every CTA), forms xh = (m r) g for
+//       its own features and publishes their max |xh| per token; exchange X2;
+//   P4  s = 127 / max over the CTAs' maxima (exact in any order); each CTA
+//       writes the codes of its own features to the workspace and publishes
+//       their code sum per token; exchange X3; every CTA loads all codes;
 //   P5  its down rows against those codes (mma.sync again), dequantised,
 //       plus the residual x, stored.
-// The epoch is new for every launch (a per-process 64-bit counter started at
-// a random value), so the flags need no reset and the workspace no zeroing.
+// The first exchange of a launch polls one flag per CTA holding a 64-bit
+// epoch that is new for every launch (a per-process counter started at a
+// random value), so it needs no reset and the workspace no zeroing; CTA 0
+// resets the arrival counters of the later exchanges before it publishes its
+// flag, and those exchanges poll one counter word.
 #pragma once
 
 #include "common.cuh"
@@ -48,9 +51,19 @@
 namespace bitnet {
 
 constexpr int kFdThreads = 256;           // 8 warps
-constexpr int kFdMaxGroups = 8;           // 8-feature groups per CTA (<= 64 features)
-constexpr int kFdMaxGrid = 256;           // flags / partials slots in the workspace
-constexpr int kFdRowPad = 16;             // bytes added to every staged row
+constexpr int kFdMaxSlots = 8;            // rows per gate / up sub-block (<= 64 features per CTA)
+constexpr int kFdMaxGrid = 256;           // partials / flags slots in the control block
+constexpr int kFdRowPad = 16;             // bytes added to every staged code row
+constexpr int kFdRegChunks = 24;          // float4 chunks per thread held in the row quantiser
+
+// Control block of one persistent launch, in the caller's workspace.
+struct FdControl {
+  double ss[kFdMaxGrid][16];              // per-CTA sums of m^2, per token
+  float mx[kFdMaxGrid][16];               // per-CTA max |xh|, per token
+  int cs[kFdMaxGrid][16];                 // per-CTA code sums, per token
+  unsigned long long flags[kFdMaxGrid];   // first exchange: epoch flags
+  unsigned int ctr[4];                    // later exchanges: arrival counters
+};
 
 struct FfnDecodeParams {
   const void* X;               // [M][H] bf16 or fp32
@@ -67,12 +80,11 @@ struct FfnDecodeParams {
   float eps;
   void* Y;                     // [M][H], y_bf16 ? bf16 : fp32
   int y_bf16;
-  float* hid;                  // [M][I] fp32 m (workspace)
-  int8_t* hq;                  // [M][I] sub-norm codes (written by CTA 0, for inspection)
-  float* hs;                   // [M] their scales
-  int32_t* hrs;                // [M] their code sums
-  double* partials;            // [kFdMaxGrid][16] per-CTA sums of m^2
-  unsigned long long* flags;   // [kFdMaxGrid]
+  float* hid;                  // [M][I] fp32 m (each CTA its features; for inspection)
+  int8_t* hq;                  // [M][I] sub-norm codes (each CTA its features; read back by all)
+  float* hs;                   // [M] their scales (CTA 0)
+  int32_t* hrs;                // [M] their code sums (CTA 0)
+  FdControl* ctl;
   unsigned long long epoch;
   // the block after attention (TAIL kernels only): X is the residual stream
   // x, A the attention output, h = x + o_proj(attn_sub_norm(A)) in fp32
@@ -82,31 +94,50 @@ struct FfnDecodeParams {
   const float* attn_gain;      // [H] or null
   float* hbuf;                 // [M][H] fp32 h (workspace)
   void* H_out;                 // [M][H] h in Y's type, or null
-  unsigned long long* flags_a; // [kFdMaxGrid] flags of the first exchange
-  int off_o;                   // o_proj rows in shared memory
   int ldwH, ldwI;
   int nf_per, nr_per;          // features / down rows per CTA (the last CTAs fewer)
-  int groups;                  // 8-feature groups per CTA
+  int slots;                   // rows per gate / up sub-block: ceil(nf_per / 8)
   int mpad;                    // tokens rounded up to 8
-  // shared-memory carve-up (bytes from the 128-aligned base)
-  int off_gu, off_d, off_act;
+  // shared-memory carve-up (bytes from the 128-aligned base): gate sub-blocks
+  // at 0, up at off_u, down (TAIL: o_proj first, then down) at off_d
+  int off_u, off_d, off_act;
   int sx_h, sx_i;              // staged code row strides (K + 16: conflict-free fragments)
 };
 
 struct FfnDecodeShared {
-  int red[kFdMaxGroups * 2 * 32 * 4];   // P2 sums [group][ntile][lane][4]; P5 reuses it
+  int red[kFdMaxSlots * 2 * 32 * 4];    // P2 sums [slot][ntile][lane][4]; P5 reuses it
   float f_hi[2][16], f_lo[2][16];       // dequant factors of x (gate, up) per token
   int rs_x[16];
   float s_x[16];
   float fd_hi[16], fd_lo[16];           // down dequant factors per token
   int rs_m[16];
   float s_m[16];                        // sub-norm scales per token
+  float r_m[16];                        // sub-norm 1 / rms per token
+  int zr_m[16];                         // all-zero hidden row
   float fo_hi[16], fo_lo[16];           // o_proj dequant factors per token
   int rs_a[16];
+  float s_a[16];
   int ok;                               // weights landed / exchanges completed
   int xok;
   __align__(8) uint64_t bar_gu, bar_d, bar_o;
 };
+
+// ---- sub-block layout of a CTA's n staged rows (row stride ldw bytes):
+// sub-block g (0..7) holds sb_count(n, g) consecutive rows starting at row
+// sb_first(n, g), at byte sb_base(n, ldw, g) = 16 g (mod 128).
+__host__ __device__ inline int sb_count(int n, int g) { return n / 8 + (g < n % 8 ? 1 : 0); }
+__host__ __device__ inline int sb_first(int n, int g) {
+  return g * (n / 8) + (g < n % 8 ? g : n % 8);
+}
+__host__ __device__ inline int sb_span(int n, int ldw, int g) {
+  return (sb_count(n, g) * ldw + 128 + 127) & ~127;
+}
+__host__ __device__ inline int sb_base(int n, int ldw, int g) {
+  int b = 0;
+  for (int j = 0; j < g; ++j) b += sb_span(n, ldw, j);
+  return b + 16 * g;
+}
+__host__ __device__ inline int sb_bytes(int n, int ldw) { return sb_base(n, ldw, 8) - 16 * 8; }
 
 __device__ __forceinline__ void mma_u8s8_16832(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                                uint32_t a3, uint32_t b0, uint32_t b1) {
@@ -128,11 +159,31 @@ __device__ __forceinline__ void bulk_copy_g2s(void* dst, const void* src, uint32
       : "memory");
 }
 
+// Sub-blocks of rows [row0, row0 + n) of a packed matrix into shared memory
+// at `dst` (lane g of the calling warp copies sub-block g).
+__device__ __forceinline__ void copy_sub_blocks(uint8_t* dst, const uint8_t* W, int row0, int n,
+                                                int ldw, uint64_t* bar, int lane) {
+  if (lane < 8) {
+    const int cnt = sb_count(n, lane);
+    if (cnt > 0)
+      bulk_copy_g2s(dst + sb_base(n, ldw, lane),
+                    W + (size_t)(row0 + sb_first(n, lane)) * ldw, (uint32_t)(cnt * ldw), bar);
+  }
+}
+
 // L2-coherent loads of data other CTAs of this grid wrote.
 __device__ __forceinline__ float4 ld_cg_f4(const float* p) {
   float4 v;
   asm volatile("ld.global.cg.v4.f32 {%0, %1, %2, %3}, [%4];"
                : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ uint4 ld_cg_u4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p));
   return v;
 }
@@ -156,21 +207,11 @@ __device__ __forceinline__ float warp_max_f32(float v) {
   return v;
 }
 
-// Codes of the M token rows of an [M][n] activation (RMSNorm prelude, the
-// library's arithmetic: mean square accumulated in fp64 from exact squares and
-// rounded once, r = 1/sqrt(ms + eps) in fp32, xh = (x r) g, s = 127 / max|xh|,
-// q = rint(xh s)) into shared memory rows of `stride` bytes; padded tokens
-// (M <= m < mpad) get zero codes.  Every thread of the CTA calls it.
-//   Rows are spread over the warps so that all of them work for any M: with
-//   rp rows in flight (1, 2, 4 or 8), a row gets gw = 8 / rp warps, and each
-//   of its threads holds up to kFdRegChunks float4 chunks in registers, all
-//   loaded before any is used (longer rows are done in batches, reloaded per
-//   pass).  Sums and maxima are combined in a fixed order (thread, warp xor
-//   tree, the row's warps in turn), the same in every CTA.
-//   KIND 0: fp32 rows, 1: bf16 rows, 2: fp32 rows this grid wrote (loaded
-//   from L2).  partials != null: the row's sum of squares is the sum of
-//   partials[i * 16 + m] over i < nparts instead.
-constexpr int kFdRegChunks = 8;
+// int8 code of an already scaled value y (|y| <= 127 (1 + 2^-24)^2): rint
+// half-to-even by one fp32 add of 1.5 * 2^23, the code is the sum's low byte.
+__device__ __forceinline__ int code_of(float y) {
+  return (int)(int8_t)(__float_as_uint(__fadd_rn(y, 12582912.0f)) & 0xffu);
+}
 
 template <int KIND>
 __device__ __forceinline__ float4 fd_load4(const void* src, size_t elem) {
@@ -184,10 +225,25 @@ __device__ __forceinline__ float4 fd_load4(const void* src, size_t elem) {
   return *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(src) + elem);
 }
 
+// Codes of the M token rows of an [M][n] activation (RMSNorm prelude, the
+// library's arithmetic: mean square accumulated in fp64 from exact squares and
+// rounded once, r = 1/sqrt(ms + eps) in fp32, xh = (x r) g, s = 127 / max|xh|,
+// q = rint(xh s)) into shared memory rows of `stride` bytes.  Rows past M are
+// not written (their mma columns are discarded).  Every thread of the CTA
+// calls it.
+//   Rows are spread over the warps so that all of them work for any M: with
+//   rp rows in flight (1, 2, 4 or 8), a row gets gw = 8 / rp warps, and each
+//   of its threads holds up to kFdRegChunks float4 chunks in registers, all
+//   loaded before any is used (longer rows are done in batches, reloaded per
+//   pass).  A thread keeps four fp64 sums (one per float4 lane: short
+//   dependency chains) added in a fixed order; sums and maxima are then
+//   combined in a fixed order (warp xor tree, the row's warps in turn), the
+//   same in every CTA.
+//   KIND 0: fp32 rows, 1: bf16 rows, 2: fp32 rows this grid wrote (loaded
+//   from L2).
 template <int KIND>
-__device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const float* gain,
-                              float eps, int8_t* s_act, int stride, float* s_out, int* rs_out,
-                              const double* partials = nullptr, int nparts = 0) {
+__device__ void fd_quant_rows(const void* src, int M, int n, const float* gain, float eps,
+                              int8_t* s_act, int stride, float* s_out, int* rs_out) {
   __shared__ double red_d[8];
   __shared__ float red_f[8];
   __shared__ int red_i[8];
@@ -200,13 +256,13 @@ __device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const flo
   const int per = (nc + tstride - 1) / tstride;               // chunks per thread
   const int first = lane + 32 * wg;                           // this thread's first chunk
   const bool fits = per <= kFdRegChunks;
-  for (int round = 0; round * rp < mpad; ++round) {
+  for (int round = 0; round * rp < M; ++round) {
     const int m = round * rp + grp;
     const bool row = m < M;
     const size_t base = (size_t)(row ? m : 0) * n;
     float4 v[kFdRegChunks];
-    // pass 1: sum of squares (unless given) and max|x|
-    double ss = 0.0;
+    // pass 1: sum of squares and max|x|
+    double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
     float xmax = 0.0f;
     for (int b0 = 0; b0 < per; b0 += kFdRegChunks) {
 #pragma unroll
@@ -217,16 +273,17 @@ __device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const flo
       }
 #pragma unroll
       for (int i = 0; i < kFdRegChunks; ++i) {
-        if (partials == nullptr) {
-          ss = fma((double)v[i].x, (double)v[i].x, ss); ss = fma((double)v[i].y, (double)v[i].y, ss);
-          ss = fma((double)v[i].z, (double)v[i].z, ss); ss = fma((double)v[i].w, (double)v[i].w, ss);
+        if (row && b0 + i < per && first + (b0 + i) * tstride < nc) {
+          s0 = fma((double)v[i].x, (double)v[i].x, s0);
+          s1 = fma((double)v[i].y, (double)v[i].y, s1);
+          s2 = fma((double)v[i].z, (double)v[i].z, s2);
+          s3 = fma((double)v[i].w, (double)v[i].w, s3);
+          xmax = fmaxf(xmax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)),
+                                   fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
         }
-        xmax = fmaxf(xmax, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
       }
     }
-    if (partials != nullptr && row && wg == 0)
-      for (int i = lane; i < nparts; i += 32) ss += ld_cg_f64(partials + (size_t)i * 16 + m);
-    ss = warp_sum_f64(ss);
+    double ss = warp_sum_f64((s0 + s1) + (s2 + s3));
     xmax = warp_max_f32(xmax);
     if (lane == 0) { red_d[warp] = ss; red_f[warp] = xmax; }
     __syncthreads();
@@ -278,7 +335,7 @@ __device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const flo
     if (zero_row) s = 1.0f;
     // pass 3: codes and their sum
     int rsum = 0;
-    int8_t* dst = s_act + (size_t)m * stride;
+    int8_t* dst = s_act + (size_t)(row ? m : 0) * stride;
     for (int b0 = 0; b0 < per; b0 += kFdRegChunks) {
       if (!fits) {
 #pragma unroll
@@ -291,9 +348,9 @@ __device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const flo
 #pragma unroll
       for (int i = 0; i < kFdRegChunks; ++i) {
         const int c = first + (b0 + i) * tstride;
-        if (m < mpad && b0 + i < per && c < nc) {
+        if (row && b0 + i < per && c < nc) {
           uint32_t w = 0u;
-          if (row && !zero_row) {
+          if (!zero_row) {
             const float4 g = gain ? __ldg(reinterpret_cast<const float4*>(gain) + c)
                                   : make_float4(1.f, 1.f, 1.f, 1.f);
             w = pack_codes4(__fmul_rn(__fmul_rn(__fmul_rn(v[i].x, r), g.x), s),
@@ -319,16 +376,22 @@ __device__ void fd_quant_rows(const void* src, int M, int mpad, int n, const flo
   }
 }
 
-// int32 sums of `nr` staged weight rows (stride sw) against the staged codes
-// (stride sx) over K inputs, added into red[(i * 2 + t) * 32 + lane][4]
-// (row tile i <= 1, token tile t): the 8 warps split the K steps of 32.
-__device__ __forceinline__ void fd_contract_rows(const uint8_t* s_w, int sw, int nr,
+// int32 sums of the CTA's nr staged rows (sub-block layout, stride ldw)
+// against the staged codes (stride sx) over K inputs, added into
+// red[(i * 2 + t) * 32 + lane][4]: row tile i <= 1 holds slots 2i (fragment
+// rows 0..7, one per sub-block) and 2i + 1 (rows 8..15) of the sub-blocks,
+// token tile t <= 1; the 8 warps split the K steps of 32.
+__device__ __forceinline__ void fd_contract_rows(const uint8_t* s_w, int ldw, int nr,
                                                  const int8_t* s_x, int sx, int K, int ntile,
                                                  int* red) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c4 = lane & 3;
   const int steps = K / 32;
   const int s_lo = warp * steps / 8, s_hi = (warp + 1) * steps / 8;
+  const int cmax = sb_count(nr, 0);                  // slots of the largest sub-block
+  const int cnt = sb_count(nr, g8);
+  const int clast = cnt > 0 ? cnt - 1 : 0;           // slots past cnt read a valid row
+  const uint8_t* wb = s_w + sb_base(nr, ldw, g8);
   int acc[2][2][4];
 #pragma unroll
   for (int i = 0; i < 2; ++i)
@@ -336,7 +399,6 @@ __device__ __forceinline__ void fd_contract_rows(const uint8_t* s_w, int sw, int
     for (int t = 0; t < 2; ++t)
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[i][t][e] = 0;
-  const int last = nr > 0 ? nr - 1 : 0;            // rows past nr read a valid row
   for (int s = s_lo; s < s_hi; ++s) {
     uint32_t bf[2][2];
 #pragma unroll
@@ -349,10 +411,10 @@ __device__ __forceinline__ void fd_contract_rows(const uint8_t* s_w, int sw, int
     }
 #pragma unroll
     for (int i = 0; i < 2; ++i) {
-      if (16 * i < nr) {
-        const int r0 = min(16 * i + g8, last), r1 = min(16 * i + 8 + g8, last);
-        const uint2 lo = *reinterpret_cast<const uint2*>(s_w + (size_t)r0 * sw + 8 * s);
-        const uint2 hi = *reinterpret_cast<const uint2*>(s_w + (size_t)r1 * sw + 8 * s);
+      if (2 * i < cmax) {
+        const uint2 lo = *reinterpret_cast<const uint2*>(wb + (size_t)min(2 * i, clast) * ldw + 8 * s);
+        const uint2 hi =
+            *reinterpret_cast<const uint2*>(wb + (size_t)min(2 * i + 1, clast) * ldw + 8 * s);
         const uint32_t a0 = (lo.x >> (2 * c4)) & 0x03030303u;
         const uint32_t a2 = (lo.y >> (2 * c4)) & 0x03030303u;
         const uint32_t a1 = (hi.x >> (2 * c4)) & 0x03030303u;
@@ -367,9 +429,16 @@ __device__ __forceinline__ void fd_contract_rows(const uint8_t* s_w, int sw, int
   for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int t = 0; t < 2; ++t)
-      if (16 * i < nr && t < ntile)
+      if (2 * i < cmax && t < ntile)
 #pragma unroll
         for (int e = 0; e < 4; ++e) atomicAdd(&red[((i * 2 + t) * 32 + lane) * 4 + e], acc[i][t][e]);
+}
+
+// Row index (within the CTA's nr rows) of output element (row tile i, half,
+// lane) of fd_contract_rows, or -1.
+__device__ __forceinline__ int fd_contract_row(int nr, int i, int half, int lane) {
+  const int g = lane >> 2, slot = 2 * i + half;
+  return slot < sb_count(nr, g) ? sb_first(nr, g) + slot : -1;
 }
 
 template <bool TAIL>
@@ -378,11 +447,11 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   __shared__ FfnDecodeShared sh;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(fd_smem_raw) + 127) & ~uintptr_t(127));
-  uint8_t* s_g = smem + p.off_gu;           // [nf_per][ldwH] gate rows
-  uint8_t* s_u = s_g + (size_t)p.nf_per * p.ldwH;   // [nf_per][ldwH] up rows
-  uint8_t* s_d = smem + p.off_d;            // [nr][ldwI]
-  uint8_t* s_o = smem + p.off_o;            // [nr][ldwH] (TAIL)
+  uint8_t* s_g = smem;                      // gate sub-blocks (ldwH rows)
+  uint8_t* s_u = smem + p.off_u;            // up sub-blocks
+  uint8_t* s_d = smem + p.off_d;            // down sub-blocks (ldwI rows); TAIL: o_proj first
   int8_t* s_act = reinterpret_cast<int8_t*>(smem + p.off_act);   // [mpad][sx_h or sx_i]
+  FdControl* ctl = p.ctl;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g8 = lane >> 2, c4 = lane & 3;          // mma fragment coordinates
@@ -396,7 +465,7 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   const int M = p.M;
   const int ntile = p.mpad / 8;
 
-  // ---- P0: weight rows -> shared memory (one thread issues every copy)
+  // ---- P0: weight rows -> shared memory (warp 0: lane g copies sub-block g)
   if (threadIdx.x == 0) {
     mbar_init(&sh.bar_gu, 1);
     mbar_init(&sh.bar_d, 1);
@@ -405,46 +474,51 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     sh.ok = 1;
   }
   __syncthreads();
-  // one bulk copy per block of contiguous rows (many small copies keep the
-  // copy engine busy for longer than the bytes take)
-  if (threadIdx.x == 0) {
-    if (TAIL) {                                       // needed first
-      mbar_arrive_expect_tx(&sh.bar_o, (uint32_t)(nr * p.ldwH));
-      if (nr > 0)
-        bulk_copy_g2s(s_o, p.Wo + (size_t)n0 * p.ldwH, (uint32_t)(nr * p.ldwH), &sh.bar_o);
+  if (warp == 0) {
+    if (lane == 0) {
+      if (TAIL) mbar_arrive_expect_tx(&sh.bar_o, (uint32_t)(nr * p.ldwH));
+      mbar_arrive_expect_tx(&sh.bar_gu, (uint32_t)(2 * nf * p.ldwH));
+      if (!TAIL) mbar_arrive_expect_tx(&sh.bar_d, (uint32_t)(nr * p.ldwI));
     }
-    mbar_arrive_expect_tx(&sh.bar_gu, (uint32_t)(2 * nf * p.ldwH));
-    if (nf > 0) {
-      bulk_copy_g2s(s_g, p.Wg + (size_t)f0 * p.ldwH, (uint32_t)(nf * p.ldwH), &sh.bar_gu);
-      bulk_copy_g2s(s_u, p.Wu + (size_t)f0 * p.ldwH, (uint32_t)(nf * p.ldwH), &sh.bar_gu);
-    }
-    mbar_arrive_expect_tx(&sh.bar_d, (uint32_t)(nr * p.ldwI));
-    if (nr > 0)
-      bulk_copy_g2s(s_d, p.Wd + (size_t)n0 * p.ldwI, (uint32_t)(nr * p.ldwI), &sh.bar_d);
+    __syncwarp();
+    if (TAIL) copy_sub_blocks(s_d, p.Wo, n0, nr, p.ldwH, &sh.bar_o, lane);   // needed first
+    copy_sub_blocks(s_g, p.Wg, f0, nf, p.ldwH, &sh.bar_gu, lane);
+    copy_sub_blocks(s_u, p.Wu, f0, nf, p.ldwH, &sh.bar_gu, lane);
+    if (!TAIL) copy_sub_blocks(s_d, p.Wd, n0, nr, p.ldwI, &sh.bar_d, lane);
   }
 
   // ---- TAIL: h = x + o_proj(attn_sub_norm(A)) for this CTA's rows, then
   // the first exchange; every CTA then quantises all of h
   if constexpr (TAIL) {
     if (p.x_bf16)
-      fd_quant_rows<1>(p.A, M, p.mpad, p.H, p.attn_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_a);
+      fd_quant_rows<1>(p.A, M, p.H, p.attn_gain, p.eps, s_act, p.sx_h, sh.s_a, sh.rs_a);
     else
-      fd_quant_rows<0>(p.A, M, p.mpad, p.H, p.attn_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_a);
+      fd_quant_rows<0>(p.A, M, p.H, p.attn_gain, p.eps, s_act, p.sx_h, sh.s_a, sh.rs_a);
     for (int i = threadIdx.x; i < 2 * 2 * 32 * 4; i += kFdThreads) sh.red[i] = 0;
     __syncthreads();
-    if (threadIdx.x < M) dequant_factor(__ldg(p.gamma_o), sh.s_x[threadIdx.x],
+    if (threadIdx.x < M) dequant_factor(__ldg(p.gamma_o), sh.s_a[threadIdx.x],
                                         sh.fo_hi[threadIdx.x], sh.fo_lo[threadIdx.x]);
     if (!mbar_wait(&sh.bar_o, 0, nullptr) && lane == 0) sh.ok = 0;
-    fd_contract_rows(s_o, p.ldwH, nr, s_act, p.sx_h, p.H, ntile, sh.red);
+    fd_contract_rows(s_d, p.ldwH, nr, s_act, p.sx_h, p.H, ntile, sh.red);
     __syncthreads();
+    // the o_proj rows are read: the down rows go to the same place
+    if (warp == 0) {
+      if (lane == 0) {
+        fence_proxy_async_shared();
+        mbar_arrive_expect_tx(&sh.bar_d, (uint32_t)(nr * p.ldwI));
+      }
+      __syncwarp();
+      if (lane < 8) fence_proxy_async_shared();
+      copy_sub_blocks(s_d, p.Wd, n0, nr, p.ldwI, &sh.bar_d, lane);
+    }
     if (threadIdx.x < 2 * 2 * 32) {
       const int idx = threadIdx.x;
       const int i = idx >> 6, t = (idx >> 5) & 1, ln = idx & 31;
       if (t < ntile) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          const int r = 16 * i + 8 * half + (ln >> 2);
-          if (r >= nr) continue;
+          const int r = fd_contract_row(nr, i, half, ln);
+          if (r < 0) continue;
           const int n = n0 + r;
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
@@ -467,14 +541,14 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
         }
       }
     }
-    if (!grid_exchange(p.flags_a, p.epoch, &sh.xok) && threadIdx.x == 0) sh.ok = 0;
-    fd_quant_rows<2>(p.hbuf, M, p.mpad, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
+    if (!grid_exchange(ctl->flags, p.epoch, &sh.xok, ctl->ctr, 4) && threadIdx.x == 0) sh.ok = 0;
+    fd_quant_rows<2>(p.hbuf, M, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
   } else {
     // ---- P1: codes of x (RMSNorm prelude), every token, into s_act
     if (p.x_bf16)
-      fd_quant_rows<1>(p.X, M, p.mpad, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
+      fd_quant_rows<1>(p.X, M, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
     else
-      fd_quant_rows<0>(p.X, M, p.mpad, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
+      fd_quant_rows<0>(p.X, M, p.H, p.pre_gain, p.eps, s_act, p.sx_h, sh.s_x, sh.rs_x);
   }
   __syncthreads();
   if (threadIdx.x < M) {
@@ -482,19 +556,25 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     dequant_factor(__ldg(p.gamma_g), sh.s_x[m], sh.f_hi[0][m], sh.f_lo[0][m]);
     dequant_factor(__ldg(p.gamma_u), sh.s_x[m], sh.f_hi[1][m], sh.f_lo[1][m]);
   }
-  for (int i = threadIdx.x; i < kFdMaxGroups * 2 * 32 * 4; i += kFdThreads) sh.red[i] = 0;
+  for (int i = threadIdx.x; i < kFdMaxSlots * 2 * 32 * 4; i += kFdThreads) sh.red[i] = 0;
   __syncthreads();
 
-  // ---- P2: gate / up sums of this CTA's features (warps split K)
+  // ---- P2: gate / up sums of this CTA's features (warps split K).  Fragment
+  // rows 0..7 are the gate rows of one feature per sub-block (slot j), rows
+  // 8..15 the up rows of the same features.
   {
     const bool landed = mbar_wait(&sh.bar_gu, 0, nullptr);
     if (!landed && lane == 0) sh.ok = 0;
-    const int flast = nf > 0 ? nf - 1 : 0;
+    const int cnt = sb_count(nf, g8);
+    const int clast = cnt > 0 ? cnt - 1 : 0;         // slots past cnt read a valid row
+    const int sbase = sb_base(nf, p.ldwH, g8);
+    const uint8_t* gb = s_g + sbase;
+    const uint8_t* ub = s_u + sbase;
     const int steps = p.H / 32;
     const int s_lo = warp * steps / 8, s_hi = (warp + 1) * steps / 8;
-    int acc[kFdMaxGroups][2][4];
+    int acc[kFdMaxSlots][2][4];
 #pragma unroll
-    for (int j = 0; j < kFdMaxGroups; ++j)
+    for (int j = 0; j < kFdMaxSlots; ++j)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
@@ -510,13 +590,11 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
         }
       }
 #pragma unroll
-      for (int j = 0; j < kFdMaxGroups; ++j) {
-        if (j < p.groups) {
-          // fragment rows g8 (gate) and 8 + g8 (up) of feature 8 j + g8;
-          // features past nf read a valid row (results discarded)
-          const size_t off = (size_t)min(8 * j + g8, flast) * p.ldwH + 8 * s;
-          const uint2 lo = *reinterpret_cast<const uint2*>(s_g + off);       // gate row
-          const uint2 hi = *reinterpret_cast<const uint2*>(s_u + off);       // up row
+      for (int j = 0; j < kFdMaxSlots; ++j) {
+        if (j < p.slots) {
+          const size_t off = (size_t)min(j, clast) * p.ldwH + 8 * s;
+          const uint2 lo = *reinterpret_cast<const uint2*>(gb + off);       // gate row
+          const uint2 hi = *reinterpret_cast<const uint2*>(ub + off);       // up row
           const uint32_t a0 = (lo.x >> (2 * c4)) & 0x03030303u;
           const uint32_t a2 = (lo.y >> (2 * c4)) & 0x03030303u;
           const uint32_t a1 = (hi.x >> (2 * c4)) & 0x03030303u;
@@ -528,17 +606,17 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
       }
     }
 #pragma unroll
-    for (int j = 0; j < kFdMaxGroups; ++j)
+    for (int j = 0; j < kFdMaxSlots; ++j)
 #pragma unroll
       for (int t = 0; t < 2; ++t)
-        if (j < p.groups && t < ntile)
+        if (j < p.slots && t < ntile)
 #pragma unroll
           for (int e = 0; e < 4; ++e) atomicAdd(&sh.red[((j * 2 + t) * 32 + lane) * 4 + e], acc[j][t][e]);
   }
   __syncthreads();
-  // m = relu(g)^2 * u for (feature, token): thread (group j, tile t, lane)
-  // holds gate sums of feature 8j + g8 for tokens 8t + 2c4 + {0, 1} in
-  // red[.][0..1] and the up sums in red[.][2..3]
+  // m = relu(g)^2 * u for (feature, token): thread (slot j, tile t, lane)
+  // holds gate sums of the feature in slot j of sub-block lane / 4 for tokens
+  // 8t + 2 (lane % 4) + {0, 1} in red[.][0..1] and the up sums in red[.][2..3]
   float* m_loc = reinterpret_cast<float*>(sh.red);   // reused below: [16][64] after a barrier
   float mvals[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   int mf[2] = {-1, -1};
@@ -547,8 +625,9 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     const int idx = threadIdx.x + it * kFdThreads;     // (j * 2 + t) * 32 + lane
     const int jt = idx >> 5, ln = idx & 31;
     const int j = jt >> 1, t = jt & 1;
-    const int f = 8 * j + (ln >> 2);
-    if (j >= p.groups || t >= ntile || f >= nf) continue;
+    const int g = ln >> 2;
+    if (j >= p.slots || t >= ntile || j >= sb_count(nf, g)) continue;
+    const int f = sb_first(nf, g) + j;
     mf[it] = f;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -583,17 +662,99 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
       v = fma(d, d, v);
     }
     v = warp_sum_f64(v);
-    if (lane == 0) p.partials[(size_t)b * 16 + m] = v;
+    if (lane == 0) ctl->ss[b][m] = v;
   }
 
-  // ---- P3: grid-wide exchange (bounded)
-  if (!grid_exchange(p.flags, p.epoch, &sh.xok) && threadIdx.x == 0) sh.ok = 0;
-  __syncthreads();
+  // ---- X1: the sums of m^2
+  if (TAIL) {
+    if (!grid_count_exchange(&ctl->ctr[0], (unsigned)G, &sh.xok) && threadIdx.x == 0) sh.ok = 0;
+  } else {
+    if (!grid_exchange(ctl->flags, p.epoch, &sh.xok, ctl->ctr, 4) && threadIdx.x == 0) sh.ok = 0;
+  }
 
-  // ---- P4: sub-norm codes of all of m (every CTA), into s_act; the sum of
-  // squares of each token from the CTAs' partials (fixed order)
-  fd_quant_rows<2>(p.hid, M, p.mpad, p.I, p.sub_gain, p.eps, s_act, p.sx_i, sh.s_m, sh.rs_m,
-                   p.partials, G);
+  // ---- P3: r per token (the G partial sums in one fixed order: lanes take
+  // every 32nd CTA in turn, then the warp's xor tree), then xh of this CTA's
+  // features and their max
+  for (int m = warp; m < M; m += kFdThreads / 32) {
+    double v = 0.0;
+    for (int i = lane; i < G; i += 32) v += ld_cg_f64(&ctl->ss[i][m]);
+    v = warp_sum_f64(v);
+    if (lane == 0) {
+      const float ms = (float)(v / (double)p.I);
+      sh.r_m[m] = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
+    }
+  }
+  __syncthreads();
+  for (int m = warp; m < M; m += kFdThreads / 32) {
+    const float r = sh.r_m[m];
+    float amax = 0.0f;
+    for (int f = lane; f < nf; f += 32) {
+      const float g = p.sub_gain ? __ldg(p.sub_gain + f0 + f) : 1.0f;
+      const float xh = __fmul_rn(__fmul_rn(m_loc[m * 64 + f], r), g);
+      m_loc[m * 64 + f] = xh;
+      amax = fmaxf(amax, fabsf(xh));
+    }
+    amax = warp_max_f32(amax);
+    if (lane == 0) ctl->mx[b][m] = amax;
+  }
+
+  // ---- X2: the maxima
+  if (!grid_count_exchange(&ctl->ctr[TAIL ? 1 : 0], (unsigned)G, &sh.xok) && threadIdx.x == 0)
+    sh.ok = 0;
+
+  // ---- P4: s per token, codes of this CTA's features -> workspace
+  for (int m = warp; m < M; m += kFdThreads / 32) {
+    float amax = 0.0f;
+    for (int i = lane; i < G; i += 32) amax = fmaxf(amax, __ldcg(&ctl->mx[i][m]));
+    amax = warp_max_f32(amax);
+    float s = __fdiv_rn(127.0f, amax);
+    const bool zero_row = (amax == 0.0f) || isinf(s);
+    if (zero_row) s = 1.0f;
+    int csum = 0;
+    for (int f = lane; f < nf; f += 32) {
+      const int q = zero_row ? 0 : code_of(__fmul_rn(m_loc[m * 64 + f], s));
+      p.hq[(size_t)m * p.I + f0 + f] = (int8_t)q;
+      csum += q;
+    }
+    csum = __reduce_add_sync(0xffffffffu, csum);
+    if (lane == 0) {
+      ctl->cs[b][m] = csum;
+      sh.s_m[m] = s;
+    }
+  }
+
+  // ---- X3: the codes
+  if (!grid_count_exchange(&ctl->ctr[TAIL ? 2 : 1], (unsigned)G, &sh.xok) && threadIdx.x == 0)
+    sh.ok = 0;
+
+  // every CTA: code sums, and all codes into s_act (16-byte loads from L2,
+  // up to 16 in flight per thread)
+  for (int m = warp; m < M; m += kFdThreads / 32) {
+    int v = 0;
+    for (int i = lane; i < G; i += 32) v += __ldcg(&ctl->cs[i][m]);
+    v = __reduce_add_sync(0xffffffffu, v);
+    if (lane == 0) sh.rs_m[m] = v;
+  }
+  {
+    const int per_row = p.I / 16;
+    const int total = M * per_row;
+    for (int base = threadIdx.x; base < total; base += 16 * kFdThreads) {
+      uint4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = base + u * kFdThreads;
+        if (idx < total)
+          v[u] = ld_cg_u4(p.hq + (size_t)(idx / per_row) * p.I + 16 * (idx % per_row));
+      }
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int idx = base + u * kFdThreads;
+        if (idx < total)
+          *reinterpret_cast<uint4*>(s_act + (size_t)(idx / per_row) * p.sx_i + 16 * (idx % per_row)) = v[u];
+      }
+    }
+  }
+  __syncthreads();
   if (threadIdx.x < M) {
     const int m = threadIdx.x;
     dequant_factor(__ldg(p.gamma_d), sh.s_m[m], sh.fd_hi[m], sh.fd_lo[m]);
@@ -604,27 +765,21 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   }
   for (int i = threadIdx.x; i < 2 * 2 * 32 * 4; i += kFdThreads) sh.red[i] = 0;
   __syncthreads();
-  if (b == 0) {                                      // the codes, for inspection
-    for (int m = 0; m < M; ++m)
-      for (int k = 4 * (int)threadIdx.x; k < p.I; k += 4 * kFdThreads)
-        *reinterpret_cast<uint32_t*>(p.hq + (size_t)m * p.I + k) =
-            *reinterpret_cast<const uint32_t*>(s_act + (size_t)m * p.sx_i + k);
-  }
 
   // ---- P5: down rows of this CTA (warps split K), residual, store
   if (!mbar_wait(&sh.bar_d, 0, nullptr) && lane == 0) sh.ok = 0;
   fd_contract_rows(s_d, p.ldwI, nr, s_act, p.sx_i, p.I, ntile, sh.red);
   __syncthreads();
   if (threadIdx.x < 2 * 2 * 32) {
-    // thread (row tile i, token tile t, lane): rows 16 i + g and 16 i + 8 + g,
-    // tokens 8 t + 2 c + {0, 1}
+    // thread (row tile i, token tile t, lane): slots 2i and 2i + 1 of sub-block
+    // lane / 4, tokens 8 t + 2 (lane % 4) + {0, 1}
     const int idx = threadIdx.x;
     const int i = idx >> 6, t = (idx >> 5) & 1, ln = idx & 31;
     if (t < ntile && sh.ok) {
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const int r = 16 * i + 8 * half + (ln >> 2);
-        if (r >= nr) continue;
+        const int r = fd_contract_row(nr, i, half, ln);
+        if (r < 0) continue;
         const int n = n0 + r;
 #pragma unroll
         for (int e = 0; e < 2; ++e) {

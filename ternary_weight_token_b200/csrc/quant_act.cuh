@@ -510,31 +510,44 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// FWHT prelude, one warp per token row, the row in registers (K = 2^n with
-// VEC * 32 <= K <= 2048).  Lane l holds the 16-byte vectors j = 0 .. J-1 at
-// elements k = VEC * l + 32 * VEC * j + e.  The butterfly stages run in the
-// fixed order h = 1, 2, 4, ...: h < VEC inside a vector, VEC <= h < 32 VEC
-// between lanes (shuffle with lane ^ (h / VEC); the lower partner keeps a + b,
-// the upper a - b, the same fp32 operations as the staged kernel), h >= 32 VEC
-// between a lane's own vectors.  No block barrier anywhere.
-template <int K, bool BF16, bool SILU = false>
+// FWHT prelude with the row in registers (K = 2^n, VEC * 32 * WPR <= K <=
+// 2048), WPR warps per token row (1, 2 or 4; a 128-thread CTA takes 4 / WPR
+// rows at a time).  Warp w of a row holds elements k = KW w + 32 VEC j +
+// VEC l + e (KW = K / WPR, lane l, vector j, element e of a 16-byte vector).
+// The butterfly stages run in the fixed order h = 1, 2, 4, ...: h < VEC
+// inside a vector, VEC <= h < 32 VEC between lanes (shuffle with lane ^
+// (h / VEC); the lower partner keeps a + b, the upper a - b, the same fp32
+// operations as the staged kernel), 32 VEC <= h < KW between a lane's own
+// vectors, and h >= KW between the row's warps through shared memory (each
+// thread reads the WPR values of its position and runs those stages in the
+// same order).  Several warps per row keep more rows in flight and shorten
+// each warp's chain of dependent instructions.
+template <int K, bool BF16, bool SILU = false, int WPR = 1>
 __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
   constexpr int VEC = BF16 ? 8 : 4;
-  constexpr int J = K / (32 * VEC);
-  static_assert(J >= 1 && J * 32 * VEC == K, "row width");
-  const int lane = threadIdx.x & 31;
-  const int warp_g = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int nwarps = gridDim.x * 4;
+  constexpr int KW = K / WPR;
+  constexpr int J = KW / (32 * VEC);
+  constexpr int RPC = 4 / WPR;                      // rows per CTA at a time
+  static_assert(WPR == 1 || WPR == 2 || WPR == 4, "warps per row");
+  static_assert(J >= 1 && J * 32 * VEC * WPR == K, "row width");
+  __shared__ float xw[WPR > 1 ? 4 * KW : 1];        // [warp][KW] for the cross-warp stages
+  __shared__ float red_f[4];
+  __shared__ int red_i[4];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int rg = warp / WPR, wr = warp - rg * WPR;  // row slot of the CTA, warp within the row
   grid_launch_dependents();       // launched with programmatic dependent launch:
   grid_dependency_wait();         // no global access before the preceding grid completed
-  for (int m = warp_g; m < p.M; m += nwarps) {
+  for (int m0 = blockIdx.x * RPC; m0 < p.M; m0 += gridDim.x * RPC) {   // same trip count CTA-wide
+    const int m = m0 + rg;
+    const bool row = m < p.M;
+    const size_t rbase = (size_t)(row ? m : 0) * K + (size_t)wr * KW;
     float v[J][VEC];
     if (BF16) {
       const uint4* src = reinterpret_cast<const uint4*>(
-          reinterpret_cast<const uint16_t*>(p.X) + (size_t)m * K) + lane;
+          reinterpret_cast<const uint16_t*>(p.X) + rbase) + lane;
 #pragma unroll
       for (int j = 0; j < J; ++j) {
-        const uint4 u = ld_stream_v4(src + 32 * j);
+        const uint4 u = row ? ld_stream_v4(src + 32 * j) : make_uint4(0u, 0u, 0u, 0u);
         const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -544,10 +557,10 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
       }
     } else {
       const float4* src = reinterpret_cast<const float4*>(
-          reinterpret_cast<const float*>(p.X) + (size_t)m * K) + lane;
+          reinterpret_cast<const float*>(p.X) + rbase) + lane;
 #pragma unroll
       for (int j = 0; j < J; ++j) {
-        const uint4 u = ld_stream_v4(src + 32 * j);
+        const uint4 u = row ? ld_stream_v4(src + 32 * j) : make_uint4(0u, 0u, 0u, 0u);
         v[j][0] = __uint_as_float(u.x); v[j][1] = __uint_as_float(u.y);
         v[j][2] = __uint_as_float(u.z); v[j][3] = __uint_as_float(u.w);
       }
@@ -583,7 +596,7 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
           v[j][e] = upper ? __fsub_rn(other, mine) : __fadd_rn(mine, other);
         }
     }
-    // h >= 32 VEC: between this lane's vectors
+    // 32 VEC <= h < KW: between this lane's vectors
 #pragma unroll
     for (int hj = 1; hj < J; hj <<= 1)
 #pragma unroll
@@ -595,6 +608,32 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
             v[j][e] = __fadd_rn(a, b);
             v[j + hj][e] = __fsub_rn(a, b);
           }
+    // h >= KW: between the row's warps
+    if constexpr (WPR > 1) {
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) xw[warp * KW + 32 * VEC * j + VEC * lane + e] = v[j][e];
+      __syncthreads();
+#pragma unroll
+      for (int j = 0; j < J; ++j)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          float t[WPR];
+#pragma unroll
+          for (int w = 0; w < WPR; ++w) t[w] = xw[(rg * WPR + w) * KW + 32 * VEC * j + VEC * lane + e];
+#pragma unroll
+          for (int hb = 1; hb < WPR; hb <<= 1)
+#pragma unroll
+            for (int w = 0; w < WPR; ++w)
+              if ((w & hb) == 0) {
+                const float a = t[w], b = t[w + hb];
+                t[w] = __fadd_rn(a, b);
+                t[w + hb] = __fsub_rn(a, b);
+              }
+          v[j][e] = t[wr];
+        }
+    }
     // normalisation, absmax, codes
     float amax = 0.0f;
 #pragma unroll
@@ -606,11 +645,17 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
       }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    if constexpr (WPR > 1) {
+      if (lane == 0) red_f[warp] = amax;
+      __syncthreads();
+#pragma unroll
+      for (int w = 0; w < WPR; ++w) amax = fmaxf(amax, red_f[rg * WPR + w]);
+    }
     float s = __fdiv_rn(127.0f, amax);
     const bool zero_row = (amax == 0.0f) || isinf(s);
     if (zero_row) s = 1.0f;
     int rsum = 0;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(p.Xq + (size_t)m * K);
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.Xq + rbase);
 #pragma unroll
     for (int j = 0; j < J; ++j)
 #pragma unroll
@@ -621,10 +666,21 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
                           __fmul_rn(v[j][e + 2], s), __fmul_rn(v[j][e + 3], s));
           rsum = __dp4a((int)w, 0x01010101, rsum);
         }
-        dst[(VEC * lane + 32 * VEC * j + e) / 4] = w;
+        if (row) dst[(VEC * lane + 32 * VEC * j + e) / 4] = w;
       }
     rsum = __reduce_add_sync(0xffffffffu, rsum);
-    if (lane == 0) {
+    if constexpr (WPR > 1) {
+      if (lane == 0) red_i[warp] = rsum;
+      __syncthreads();
+      if (row && wr == 0 && lane == 0) {
+        int t = 0;
+#pragma unroll
+        for (int w = 0; w < WPR; ++w) t += red_i[rg * WPR + w];
+        p.scale[m] = s;
+        if (p.rowsum != nullptr) p.rowsum[m] = t;
+      }
+      __syncthreads();             // xw / red_* are rewritten by the next rows
+    } else if (row && lane == 0) {
       p.scale[m] = s;
       if (p.rowsum != nullptr) p.rowsum[m] = rsum;
     }
