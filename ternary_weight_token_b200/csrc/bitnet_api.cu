@@ -22,7 +22,6 @@
 #include "ffn_decode.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
-#include "gemv_mma.cuh"
 #include "gemv_tc.cuh"
 #include "pack_weights.cuh"
 #include "quant_act.cuh"
@@ -516,45 +515,6 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   const size_t smem = (size_t)(p.M <= 1 ? 1 : 2) * (size_t)p.K;
   if (p.M <= 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
   return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
-}
-
-// Decode for 1..16 tokens on short-lived CTAs (gemv_mma.cuh): 16 * RT weight
-// rows per CTA, RT chosen so the grid covers the SMs about twice.  Returns
-// BITNET_ERR_UNSUPPORTED when K is not a multiple of 32 or the staged rows
-// do not fit shared memory.
-template <int RT, int NTILE>
-int launch_gemv_mma_rt(const LinearParams& p, cudaStream_t st, const DeviceInfo& di) {
-  GmParams gp;
-  gp.lp = p;
-  gp.lp.flags &= ~LAUNCH_PDL;                  // keeps LAUNCH_PDL_INPUTS for the kernel
-  gp.rows_per_cta = 16 * RT;
-  gp.sw = p.ldw;
-  gp.sx = p.K;
-  gp.off_x = (int)align128((size_t)16 * RT * gp.sw);
-  const size_t smem = (size_t)gp.off_x + (size_t)p.M * gp.sx + 128;
-  if (smem > (size_t)di.max_smem_optin - 4096) return BITNET_ERR_UNSUPPORTED;
-  auto kern = gemv_mma_kernel<RT, NTILE>;
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  const int grid = (p.N + 16 * RT - 1) / (16 * RT);
-  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(kGmThreads), smem, st,
-                       gp);
-}
-
-int launch_gemv_mma(const LinearParams& p, cudaStream_t st) {
-  if (p.M < 1 || p.M > 16 || p.K % 32 != 0) return BITNET_ERR_UNSUPPORTED;
-  DeviceInfo di;
-  if (int rc = device_info(di)) return rc;
-  const int tiles = (p.N + 15) / 16;
-  int rt = 1;
-  while (rt < 4 && (tiles + 2 * rt - 1) / (2 * rt) >= 2 * di.sms) rt *= 2;
-  if (p.M <= 8) {
-    if (rt == 1) return launch_gemv_mma_rt<1, 1>(p, st, di);
-    if (rt == 2) return launch_gemv_mma_rt<2, 1>(p, st, di);
-    return launch_gemv_mma_rt<4, 1>(p, st, di);
-  }
-  if (rt == 1) return launch_gemv_mma_rt<1, 2>(p, st, di);
-  if (rt == 2) return launch_gemv_mma_rt<2, 2>(p, st, di);
-  return launch_gemv_mma_rt<4, 2>(p, st, di);
 }
 
 // Projection i of a call as a call of its own.
