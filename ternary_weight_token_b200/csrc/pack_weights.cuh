@@ -194,6 +194,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const void* W, int N
 // smaller than L2.
 constexpr int kPackFusedThreads = 512;
 constexpr int kPackMaxGrid = 1024;        // partial / flag slots in the workspace
+constexpr int kPackWords = 4;             // output words per thread per batch (pass 2)
 
 template <bool BF16>
 __global__ void __launch_bounds__(kPackFusedThreads) pack_fused_kernel(
@@ -271,8 +272,16 @@ __global__ void __launch_bounds__(kPackFusedThreads) pack_fused_kernel(
   // adds partials l, l + 32, ... in turn, then a fixed xor tree)
   const bool ok = grid_exchange(flags, epoch, &xok);
   if (threadIdx.x < 32) {
+    // every partial of a lane loaded before any is added (one L2 round trip)
+    double pv[kPackMaxGrid / 32];
+#pragma unroll
+    for (int j = 0; j < kPackMaxGrid / 32; ++j) {
+      const int i = (int)threadIdx.x + 32 * j;
+      pv[j] = i < (int)gridDim.x ? __ldcg(partials + i) : 0.0;
+    }
     double v = 0.0;
-    for (int i = threadIdx.x; i < (int)gridDim.x; i += 32) v += __ldcg(partials + i);
+#pragma unroll
+    for (int j = 0; j < kPackMaxGrid / 32; ++j) v += pv[j];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (threadIdx.x == 0) {
@@ -283,48 +292,74 @@ __global__ void __launch_bounds__(kPackFusedThreads) pack_fused_kernel(
   }
   __syncthreads();
   if (!ok) return;
-  // pass 2: codes, one thread per 32-bit word of the packed layout
+  // pass 2: codes, one thread per 32-bit word of the packed layout; each
+  // thread takes kPackWords words of the grid-stride sequence at a time, all
+  // their loads (from L2: pass 1 just read them) issued before any is used
   const float g = s_gamma;
   const float thr = ternary_threshold(g);
   const int words_per_row = ldw / 4;
-  const long long total = (long long)N * words_per_row;
-  for (long long idx = t0; idx < total; idx += stride) {
-    const int n = (int)(idx / words_per_row);
-    const int wi = (int)(idx % words_per_row);
-    const int k0 = 16 * wi;
-    uint32_t word = 0x55555555u;                    // padding: code 1 everywhere
-    if (k0 < K) {
-      float w[16];
-      if (BF16) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            reinterpret_cast<const uint16_t*>(W) + (size_t)n * K + k0);
-        const uint4 a = ld_stream_v4(src), b = ld_stream_v4(src + 1);
-        const uint32_t u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  constexpr int VPW = BF16 ? 2 : 4;               // 16-byte loads per word
+  // word index t0 + j * stride as (row, word) without a division per word:
+  // one division here, then steps of (stride / wpr, stride % wpr) with a carry
+  const long long st_rows = stride / words_per_row;
+  const int st_words = (int)(stride - st_rows * words_per_row);
+  long long cur_n = t0 / words_per_row;
+  int cur_w = (int)(t0 - cur_n * words_per_row);
+  while (cur_n < N) {
+    uint4 raw[kPackWords][VPW];
+    int rown[kPackWords], wordi[kPackWords];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          w[2 * j] = bf16_bits_to_f32(u[j] & 0xffffu);
-          w[2 * j + 1] = bf16_bits_to_f32(u[j] >> 16);
+    for (int u = 0; u < kPackWords; ++u) {
+      rown[u] = -1;
+      if (cur_n < N) {
+        const int n = (int)cur_n;
+        const int wi = cur_w;
+        rown[u] = n;
+        wordi[u] = wi;
+        cur_n += st_rows;
+        cur_w += st_words;
+        if (cur_w >= words_per_row) {
+          cur_w -= words_per_row;
+          ++cur_n;
         }
-      } else {
-        const float4* src = reinterpret_cast<const float4*>(
-            reinterpret_cast<const float*>(W) + (size_t)n * K + k0);
-        uint4 v[4];
+        if (16 * wi < K) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              reinterpret_cast<const uint8_t*>(W) + ((size_t)n * K + 16 * (size_t)wi) * (BF16 ? 2 : 4));
 #pragma unroll
-        for (int j = 0; j < 4; ++j) v[j] = ld_stream_v4(src + j);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          w[4 * j] = __uint_as_float(v[j].x); w[4 * j + 1] = __uint_as_float(v[j].y);
-          w[4 * j + 2] = __uint_as_float(v[j].z); w[4 * j + 3] = __uint_as_float(v[j].w);
+          for (int j = 0; j < VPW; ++j) raw[u][j] = ld_stream_v4(src + j);
         }
       }
-      word = 0;
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j)
-          word |= ternary_code(w[4 * i + j], g, thr) << (8 * j + 2 * i);
     }
-    reinterpret_cast<uint32_t*>(packed + (size_t)n * ldw)[wi] = word;
+#pragma unroll
+    for (int u = 0; u < kPackWords; ++u) {
+      if (rown[u] < 0) continue;
+      uint32_t word = 0x55555555u;                  // padding: code 1 everywhere
+      if (16 * wordi[u] < K) {
+        float w[16];
+        if (BF16) {
+          const uint32_t v[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                 raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            w[2 * j] = bf16_bits_to_f32(v[j] & 0xffffu);
+            w[2 * j + 1] = bf16_bits_to_f32(v[j] >> 16);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            w[4 * j] = __uint_as_float(raw[u][j].x); w[4 * j + 1] = __uint_as_float(raw[u][j].y);
+            w[4 * j + 2] = __uint_as_float(raw[u][j].z); w[4 * j + 3] = __uint_as_float(raw[u][j].w);
+          }
+        }
+        word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            word |= ternary_code(w[4 * i + j], g, thr) << (8 * j + 2 * i);
+      }
+      reinterpret_cast<uint32_t*>(packed + (size_t)rown[u] * ldw)[wordi[u]] = word;
+    }
   }
 }
 
