@@ -397,6 +397,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
 std::atomic<uint64_t> g_dec_attr_set{0};
 
 using TcPlain = TcConfig<128, 256, 4, false>;
+using TcPlain96 = TcConfig<96, 256, 4, false>;     // 96-token tiles (tile quantisation, below)
 using TcSilu = TcConfig<128, 256, 4, false, true>;
 using TcGlu = TcConfig<128, 256, 4, true>;
 
@@ -528,6 +529,24 @@ LinearParams segment_params(const LinearParams& p, int i) {
   return q;
 }
 
+// The persistent GEMM runs ceil(tiles / SMs) waves of tiles.  A tile's time is
+// a fixed part (converting its 128 weight rows, the epilogue's setup) plus a
+// part proportional to its tokens; timing 6912 -> 2560 at 4096 tokens with
+// 128- and 96-token tiles (5 and 6 waves: 61.8 and 68.5 us) puts the fixed
+// part at ~270 tokens' worth.  96-token tiles are taken when
+// waves x (tokens + 270) is clearly smaller: a last wave of 128-token tiles
+// that would leave most SMs idle, e.g. 2048 tokens x 2560 rows (320 tiles,
+// 3 waves; 440 tiles of 96, still 3 waves).
+bool token_tile_96(int M, int N) {
+  DeviceInfo di;
+  if (device_info(di) != BITNET_OK || di.sms <= 0) return false;
+  auto cost = [&](int bn) {
+    const long long tiles = (long long)((M + bn - 1) / bn) * ((N + 127) / 128);
+    return ((tiles + di.sms - 1) / di.sms) * (bn + 270);
+  };
+  return cost(96) * 100 < cost(128) * 97;
+}
+
 int launch_linear(const LinearParams& p, cudaStream_t st) {
   // 1-2 tokens: the dp4a streaming kernel (measured faster than the cluster
   // tensor-core path there; from 4 tokens on, its dp4a work and shared-memory
@@ -548,6 +567,8 @@ int launch_linear(const LinearParams& p, cudaStream_t st) {
       rc = launch_gemv(q, st);
     } else if (q.flags & EPI_SILU) {
       rc = launch_tc_cfg<TcSilu>(q, nullptr, nullptr, st);
+    } else if (token_tile_96(q.M, q.N)) {
+      rc = launch_tc_cfg<TcPlain96>(q, nullptr, nullptr, st);
     } else {
       rc = launch_tc_cfg<TcPlain>(q, nullptr, nullptr, st);
     }
