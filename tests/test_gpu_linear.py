@@ -178,13 +178,16 @@ def test_decode_with_programmatic_dependent_launch():
         assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="pdl step")
 
 
-def test_decode_independent_projections_overlap():
+@pytest.mark.parametrize("M", [1, 3, 4, 16])
+def test_decode_independent_projections_overlap(M):
     """BITNET_LAUNCH_PDL_INPUTS: consecutive decode calls that read one set of
     activation codes (as q/k/v or gate/up do) may run everything but their
     output stores under the preceding call.  Distinct weights, a shared
     output written by every call (the last call's values must remain) and
-    distinct outputs, all bit-exact against the oracle (int32)."""
-    M, K = 16, 2560
+    distinct outputs, all bit-exact against the oracle (int32); one fp32
+    output per round against the oracle's dequantisation.  One token runs the
+    streaming dp4a kernel, 3-16 the cluster tensor-core decode kernel."""
+    K = 2560
     rng_w, rng_x = synthetic.streams(43, 2)
     X = synthetic.activations(rng_x, M, K)
     q, s, rs = oracle.quant_act(X)
@@ -198,6 +201,7 @@ def test_decode_independent_projections_overlap():
     shared = torch.empty((M, 6912), dtype=torch.int32, device="cuda")
     outs = []
     flags = bn.BITNET_I32 | bn.BITNET_LAUNCH_PDL_INPUTS
+    f32_outs = []
     for rnd in range(3):
         for N, T, Pd, gd in packs:
             Y = torch.empty((M, N), dtype=torch.int32, device="cuda")
@@ -205,9 +209,17 @@ def test_decode_independent_projections_overlap():
             if N == 6912:
                 bn.bitnet_linear(qd, sd, rsd, Pd, gd, K, shared, epilogue=flags)
             outs.append((Y, T))
+        N, T, Pd, gd = packs[rnd]
+        Yf = torch.empty((M, N), dtype=torch.float32, device="cuda")
+        bn.bitnet_linear(qd, sd, rsd, Pd, gd, K, Yf,
+                         epilogue=bn.BITNET_F32 | bn.BITNET_LAUNCH_PDL_INPUTS)
+        f32_outs.append((Yf, T, float(gd.cpu()[0])))
     torch.cuda.synchronize()
     for Y, T in outs:
         np.testing.assert_array_equal(Y.cpu().numpy(), oracle.contract(q, T))
+    for Yf, T, g in f32_outs:
+        assert_f32_close(Yf.cpu().numpy(), oracle.dequant(oracle.contract(q, T), s, g),
+                         what="independent f32")
     np.testing.assert_array_equal(shared.cpu().numpy(), oracle.contract(q, packs[-1][1]))
     assert bn.bitnet_check_device_error() == bn.BITNET_OK
 
