@@ -54,7 +54,9 @@ constexpr int kFdThreads = 256;           // 8 warps
 constexpr int kFdMaxSlots = 8;            // rows per gate / up sub-block (<= 64 features per CTA)
 constexpr int kFdMaxGrid = 256;           // partials / flags slots in the control block
 constexpr int kFdRowPad = 16;             // bytes added to every staged code row
-constexpr int kFdRegChunks = 24;          // float4 chunks per thread held in the row quantiser
+constexpr int kFdRegChunks = 8;           // float4 chunks per thread held in the row quantiser
+                                          // (24 held every 1-4-token row at once but made the
+                                          // phase code ~3x longer: 34 vs 29 us per FFN at M = 1)
 
 // Control block of one persistent launch, in the caller's workspace.
 struct FdControl {
@@ -728,7 +730,7 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
     sh.ok = 0;
 
   // every CTA: code sums, and all codes into s_act (16-byte loads from L2,
-  // up to 16 in flight per thread)
+  // four in flight per thread)
   for (int m = warp; m < M; m += kFdThreads / 32) {
     int v = 0;
     for (int i = lane; i < G; i += 32) v += __ldcg(&ctl->cs[i][m]);
@@ -738,16 +740,16 @@ __global__ void __launch_bounds__(kFdThreads, 1) ffn_decode_kernel(FfnDecodePara
   {
     const int per_row = p.I / 16;
     const int total = M * per_row;
-    for (int base = threadIdx.x; base < total; base += 16 * kFdThreads) {
-      uint4 v[16];
+    for (int base = threadIdx.x; base < total; base += 4 * kFdThreads) {
+      uint4 v[4];
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 4; ++u) {
         const int idx = base + u * kFdThreads;
         if (idx < total)
           v[u] = ld_cg_u4(p.hq + (size_t)(idx / per_row) * p.I + 16 * (idx % per_row));
       }
 #pragma unroll
-      for (int u = 0; u < 16; ++u) {
+      for (int u = 0; u < 4; ++u) {
         const int idx = base + u * kFdThreads;
         if (idx < total)
           *reinterpret_cast<uint4*>(s_act + (size_t)(idx / per_row) * p.sx_i + 16 * (idx % per_row)) = v[u];
