@@ -194,8 +194,9 @@ BITNET_API int bitnet_quant_act(const void *X, int x_dtype, int M, int K,
  *             y = fp32( acc * gamma / s[m] ) (evaluated in fp64, rounded once),
  *             then the optional SiLU / residual add in fp32, then the cast.
  *   residual  [M][N] of Y's type when BITNET_EPI_RESIDUAL is set, else NULL.
- * M <= 2 (K a multiple of 64) runs the dp4a streaming GEMV, M <= 16 the cluster
- * tensor-core GEMV (both HBM-bound), larger M the tcgen05 GEMM.
+ * M <= 2 (K a multiple of 64), or M <= 8 with N K <= 2^20, runs the dp4a streaming
+ * GEMV, M <= 16 otherwise the cluster tensor-core GEMV (both HBM-bound), larger M
+ * the tcgen05 GEMM.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 BITNET_API int bitnet_linear(const int8_t *Xq, const float *x_scale, const int32_t *x_rowsum,
                   const uint8_t *packed, const float *gamma,

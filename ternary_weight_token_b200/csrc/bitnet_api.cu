@@ -512,10 +512,13 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   int R = (p.N + di.sms * warps - 1) / (di.sms * warps);
   if (R > 8) R = 8;
   while (R > 1 && R * C > 32 * 8) --R;
+  const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : 8;
+  if (mt == 8 && R > 4) R = 4;                   // lane r * MT + m holds (row, token): R MT <= 32
   const int grid = (p.N + warps * R - 1) / (warps * R);
-  const size_t smem = (size_t)(p.M <= 1 ? 1 : 2) * (size_t)p.K;
-  if (p.M <= 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
-  return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
+  const size_t smem = (size_t)mt * (size_t)p.K;
+  if (mt == 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
+  if (mt == 2) return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
+  return launch_stream_mt<8, kStreamThreads>(p, R, grid, smem, st);
 }
 
 // Projection i of a call as a call of its own.
@@ -550,9 +553,14 @@ bool token_tile_96(int M, int N) {
 int launch_linear(const LinearParams& p, cudaStream_t st) {
   // 1-2 tokens: the dp4a streaming kernel (measured faster than the cluster
   // tensor-core path there; from 4 tokens on, its dp4a work and shared-memory
-  // reads sit on the critical path of dependent calls).  Both decode kernels
-  // run every projection of the call in one launch.
-  if (p.M <= 2 && p.K % 64 == 0 && p.ldw / 16 <= 32 * 8) return launch_gemv_stream(p, st);
+  // reads sit on the critical path of dependent calls on the 2B shapes).  Up
+  // to 8 tokens on small weight matrices (<= 2^20 weights, e.g. 256 x 512):
+  // the streaming kernel too, whose short CTAs beat the cluster path's TMEM
+  // set-up and reduction there (6.2 -> 4.4 us per quantise + project pair).
+  // Both decode kernels run every projection of the call in one launch.
+  const bool stream_ok = p.K % 64 == 0 && p.ldw / 16 <= 32 * 8;
+  if (stream_ok && (p.M <= 2 || (p.M <= 8 && (long long)p.N * p.K <= (1ll << 20))))
+    return launch_gemv_stream(p, st);
   if (p.M <= 16) {
     const int rc = launch_gemv_tc(p, st);
     if (rc != BITNET_ERR_UNSUPPORTED) return rc;

@@ -66,6 +66,26 @@ def test_persistent_gemm_every_epilogue_bit_exact(M, K, N):
     assert_bf16_matches(gotr, (R + y).astype(np.float32), what="bf16 residual")
 
 
+@pytest.mark.parametrize("M", [3, 5, 8])
+@pytest.mark.parametrize("K,N", [(256, 512), (512, 300), (64, 77), (1024, 1024)])
+def test_small_matrix_decode_every_epilogue(M, K, N):
+    """3-8 tokens on weight matrices of at most 2^20 weights run the streaming
+    dp4a kernel with an 8-token instantiation (ragged N, tokens short of 8):
+    int32 bit-exact, fp32 / bf16 / residual / SiLU against the oracle."""
+    X, g, T, P, q, s, rs = _case(M, K, N, seed=M * 7 + K + N)
+    acc = oracle.contract(q, T)
+    np.testing.assert_array_equal(gpu_linear(q, s, rs, P, g, K, N, out=torch.int32), acc)
+    y = oracle.dequant(acc, s, g)
+    assert_f32_close(gpu_linear(q, s, rs, P, g, K, N, out=torch.float32), y, what="f32")
+    assert_bf16_matches(gpu_linear(q, s, rs, P, g, K, N, out=torch.bfloat16), y, what="bf16")
+    R = synthetic.activations(np.random.default_rng(N + M), M, N)
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.float32, flags=bn.BITNET_EPI_RESIDUAL,
+                     residual=R)
+    assert_f32_close(got, (R + y).astype(np.float32), what="residual")
+    got = gpu_linear(q, s, rs, P, g, K, N, out=torch.float32, flags=bn.BITNET_EPI_SILU)
+    assert_f32_close(got, oracle.silu(y), what="silu")
+
+
 @pytest.mark.parametrize("M,K,N", [(1, 2560, 2560), (16, 6912, 300), (300, 2560, 300),
                                    (200, 512, 2048)])
 def test_linear_f32_and_bf16(M, K, N):
