@@ -338,8 +338,9 @@ BITNET_API int bitnet_debug_wait_timeout(unsigned timeout_us, bitnet_stream_t st
 
 /* Empty the host-side cache of TMA tensor descriptors and forget the
  * per-context state the library keeps: the device address of the
- * no-allocation FFN scratch and which devices have the decode kernel's
- * shared-memory attribute set.  The descriptor cache is keyed by device,
+ * no-allocation FFN scratch, the kernels' shared-memory attributes it has set
+ * and the occupancies it has looked up (per device, so that warm calls make
+ * no driver query).  The descriptor cache is keyed by device,
  * pointer, shape, box and swizzle, so it stays correct when an address is
  * reused; it holds at most 16384 descriptors (it starts over when full).
  * After cudaDeviceReset (which ends the context those addresses and

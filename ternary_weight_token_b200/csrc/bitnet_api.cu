@@ -12,9 +12,12 @@
 #include <cstdio>
 #include <cstring>
 #include <chrono>
+#include <map>
 #include <mutex>
 #include <random>
 #include <string>
+#include <tuple>
+#include <utility>
 #include <unordered_map>
 
 #include "../../include/bitnet.h"
@@ -79,6 +82,47 @@ int device_info(DeviceInfo& out) {
     it = cache.emplace(dev, di).first;
   }
   out = it->second;
+  return BITNET_OK;
+}
+
+// Kernel attributes belong to each device's context: the dynamic
+// shared-memory limit set for a kernel, and the occupancy found for a launch
+// shape, are cached per device (so a call makes no driver query once warm)
+// and cleared by bitnet_release_cache.
+std::mutex g_attr_mu;
+std::map<std::pair<int, const void*>, size_t> g_smem_set;
+std::map<std::tuple<int, const void*, int, size_t>, int> g_occupancy;
+
+int set_smem_attr(const void* fn, size_t bytes) {
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    auto it = g_smem_set.find({dev, fn});
+    if (it != g_smem_set.end() && it->second >= bytes) return BITNET_OK;
+  }
+  BN_CHECK_CUDA(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes));
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  size_t& v = g_smem_set[{dev, fn}];
+  if (bytes > v) v = bytes;
+  return BITNET_OK;
+}
+
+int occupancy(int& per_sm, const void* fn, int threads, size_t smem) {
+  int dev = 0;
+  BN_CHECK_CUDA(cudaGetDevice(&dev));
+  const auto key = std::make_tuple(dev, fn, threads, smem);
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    auto it = g_occupancy.find(key);
+    if (it != g_occupancy.end()) {
+      per_sm = it->second;
+      return BITNET_OK;
+    }
+  }
+  BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem));
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  g_occupancy[key] = per_sm;
   return BITNET_OK;
 }
 
@@ -282,7 +326,7 @@ int launch_quant(const void* X, bool bf16, int M, int K, int prelude, const floa
   void (*kern)(QuantParams) =
       silu ? (bf16 ? quant_act_kernel<PRE_SILU_FWHT, true> : quant_act_kernel<PRE_SILU_FWHT, false>)
            : (bf16 ? quant_act_kernel<PRE_FWHT, true> : quant_act_kernel<PRE_FWHT, false>);
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   return launch_pdl(kern, dim3(grid), dim3(threads), smem, st, p);
 }
 
@@ -302,9 +346,9 @@ int launch_gemv(const LinearParams& p, cudaStream_t st) {
     case 8: kern = gemv_kernel<8>; break;
     default: kern = gemv_kernel<16>; break;
   }
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   int per_sm = 0;
-  BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem));
+  if (int rc = occupancy(per_sm, (const void*)kern, kGemvThreads, smem)) return rc;
   if (per_sm < 1) per_sm = 1;
   const int rows_per_cta = (kGemvThreads / 32) * kGemvRows;
   const int need = (p.N + rows_per_cta - 1) / rows_per_cta;
@@ -386,7 +430,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   if (smem < one_per_sm) smem = one_per_sm;
   if (smem > (size_t)di.max_smem_optin) smem = di.max_smem_optin;
   auto kern = gemm_tc_kernel<C>;
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   const int grid = p.num_tiles < di.sms ? p.num_tiles : di.sms;
   return launch_pdl(kern, dim3(grid), dim3(C::THREADS), smem, st, mx, mw0, mw1, my, mr, p);
 }
@@ -494,7 +538,7 @@ int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaSt
     case 7: kern = gemv_stream_kernel<MT, 7, 8, NT>; break;
     default: kern = gemv_stream_kernel<MT, 8, 8, NT>; break;
   }
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   LinearParams q = p;
   q.flags &= ~LAUNCH_PDL;
   return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(NT), smem, st, q);
@@ -630,9 +674,9 @@ int launch_ffn_decode(FfnDecodeParams p, cudaStream_t st, bool tail = false) {
       (size_t)p.off_act + (size_t)p.mpad * (size_t)std::max(p.sx_h, p.sx_i) + 128;
   if (smem + sizeof(FfnDecodeShared) + 1024 > (size_t)di.max_smem_optin) return BITNET_ERR_UNSUPPORTED;
   void (*kern)(FfnDecodeParams) = tail ? ffn_decode_kernel<true> : ffn_decode_kernel<false>;
-  BN_CHECK_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   int per_sm = 0;
-  BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFdThreads, smem));
+  if (int rc = occupancy(per_sm, (const void*)kern, kFdThreads, smem)) return rc;
   if (per_sm < 1) return BITNET_ERR_UNSUPPORTED;
   p.epoch = next_epoch();
   cudaLaunchConfig_t cfg = {};
@@ -728,7 +772,7 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
                unsigned long long, float*, uint8_t*) =
         bf16 ? pack_fused_kernel<true> : pack_fused_kernel<false>;
     int per_sm = 0;
-    BN_CHECK_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kf, kPackFusedThreads, 0));
+    if (int rc = occupancy(per_sm, (const void*)kf, kPackFusedThreads, 0)) return rc;
     const int G = std::min(std::min(per_sm, 2) * di.sms, kPackMaxGrid);
     if (G >= di.sms) {
       unsigned long long* flags = reinterpret_cast<unsigned long long*>(partials + kPackMaxGrid);
@@ -1128,6 +1172,11 @@ void bitnet_release_cache(void) {
     for (int d = 0; d < kMaxDevices; ++d) g_noalloc_ptr[d] = nullptr;
   }
   g_dec_attr_set.store(0, std::memory_order_release);
+  {
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    g_smem_set.clear();
+    g_occupancy.clear();
+  }
 }
 
 const char* bitnet_version(void) { return "bitnet-b200 0.1.0 (sm_100a)"; }
