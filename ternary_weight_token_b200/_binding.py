@@ -90,8 +90,13 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+_RAW_STREAM = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream):
     if stream is None:
+        if _RAW_STREAM is not None:          # the current stream's handle, without a Stream object
+            return ctypes.c_void_p(_RAW_STREAM(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
 
