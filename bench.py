@@ -401,7 +401,10 @@ class Prefill:
                                 prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
             if gemm_events is not None:
                 gemm_events[i][0].record()
-            bn.bitnet_linear(sh["q"], sh["s"], sh["rs"], sh["P"], sh["g"], sh["K"], sh["Y"])
+            # the weights are constant: the GEMM may load its first weight tiles
+            # while the quantiser runs
+            bn.bitnet_linear(sh["q"], sh["s"], sh["rs"], sh["P"], sh["g"], sh["K"], sh["Y"],
+                             epilogue=bn.BITNET_BF16 | bn.BITNET_LAUNCH_PDL)
             if gemm_events is not None:
                 gemm_events[i][1].record()
 
@@ -438,7 +441,7 @@ class Prefill:
                 bn.bitnet_quant_act(sh["X"][sl], sh["q"][sl], sh["s"][sl], sh["rs"][sl],
                                     prelude=bn.BITNET_PRELUDE_RMSNORM, eps=1e-5)
                 bn.bitnet_linear(sh["q"][sl], sh["s"][sl], sh["rs"][sl], sh["P"], sh["g"],
-                                 sh["K"], sh["Y"][sl])
+                                 sh["K"], sh["Y"][sl], epilogue=bn.BITNET_BF16 | bn.BITNET_LAUNCH_PDL)
                 done = torch.cuda.Event()
                 done.record(main)
                 self.copy_out.wait_event(done)

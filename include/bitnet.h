@@ -97,8 +97,9 @@ extern "C" {
  * and stream its packed weights early; activation codes, scales, code sums,
  * gamma, residual and Y are touched only after that work has completed.  Set
  * it only when the preceding work does not write the packed weights, e.g. in
- * a decode loop over static weights.  Ignored for M > 16 (the prefill GEMM
- * always uses the dependent launch, without early weight reads). */
+ * a decode loop over static weights.  For M > 16 (the prefill GEMM, always a
+ * dependent launch) it lets the GEMM load its first weight tiles before the
+ * preceding work has completed. */
 #define BITNET_LAUNCH_PDL     0x100
 /* Stronger launch hint for the decode path (implies BITNET_LAUNCH_PDL): the
  * preceding work on the stream writes none of this call's inputs (packed

@@ -421,6 +421,7 @@ int launch_tc_cfg(const LinearParams& lp, const uint8_t* W1, const float* gamma1
   const int tiles_m = (lp.M + C::BN - 1) / C::BN;
   p.num_tiles = p.tiles_n * tiles_m;
 
+  p.w_early = lp.w_early;
   p.xs = lp.xs; p.xrs = lp.xrs; p.gamma0 = lp.gamma; p.gamma1 = gamma1;
   p.Y = lp.Y; p.resid = lp.resid; p.out_type = lp.out_type; p.flags = lp.flags;
   // One CTA per SM: request enough shared memory that two never co-reside
@@ -891,7 +892,10 @@ int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsu
   p.Y = Y; p.out_type = epilogue & BITNET_EPI_TYPE_MASK;
   p.flags = epilogue & ~BITNET_EPI_TYPE_MASK; p.resid = residual;
   if (p.flags & LAUNCH_PDL_INPUTS) p.flags |= LAUNCH_PDL;
-  if (M > 16) p.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
+  if (M > 16) {
+    p.w_early = (p.flags & LAUNCH_PDL) ? 1 : 0;
+    p.flags &= ~(LAUNCH_PDL | LAUNCH_PDL_INPUTS);
+  }
   single_segment(p);
   return launch_linear(p, reinterpret_cast<cudaStream_t>(stream));
 }
@@ -1021,6 +1025,10 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
   p2.Xq = hq; p2.xs = hs; p2.xrs = hrs; p2.W = W_down; p2.gamma = gamma_down;
   p2.M = M; p2.N = H; p2.K = I; p2.ldw = (int)bitnet_packed_row_bytes(I);
   p2.Y = Y; p2.out_type = y_dtype == BITNET_BF16 ? OUT_BF16 : OUT_F32;
+  // each GEMM below follows this call's own quantiser, which writes no
+  // weights and lets it launch only after everything before it completed
+  p1.w_early = 1;
+  p2.w_early = 1;
   single_segment(p1);
   single_segment(p2);
 

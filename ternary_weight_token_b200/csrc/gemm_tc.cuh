@@ -98,6 +98,8 @@ struct TcParams {
   int flags;
   int tma_out;                // 1: output written through the TMA map tm_y
   int tma_res;                // 1: bf16 residual read through the TMA map tm_r
+  int w_early;                // 1: the preceding work does not write the packed weights:
+                              // the first stages' weight tiles load before the dependency wait
 };
 
 __device__ __forceinline__ int out_elem_bytes(int out_type) { return out_type == OUT_BF16 ? 2 : 4; }
@@ -166,9 +168,10 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   // Launched with programmatic dependent launch: the setup above touches no
-  // global memory; everything below runs after the preceding grid completed.
+  // global memory; everything below runs after the preceding grid completed,
+  // except (w_early) the producer's loads of the first stages' weight tiles.
   grid_launch_dependents();
-  grid_dependency_wait();
+  if (!(p.w_early && warp == 0)) grid_dependency_wait();
   const uint32_t tbase = *tmem_slot;
   const uint32_t a_col0 = 2 * C::ACC_COLS;
 
@@ -176,9 +179,37 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // ------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t it = 0;
+      // w_early: the first tile's first stages (fresh barriers: no empty wait)
+      // get their weight tiles before the dependency wait and their
+      // activation tiles after it
+      int pre = 0;
+      if (p.w_early && (int)blockIdx.x < p.num_tiles) {
+        const int tn = (int)blockIdx.x % p.tiles_n, tm = (int)blockIdx.x / p.tiles_n;
+        pre = p.num_kb < C::STAGES ? p.num_kb : C::STAGES;
+        for (int kb = 0; kb < pre; ++kb) {
+          mbar_arrive_expect_tx(&full[kb], C::TX_BYTES);
+          if (C::GLU) {
+            tma_load_2d(sw + kb * C::W_STAGE, &tm_w0, &full[kb], kb * (C::BK / 4), tn * C::TILE_N);
+            tma_load_2d(sw + kb * C::W_STAGE + (C::BM / 2) * (C::BK / 4), &tm_w1, &full[kb],
+                        kb * (C::BK / 4), tn * C::TILE_N);
+          } else {
+            tma_load_2d(sw + kb * C::W_STAGE, &tm_w0, &full[kb], kb * (C::BK / 4), tn * C::BM);
+          }
+        }
+        grid_dependency_wait();
+        for (int kb = 0; kb < pre; ++kb) {
+#pragma unroll
+          for (int xs = 0; xs < C::BK / 128; ++xs)
+            tma_load_2d(sx + kb * C::X_STAGE + xs * C::XSUB, &tm_x, &full[kb],
+                        kb * C::BK + 128 * xs, tm * C::BN);
+        }
+        it = (uint32_t)pre;
+      } else if (p.w_early) {
+        grid_dependency_wait();
+      }
       for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x) {
         const int tn = tile % p.tiles_n, tm = tile / p.tiles_n;
-        for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        for (int kb = tile == (int)blockIdx.x ? pre : 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t st = it % C::STAGES, ph = (it / C::STAGES) & 1u;
           if (!mbar_wait(&empty[st], ph ^ 1u, abort_flag)) goto producer_done;
           mbar_arrive_expect_tx(&full[st], C::TX_BYTES);

@@ -44,6 +44,9 @@ struct LinearParams {
   const uint8_t* seg_W[kMaxSegments];
   const float* seg_gamma[kMaxSegments];
   void* seg_Y[kMaxSegments];
+  // prefill GEMM: the preceding work does not write the packed weights, so
+  // the first stages' weight tiles may load before the dependency wait
+  int w_early = 0;
 };
 
 __host__ __device__ inline void single_segment(LinearParams& p) {

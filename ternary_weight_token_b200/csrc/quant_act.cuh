@@ -151,8 +151,12 @@ __global__ void __launch_bounds__(256) quant_act_kernel(QuantParams p) {
 
   const int K = p.K;
   const int tid = threadIdx.x, nt = blockDim.x;
-  grid_launch_dependents();       // launched with programmatic dependent launch:
-  grid_dependency_wait();         // no global access before the preceding grid completed
+  // launched with programmatic dependent launch: no global access before the
+  // preceding grid completed; the next grid may launch only after that (so a
+  // GEMM behind this kernel that loads its weights early never overlaps work
+  // from before it)
+  grid_dependency_wait();
+  grid_launch_dependents();
   for (int m = blockIdx.x; m < p.M; m += gridDim.x) {
     // 1. stage the row as fp32; the RMS sum of squares is exact per term in fp64
     double ss = 0.0;
@@ -474,8 +478,12 @@ __global__ void __launch_bounds__(NT) quant_act_reg_kernel(QuantParams p) {
   const int K = p.K;
   const int units = BF16 ? K / 8 : K / 4;
   const int row_bytes = K * (BF16 ? 2 : 4);
-  grid_launch_dependents();       // launched with programmatic dependent launch:
-  grid_dependency_wait();         // no global access before the preceding grid completed
+  // launched with programmatic dependent launch: no global access before the
+  // preceding grid completed; the next grid may launch only after that (so a
+  // GEMM behind this kernel that loads its weights early never overlaps work
+  // from before it)
+  grid_dependency_wait();
+  grid_launch_dependents();
   int par = 0;
   for (int m = blockIdx.x; m < p.M; m += gridDim.x, par ^= 1) {
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const char*>(p.X) +
@@ -535,8 +543,12 @@ __global__ void __launch_bounds__(128) quant_fwht_warp_kernel(QuantParams p) {
   __shared__ int red_i[4];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int rg = warp / WPR, wr = warp - rg * WPR;  // row slot of the CTA, warp within the row
-  grid_launch_dependents();       // launched with programmatic dependent launch:
-  grid_dependency_wait();         // no global access before the preceding grid completed
+  // launched with programmatic dependent launch: no global access before the
+  // preceding grid completed; the next grid may launch only after that (so a
+  // GEMM behind this kernel that loads its weights early never overlaps work
+  // from before it)
+  grid_dependency_wait();
+  grid_launch_dependents();
   for (int m0 = blockIdx.x * RPC; m0 < p.M; m0 += gridDim.x * RPC) {   // same trip count CTA-wide
     const int m = m0 + rg;
     const bool row = m < p.M;

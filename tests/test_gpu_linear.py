@@ -173,6 +173,34 @@ def test_full_chain_matches_oracle():
     assert_f32_close(Y.cpu().numpy(), oracle.bitlinear(X, T, g), what="chain")
 
 
+def test_prefill_early_weight_loads_see_the_weights_packed_before():
+    """BITNET_LAUNCH_PDL on a prefill call (M > 16): the GEMM loads its first
+    weight tiles while the quantiser before it runs.  Each round re-packs new
+    weights into the same buffer, quantises a new batch and projects it on one
+    stream with no host synchronisation: every output must be the oracle's for
+    that round's weights (the quantiser lets the GEMM launch only after the
+    pack has completed)."""
+    M, K, N = 300, 512, 640
+    rng_w, rng_x = synthetic.streams(47, 2)
+    P, g, ws = bn.alloc_packed(N, K)
+    q, s, rs = bn.alloc_quant(M, K)
+    outs = []
+    for rnd in range(4):
+        W = synthetic.weight(rng_w, N, K)
+        X = synthetic.activations(rng_x, M, K)
+        Wd, Xd = dev(W), dev(X)
+        bn.bitnet_pack_weights(Wd, P, g, ws)
+        bn.bitnet_quant_act(Xd, q, s, rs)
+        Y = torch.empty((M, N), dtype=torch.int32, device="cuda")
+        bn.bitnet_linear(q, s, rs, P, g, K, Y, epilogue=bn.BITNET_I32 | bn.BITNET_LAUNCH_PDL)
+        outs.append((W, X, Y, Wd, Xd))
+    torch.cuda.synchronize()
+    for W, X, Y, _, _ in outs:
+        _, T, _ = oracle.quantize_weights(W)
+        qo, _, _ = oracle.quant_act(X)
+        np.testing.assert_array_equal(Y.cpu().numpy(), oracle.contract(qo, T))
+
+
 def test_decode_with_programmatic_dependent_launch():
     """Decode calls launched with BITNET_LAUNCH_PDL right behind the kernel that
     writes their activation codes still read the new codes: each step quantises
