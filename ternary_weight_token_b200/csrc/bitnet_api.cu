@@ -1057,12 +1057,14 @@ int bitnet_ffn(const void* X, int x_dtype, int M, int H, int I, const uint8_t* W
     p1.nseg = 2;
     p1.seg_row0[0] = 0; p1.seg_row0[1] = I; p1.seg_row0[2] = 2 * I;
     p1.seg_W[1] = W_up; p1.seg_gamma[1] = gamma_up; p1.seg_Y[1] = hid_up;
-    p1.flags = LAUNCH_PDL;
+    // (each decode launch is followed by a quantiser: the early trigger lets
+    // it be resident when the launch completes)
+    p1.flags = LAUNCH_PDL | LAUNCH_TRIGGER_EARLY;
     if (int rc = launch_linear(p1, st)) return rc;
     if (int rc = launch_quant(hid, false, M, I, PRE_GLU_RMSNORM, sub_norm_gain, eps, hq, hs, hrs,
                               st, hid_up))
       return rc;
-    p2.flags = EPI_RESIDUAL | LAUNCH_PDL;
+    p2.flags = EPI_RESIDUAL | LAUNCH_PDL | LAUNCH_TRIGGER_EARLY;
     p2.resid = X;
     return launch_linear(p2, st);
   }
