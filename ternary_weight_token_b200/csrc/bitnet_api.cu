@@ -65,6 +65,7 @@ int check_k(int K) {
 struct DeviceInfo {
   int sms = 0;
   int max_smem_optin = 0;
+  int smem_per_sm = 0;
 };
 
 int device_info(DeviceInfo& out) {
@@ -79,6 +80,8 @@ int device_info(DeviceInfo& out) {
     BN_CHECK_CUDA(cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev));
     BN_CHECK_CUDA(
         cudaDeviceGetAttribute(&di.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev));
+    BN_CHECK_CUDA(
+        cudaDeviceGetAttribute(&di.smem_per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev));
     it = cache.emplace(dev, di).first;
   }
   out = it->second;
@@ -741,8 +744,9 @@ size_t bitnet_packed_row_bytes(int K) {
 size_t bitnet_pack_workspace_size(int N, int K) {
   (void)N;
   (void)K;
-  // one-launch path: partials and exchange flags; three-launch path: partials
-  const size_t fused = (size_t)kPackMaxGrid * (sizeof(double) + sizeof(unsigned long long));
+  // one-launch path: two tagged words per CTA's partial sum and the two
+  // gamma words; three-launch path: partials
+  const size_t fused = (size_t)(2 * kPackMaxGrid + 2) * sizeof(unsigned long long);
   const size_t split = (size_t)kPackPartialBlocks * sizeof(double);
   return fused > split ? fused : split;
 }
@@ -766,30 +770,36 @@ int bitnet_pack_weights(const void* W, int w_dtype, int N, int K, uint8_t* packe
   const long long count = (long long)N * K;
   double* partials = reinterpret_cast<double*>(workspace);
   if (N > 0) {
-    // one cooperative launch: two CTAs of 512 threads per SM
+    // one cooperative launch: two CTAs of 512 threads per SM, each staging
+    // up to half of the SM's shared memory of its weights
     DeviceInfo di;
     if (int rc = device_info(di)) return rc;
-    void (*kf)(const void*, int, int, int, long long, double*, unsigned long long*,
-               unsigned long long, float*, uint8_t*) =
-        bf16 ? pack_fused_kernel<true> : pack_fused_kernel<false>;
+    void (*kf)(const void*, int, int, int, long long, unsigned long long*, unsigned long long, int,
+               float*, uint8_t*) = bf16 ? pack_fused_kernel<true> : pack_fused_kernel<false>;
+    int smem = (di.smem_per_sm / 2 - 2048) & ~1023;
+    if (smem > kPackMaxStage) smem = kPackMaxStage;
+    if (smem > di.max_smem_optin) smem = di.max_smem_optin & ~1023;
+    if (smem < 0) smem = 0;
+    if (int rc = set_smem_attr((const void*)kf, (size_t)smem)) return rc;
     int per_sm = 0;
-    if (int rc = occupancy(per_sm, (const void*)kf, kPackFusedThreads, 0)) return rc;
+    if (int rc = occupancy(per_sm, (const void*)kf, kPackFusedThreads, (size_t)smem)) return rc;
     const int G = std::min(std::min(per_sm, 2) * di.sms, kPackMaxGrid);
     if (G >= di.sms) {
-      unsigned long long* flags = reinterpret_cast<unsigned long long*>(partials + kPackMaxGrid);
+      unsigned long long* xw = reinterpret_cast<unsigned long long*>(workspace);
       const int ldw = (int)bitnet_packed_row_bytes(K);
       const unsigned long long epoch = next_epoch();
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3((unsigned)G);
       cfg.blockDim = dim3(kPackFusedThreads);
+      cfg.dynamicSmemBytes = (size_t)smem;
       cfg.stream = st;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeCooperative;
       attr[0].val.cooperative = 1;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
-      BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kf, W, N, K, ldw, count, partials, flags, epoch,
-                                       gamma, packed));
+      BN_CHECK_CUDA(cudaLaunchKernelEx(&cfg, kf, W, N, K, ldw, count, xw, epoch, smem, gamma,
+                                       packed));
       return BITNET_OK;
     }
   }

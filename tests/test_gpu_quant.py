@@ -210,6 +210,75 @@ def test_pack_threshold_boundary():
     np.testing.assert_array_equal(packed, oracle.pack(t))
 
 
+def _bf16_run(center_bits, n):
+    """n consecutive positive bf16 bit patterns centred on center_bits."""
+    return (np.arange(n, dtype=np.int64) - n // 2 + int(center_bits)).astype(np.uint16)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_pack_bf16_threshold_sweep(seed):
+    """bf16 weights: a ballast of +-b (b a random bf16 in [0.5, 2)) fixes
+    gamma near b, and 64 consecutive bf16 magnitudes around b / 2 with
+    alternating signs straddle the rounding boundary of fl(w / gamma).  The
+    packer decides t != 0 from the weight's bits; the oracle divides."""
+    rng = np.random.default_rng(100 + seed)
+    b_bits = np.uint16(0x3F00 + rng.integers(0, 0x100))          # [0.5, 2)
+    b = oracle.bf16_bits_to_f32(np.array([b_bits]))[0]
+    half_bits = synthetic.to_bf16_bits(np.array([b * np.float32(0.5)]))[0]
+    cand = _bf16_run(half_bits, 64)
+    cand = np.where(np.arange(64) % 2 == 0, cand, cand | np.uint16(0x8000)).astype(np.uint16)
+    ball = np.where(np.arange(4096) % 2 == 0, b_bits, b_bits | np.uint16(0x8000)).astype(np.uint16)
+    bits = np.concatenate([ball, cand]).reshape(-1, 64)
+    Ww = oracle.bf16_bits_to_f32(bits)
+    go = oracle.absmean(Ww)
+    t = oracle.ternarize(Ww, go)
+    tc = t.ravel()[4096:]
+    assert (tc == 0).any() and (tc != 0).any()            # the boundary lies inside the run
+    N, K = bits.shape
+    packed, gamma, ws = bn.alloc_packed(N, K)
+    bn.bitnet_pack_weights(bf16_dev(bits), packed, gamma, ws)
+    torch.cuda.synchronize()
+    assert gamma.item() == go
+    np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack(t))
+
+
+@pytest.mark.parametrize("wdtype", ["f32", "bf16"])
+def test_pack_special_magnitudes(wdtype):
+    """Signed zeros, subnormals, the largest finite values and ties at
+    gamma / 2 and 3 gamma / 2, in both weight types: codes and gamma bit for
+    bit against the oracle (subnormal-only and huge-only matrices included, so
+    the threshold itself is subnormal or near the top of the range)."""
+    if wdtype == "f32":
+        big, sub = np.float32(3.0e38), np.float32(1.0e-40)
+        mats = [
+            np.array([[0.0, -0.0, sub, -sub, 2 * sub, 1e-45, -1e-45, 0.0] * 4], np.float32),
+            np.array([[big, -big, big / 3, 0.0, -big / 2, big, 1.0, -1.0] * 2], np.float32),
+            np.array([[0.5, -1.5, 2.5, -0.5, 1.0, 0.0, -1.0, 1.0] * 4, [1e-30, -3.0] * 16], np.float32),
+        ]
+        for W in mats:
+            packed, gamma = gpu_pack(np.ascontiguousarray(W))
+            go = oracle.absmean(W)
+            assert gamma == go, (W[0, :4], gamma, go)
+            np.testing.assert_array_equal(packed, oracle.pack(oracle.ternarize(W, go)))
+        return
+    sets = [
+        np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x007F, 0x807F, 0x0080, 0x0002] * 4, np.uint16),
+        np.array([0x7F7F, 0xFF7F, 0x7F00, 0x0000, 0xFEFF, 0x7F7F, 0x3F80, 0xBF80] * 2, np.uint16),
+        synthetic.to_bf16_bits(np.array([0.5, -1.5, 2.5, -0.5, 1.0, 0.0, -1.0, 1.0] * 4, np.float32)),
+        np.array([0x0001] * 31 + [0x0003], np.uint16),
+    ]
+    for bits in sets:
+        bits = bits.reshape(1, -1)
+        Ww = oracle.bf16_bits_to_f32(bits)
+        go = oracle.absmean(Ww)
+        N, K = bits.shape
+        packed, gamma, ws = bn.alloc_packed(N, K)
+        bn.bitnet_pack_weights(bf16_dev(bits), packed, gamma, ws)
+        torch.cuda.synchronize()
+        assert gamma.item() == go, (bits[0, :4], gamma.item(), go)
+        np.testing.assert_array_equal(packed.cpu().numpy(), oracle.pack(oracle.ternarize(Ww, go)))
+
+
 def test_pack_is_deterministic():
     W = synthetic.weight(np.random.default_rng(12), 2560, 2560)
     a = gpu_pack(W)
