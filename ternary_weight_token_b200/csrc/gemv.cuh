@@ -78,17 +78,15 @@ __device__ __forceinline__ float int_to_float_exact(int v) {
   return __fsub_rn(__int_as_float(0x4B400000 + v), 12582912.0f);
 }
 
-// y = v * (f_hi + f_lo) in fp32 double-word arithmetic, where f_hi + f_lo is
-// gamma / s to about 2^-48 relative: the two-product error term is exact
-// (FMA), so the one rounding of the sum gives the correctly rounded fp32 of
+// y = v * (f_hi + f_lo), where f_hi + f_lo is gamma / s to about 2^-48
+// relative: one FMA adds the exact product v * f_hi to the rounded small term
+// v * f_lo (|f_lo| <= 2^-24 f_hi, so that term's rounding error is ~2^-48 of
+// the result), and its one rounding gives the correctly rounded fp32 of
 // v * gamma / s except when that value lies within ~2^-46 of an fp32
 // midpoint.  The accumulator |v| <= 128 * K <= 2^21 is exact in fp32.
 __device__ __forceinline__ float dequant_dw(int v, float f_hi, float f_lo) {
   const float a = int_to_float_exact(v);
-  const float p = __fmul_rn(a, f_hi);
-  const float e = __fmaf_rn(a, f_hi, -p);
-  const float t = __fmaf_rn(a, f_lo, e);
-  return __fadd_rn(p, t);
+  return __fmaf_rn(a, f_hi, __fmul_rn(a, f_lo));
 }
 
 // Split gamma / s into an fp32 head and tail: the head is the correctly
