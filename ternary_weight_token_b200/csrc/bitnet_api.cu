@@ -531,17 +531,31 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
 // (a warp per R rows, all of a lane's weight loads in flight at once).
 template <int MT, int NT>
 int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaStream_t st) {
+  // independent calls (LAUNCH_PDL_INPUTS) on matrices of 2 MB and more
+  // bulk-copy their weight rows into shared memory, so that more calls' CTAs
+  // share an SM; a dependent call keeps them in registers (its critical path
+  // starts at its wait), and so does a smaller matrix, whose calls are bound
+  // by launch rate rather than by bytes in flight
+  const bool bulk = (p.flags & LAUNCH_PDL_INPUTS) != 0 && (long long)p.N * p.ldw >= (1ll << 21);
   void (*kern)(LinearParams) = nullptr;
+#define BN_STREAM_CASE(RR)                                                        \
+  case RR:                                                                        \
+    kern = bulk ? gemv_stream_kernel<MT, RR, 8, NT, true> : gemv_stream_kernel<MT, RR, 8, NT, false>; \
+    break;
   switch (R) {
-    case 1: kern = gemv_stream_kernel<MT, 1, 8, NT>; break;
-    case 2: kern = gemv_stream_kernel<MT, 2, 8, NT>; break;
-    case 3: kern = gemv_stream_kernel<MT, 3, 8, NT>; break;
-    case 4: kern = gemv_stream_kernel<MT, 4, 8, NT>; break;
-    case 5: kern = gemv_stream_kernel<MT, 5, 8, NT>; break;
-    case 6: kern = gemv_stream_kernel<MT, 6, 8, NT>; break;
-    case 7: kern = gemv_stream_kernel<MT, 7, 8, NT>; break;
-    default: kern = gemv_stream_kernel<MT, 8, 8, NT>; break;
+    BN_STREAM_CASE(1)
+    BN_STREAM_CASE(2)
+    BN_STREAM_CASE(3)
+    BN_STREAM_CASE(4)
+    BN_STREAM_CASE(5)
+    BN_STREAM_CASE(6)
+    BN_STREAM_CASE(7)
+    default:
+      kern = bulk ? gemv_stream_kernel<MT, 8, 8, NT, true> : gemv_stream_kernel<MT, 8, 8, NT, false>;
+      break;
   }
+#undef BN_STREAM_CASE
+  if (!bulk) smem = (size_t)MT * (size_t)p.K;    // activation codes only
   if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   LinearParams q = p;
   q.flags &= ~LAUNCH_PDL;
@@ -563,7 +577,9 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : 8;
   if (mt == 8 && R > 4) R = 4;                   // lane r * MT + m holds (row, token): R MT <= 32
   const int grid = (p.N + warps * R - 1) / (warps * R);
-  const size_t smem = (size_t)mt * (size_t)p.K;
+  // the CTA's weight rows (bulk-copied by independent calls), then the
+  // activation codes
+  const size_t smem = (size_t)warps * R * p.ldw + (size_t)mt * (size_t)p.K;
   if (mt == 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
   if (mt == 2) return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
   return launch_stream_mt<8, kStreamThreads>(p, R, grid, smem, st);

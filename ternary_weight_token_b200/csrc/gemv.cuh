@@ -217,47 +217,92 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
 
 // ---------------------------------------------------------------------------
 // Streaming decode for 1..2 tokens (dp4a on the CUDA cores, no tensor memory,
-// no cluster).  A warp owns R whole weight rows; its R * C 16-byte packed
-// chunks (C = row_bytes / 16) are spread over the 32 lanes, J per lane, and
-// every lane issues all of its loads before anything waits: for a decode
-// call the whole matrix is a few tens of KB per SM, so the call is bound by
-// load latency, and consecutive calls are meant to overlap (several of these
-// small CTAs fit on an SM next to the previous call's).  Activation codes are
-// staged in shared memory (K a multiple of 64).  The weights are read before griddepcontrol.wait
-// (the caller's LAUNCH_PDL statement covers them); with LAUNCH_PDL_INPUTS the
-// activations and the whole contraction also precede it, and only the output
-// stores wait.  A dependent call (LAUNCH_PDL without _INPUTS) lets the next
-// grid launch only after its own wait: in a chain of dependent calls that
-// bounds the look-ahead to one call, whose weight loads then do not queue in
-// front of the current call's (1-token 4.4 MB calls: 0.95-1.0 -> 1.22-1.27
-// TB/s); LAUNCH_TRIGGER_EARLY keeps the trigger at the start.
+// no cluster).  A CTA owns NT / 32 * R consecutive weight rows and a warp R
+// of them, their R * C 16-byte packed chunks (C = row_bytes / 16) spread over
+// the 32 lanes, J per lane.  For a decode call the whole matrix is a few tens
+// of KB per SM, so a call is bound by load latency, and consecutive calls are
+// meant to overlap.  The weights are requested before anything waits: with
+// BULK (independent calls on 2 MB or more) one thread bulk-copies the CTA's
+// rows into shared memory (one copy per projection they fall in, completing
+// on an mbarrier), so no register holds a load in flight and more calls'
+// CTAs fit on an SM at once (back-to-back 1-token 4.4 MB calls: 1.62 -> 1.26
+// us); otherwise each lane loads its chunks into registers, all in flight at
+// once.  Activation codes are staged in shared memory (K a multiple of 64)
+// while the weights land.  The weights (and gamma) are read before
+// griddepcontrol.wait (the caller's LAUNCH_PDL statement covers them); with
+// LAUNCH_PDL_INPUTS the activations and the whole contraction also precede
+// it, and only the output stores wait.  A dependent call (LAUNCH_PDL without
+// _INPUTS) lets the next grid launch only after its own wait: in a chain of
+// dependent calls that bounds the look-ahead to one call, whose weight loads
+// then do not queue in front of the current call's; LAUNCH_TRIGGER_EARLY
+// keeps the trigger at the start.
 
-template <int MT, int R, int J, int NT>
+template <int MT, int R, int J, int NT, bool BULK>
 __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
-  // activation codes as [MT][4][C] 16-byte units: unit u of a token row (its
-  // inputs 16u .. 16u + 15) sits in plane u % 4 at index u / 4, so the lanes
-  // of a warp, which hold consecutive chunks, read consecutive 16-byte words
+  // shared memory: (BULK) the CTA's weight rows (NT / 32 * R rows of ldw
+  // bytes, as stored), then the activation codes as [MT][4][C] 16-byte units:
+  // unit u of a token row (its inputs 16u .. 16u + 15) sits in plane u % 4 at
+  // index u / 4, so the lanes of a warp, which hold consecutive chunks, read
+  // consecutive 16-byte words
   extern __shared__ uint4 gs_smem[];
+  __shared__ __align__(8) uint64_t s_wbar;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int C = p.ldw / 16;                    // packed chunks per row
-  const int n0 = (blockIdx.x * (NT / 32) + warp) * R;
+  // f / C = umulhi(f, ceil(2^32 / C)) exactly for f < 2^16 and 2 <= C <= 2^16
+  // (the error term f (cmul C - 2^32) / 2^32 stays below 1 / C; C = 1 is f
+  // itself): chunk f of the warp's rows is row f / C, chunk f % C of the
+  // row, with no division and no dependence between chunks
+  const uint32_t cmul = C > 1 ? 0xffffffffu / (uint32_t)C + 1u : 0u;
+  constexpr int RB = (NT / 32) * R;            // weight rows of the CTA
+  const int nb0 = blockIdx.x * RB;
+  const int n0 = nb0 + warp * R;
+  uint4* s_w = gs_smem;
+  uint4* s_x = gs_smem + (BULK ? RB * C : 0);
   const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
   const bool trigger_early = inputs_ready || (p.flags & LAUNCH_TRIGGER_EARLY) != 0;
   if (trigger_early) grid_launch_dependents();
 
-  // 1. every packed chunk of this warp's rows, in flight at once (rows are
-  // the concatenated rows of the call's projections)
-  uint4 w[J];
-#pragma unroll
-  for (int j = 0; j < J; ++j) {
-    const int f = lane + 32 * j;
-    const int r = f / C, c = f - r * C;
-    w[j] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // t = 0
-    if (r < R && n0 + r < p.N) {
-      int nl;
-      const int sg = segment_of(p, n0 + r, nl);
-      w[j] = ld_stream_v4(p.seg_W[sg] + (size_t)nl * p.ldw + 16 * c);
+  // 1. the weights, requested before anything waits.  BULK: the CTA's rows
+  // by bulk copies (one per projection they fall in) completing on an
+  // mbarrier; no register holds a load in flight, so several calls' CTAs fit
+  // on an SM at once.  Otherwise every packed chunk of the warp's rows into
+  // registers, all in flight at once (chunk f = lane + 32 j as row f / C,
+  // chunk f % C of the row).
+  uint4 w[BULK ? 1 : J];
+  if constexpr (BULK) {
+    if (threadIdx.x == 0) {
+      mbar_init(&s_wbar, 1);
+      fence_barrier_init();
+      const int nb1 = nb0 + RB < p.N ? nb0 + RB : p.N;
+      mbar_arrive_expect_tx(&s_wbar, (uint32_t)((nb1 - nb0) * p.ldw));
+      for (int sg = 0; sg < p.nseg; ++sg) {
+        const int lo = nb0 > p.seg_row0[sg] ? nb0 : p.seg_row0[sg];
+        const int hi = nb1 < p.seg_row0[sg + 1] ? nb1 : p.seg_row0[sg + 1];
+        if (lo < hi)
+          bulk_load_1d(reinterpret_cast<uint8_t*>(s_w) + (size_t)(lo - nb0) * p.ldw,
+                       p.seg_W[sg] + (size_t)(lo - p.seg_row0[sg]) * p.ldw,
+                       (uint32_t)((hi - lo) * p.ldw), &s_wbar);
+      }
     }
+  } else {
+#pragma unroll
+    for (int j = 0; j < J; ++j) {
+      const int f = lane + 32 * j;
+      const int r = C > 1 ? (int)__umulhi((uint32_t)f, cmul) : f, c = f - r * C;
+      w[j] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // t = 0
+      if (r < R && n0 + r < p.N) {
+        int nl;
+        const int sg = segment_of(p, n0 + r, nl);
+        w[j] = ld_stream_v4(p.seg_W[sg] + (size_t)nl * p.ldw + 16 * c);
+      }
+    }
+  }
+  // the weight scale of this lane's output (lane r * MT + m: row n0 + r,
+  // token m), part of the packed weights: fetched before any wait
+  float gam = 0.0f;
+  if (lane < R * MT && n0 + lane / MT < p.N) {
+    int nl;
+    gam = __ldg(p.seg_gamma[segment_of(p, n0 + lane / MT, nl)]);
   }
 
   // 2. activation codes, token scales and code sums
@@ -270,43 +315,74 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
     const int m = i / units, u = i - m * units;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (m < p.M) v = *reinterpret_cast<const uint4*>(p.Xq + (size_t)m * p.K + 16 * u);
-    gs_smem[(m * 4 + (u & 3)) * C + (u >> 2)] = v;
+    s_x[(m * 4 + (u & 3)) * C + (u >> 2)] = v;
   }
   const int mt = lane < MT ? lane : 0;
   const bool tok = lane < p.M;
   const float s_m = tok ? p.xs[mt] : 1.0f;
   const int rs_m = tok ? p.xrs[mt] : 0;
-  __syncthreads();
+  __syncthreads();                             // also publishes the barrier's initialisation
+  if constexpr (BULK) {
+    if (!mbar_wait(&s_wbar, 0u, nullptr)) {
+      // never leave with a bulk copy in flight into this CTA's shared memory
+      mbar_wait(&s_wbar, 0u, nullptr);
+      return;
+    }
+  }
 
-  // 3. unsigned codes x signed activations, per row and token
+  // 3. unsigned codes x signed activations, per row and token.  Word u of a
+  // chunk holds weight 16u + 4i + j at byte j, bits 2i; masking it with
+  // 0x03030303 << 2i (no shift) leaves 4^i times the codes of weights
+  // 16u + 4i .. 16u + 4i + 3, so the dp4a chain A_i of mask i carries a
+  // factor 4^i, removed once per chunk: A_0 + A_1 / 4 + A_2 / 16 + A_3 / 64,
+  // exact (each A_i is a multiple of 4^i; |A_i| < 2^19).
   int acc[R][MT];
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int m = 0; m < MT; ++m) acc[r][m] = 0;
+  // chunk f = lane + 32 j as (row r, chunk c of the row): with the weights
+  // in registers (a dependent call, latency-bound) from f directly, so that
+  // the chunks' shared-memory reads are independent; with bulk-copied
+  // weights (independent calls, throughput-bound) stepped from the previous
+  // chunk, which takes fewer instructions
+  int r = 0, c = lane;
+  if constexpr (BULK) {
+    while (c >= C) {
+      c -= C;
+      ++r;
+    }
+  }
 #pragma unroll
   for (int j = 0; j < J; ++j) {
-    const int f = lane + 32 * j;
-    const int r = f / C, c = f - r * C;
-    if (r < R) {
-      uint32_t e[16];
-      expand_codes(w[j].x, e[0], e[1], e[2], e[3]);
-      expand_codes(w[j].y, e[4], e[5], e[6], e[7]);
-      expand_codes(w[j].z, e[8], e[9], e[10], e[11]);
-      expand_codes(w[j].w, e[12], e[13], e[14], e[15]);
+    if constexpr (BULK) {
+      if (j > 0) {
+        c += 32;
+        while (c >= C) {
+          c -= C;
+          ++r;
+        }
+      }
+    } else {
+      const int f = lane + 32 * j;
+      r = C > 1 ? (int)__umulhi((uint32_t)f, cmul) : f;
+      c = f - r * C;
+    }
+    if (r < R && n0 + r < p.N) {
+      const uint4 wj = BULK ? s_w[(warp * R + r) * C + c] : w[j];
+      const uint32_t wv[4] = {wj.x, wj.y, wj.z, wj.w};
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        const uint4* qp = gs_smem + m * 4 * C + c;       // 64 activation codes
-        const uint4 q0 = qp[0], q1 = qp[C], q2 = qp[2 * C], q3 = qp[3 * C];
-        int a = 0;
-        a = dp4a_us(e[0], q0.x, a);  a = dp4a_us(e[1], q0.y, a);
-        a = dp4a_us(e[2], q0.z, a);  a = dp4a_us(e[3], q0.w, a);
-        a = dp4a_us(e[4], q1.x, a);  a = dp4a_us(e[5], q1.y, a);
-        a = dp4a_us(e[6], q1.z, a);  a = dp4a_us(e[7], q1.w, a);
-        a = dp4a_us(e[8], q2.x, a);  a = dp4a_us(e[9], q2.y, a);
-        a = dp4a_us(e[10], q2.z, a); a = dp4a_us(e[11], q2.w, a);
-        a = dp4a_us(e[12], q3.x, a); a = dp4a_us(e[13], q3.y, a);
-        a = dp4a_us(e[14], q3.z, a); a = dp4a_us(e[15], q3.w, a);
+        const uint4* qp = s_x + m * 4 * C + c;           // 64 activation codes
+        const uint4 qv[4] = {qp[0], qp[C], qp[2 * C], qp[3 * C]};
+        int A[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t q4[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) A[i] = dp4a_us(wv[u] & (0x03030303u << (2 * i)), q4[i], A[i]);
+        }
+        const int a = A[0] + (A[1] >> 2) + (A[2] >> 4) + (A[3] >> 6);
 #pragma unroll
         for (int rr = 0; rr < R; ++rr)
           if (rr == r) acc[rr][m] += a;
@@ -342,7 +418,7 @@ __global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
     sg = segment_of(p, n, nl);
     if (p.out_type != OUT_I32) {
       float fh, fl;
-      dequant_factor(__ldg(p.seg_gamma[sg]), y, fh, fl);
+      dequant_factor(gam, y, fh, fl);
       y = dequant_dw(yint, fh, fl);
     }
   }
