@@ -531,12 +531,13 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
 // (a warp per R rows, all of a lane's weight loads in flight at once).
 template <int MT, int NT>
 int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaStream_t st) {
-  // independent calls (LAUNCH_PDL_INPUTS) on matrices of 2 MB and more
+  // independent calls (LAUNCH_PDL_INPUTS) on 4 MB of weights or more
   // bulk-copy their weight rows into shared memory, so that more calls' CTAs
   // share an SM; a dependent call keeps them in registers (its critical path
-  // starts at its wait), and so does a smaller matrix, whose calls are bound
-  // by launch rate rather than by bytes in flight
-  const bool bulk = (p.flags & LAUNCH_PDL_INPUTS) != 0 && (long long)p.N * p.ldw >= (1ll << 21);
+  // starts at its wait), and so does a smaller call, whose pace is set by
+  // launch rate rather than by bytes in flight (1.6 MB single and 2.5 MB
+  // q/k/v calls measured slower with the bulk copies, 4.4 MB ones faster)
+  const bool bulk = (p.flags & LAUNCH_PDL_INPUTS) != 0 && (long long)p.N * p.ldw >= (1ll << 22);
   void (*kern)(LinearParams) = nullptr;
 #define BN_STREAM_CASE(RR)                                                        \
   case RR:                                                                        \

@@ -222,7 +222,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
 // the 32 lanes, J per lane.  For a decode call the whole matrix is a few tens
 // of KB per SM, so a call is bound by load latency, and consecutive calls are
 // meant to overlap.  The weights are requested before anything waits: with
-// BULK (independent calls on 2 MB or more) one thread bulk-copies the CTA's
+// BULK (independent calls on 4 MB or more) one thread bulk-copies the CTA's
 // rows into shared memory (one copy per projection they fall in, completing
 // on an mbarrier), so no register holds a load in flight and more calls'
 // CTAs fit on an SM at once (back-to-back 1-token 4.4 MB calls: 1.62 -> 1.26
