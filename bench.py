@@ -914,9 +914,10 @@ def run_b200(args, world, rank, local):
     return 0
 
 
-def decode_single(torch, bn, device, M, K, N, iters):
+def decode_single(torch, bn, device, M, K, N, iters, independent=False):
     """Plain back-to-back launches of one decode shape (no graph): the short
-    command the decode kernel is profiled with."""
+    command the decode kernel is profiled with (independent: the calls carry
+    BITNET_LAUNCH_PDL_INPUTS, as independent projections do)."""
     inp = synthetic.linear_inputs(M, K, N, seed=K + N)
     W = torch.from_numpy(inp["W"]).to(device)
     P, g, ws = bn.alloc_packed(N, K, device)
@@ -926,12 +927,14 @@ def decode_single(torch, bn, device, M, K, N, iters):
     bn.bitnet_quant_act(X, q, s, rs)
     Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
 
+    epi = bn.BITNET_BF16 | (bn.BITNET_LAUNCH_PDL_INPUTS if independent else 0)
+
     def run():
-        bn.bitnet_linear(q, s, rs, P, g, K, Y)
+        bn.bitnet_linear(q, s, rs, P, g, K, Y, epilogue=epi)
     for _ in range(3):
         run()
     dt = time_loop(torch, run, iters) / iters
-    return {"M": M, "K": K, "N": N, "us_per_call": dt * 1e6,
+    return {"M": M, "K": K, "N": N, "independent": independent, "us_per_call": dt * 1e6,
             "GB_s": decode_bytes(M, K, N) / dt / 1e9}
 
 
@@ -941,8 +944,10 @@ def run_only(args, local):
     device = torch.device("cuda", local)
     import ternary_weight_token_b200 as bn
     if args.only == "decode" and args.decode_shape:
-        M, K, N = (int(v) for v in args.decode_shape.split(","))
-        out = decode_single(torch, bn, device, M, K, N, max(1, args.steps))
+        fields = args.decode_shape.split(",")
+        M, K, N = (int(v) for v in fields[:3])
+        out = decode_single(torch, bn, device, M, K, N, max(1, args.steps),
+                            independent=len(fields) > 3 and fields[3] == "independent")
     else:
         fn = {"decode": bench_decode, "ffn": bench_ffn, "hffn": bench_hffn,
               "tiny": bench_tiny, "qkv": bench_decode_qkv, "online": bench_online,
@@ -967,7 +972,7 @@ def main(argv=None):
                     default=None,
                     help="time one secondary workload and print its JSON (profiling aid)")
     ap.add_argument("--decode-shape", default=None,
-                    help="with --only decode: one 'M,K,N' case, no CUDA graph")
+                    help="with --only decode: one 'M,K,N[,independent]' case, no CUDA graph")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -529,61 +529,93 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
 
 // Decode for 1..2 tokens with K a multiple of 64: the dp4a streaming kernel
 // (a warp per R rows, all of a lane's weight loads in flight at once).
-template <int MT, int NT>
-int launch_stream_mt(const LinearParams& p, int R, int grid, size_t smem, cudaStream_t st) {
-  // independent calls (LAUNCH_PDL_INPUTS) on 4 MB of weights or more
-  // bulk-copy their weight rows into shared memory, so that more calls' CTAs
-  // share an SM; a dependent call keeps them in registers (its critical path
-  // starts at its wait), and so does a smaller call, whose pace is set by
-  // launch rate rather than by bytes in flight (1.6 MB single and 2.5 MB
-  // q/k/v calls measured slower with the bulk copies, 4.4 MB ones faster)
-  const bool bulk = (p.flags & LAUNCH_PDL_INPUTS) != 0 && (long long)p.N * p.ldw >= (1ll << 22);
-  void (*kern)(LinearParams) = nullptr;
-#define BN_STREAM_CASE(RR)                                                        \
-  case RR:                                                                        \
-    kern = bulk ? gemv_stream_kernel<MT, RR, 8, NT, true> : gemv_stream_kernel<MT, RR, 8, NT, false>; \
-    break;
-  switch (R) {
-    BN_STREAM_CASE(1)
-    BN_STREAM_CASE(2)
-    BN_STREAM_CASE(3)
-    BN_STREAM_CASE(4)
-    BN_STREAM_CASE(5)
-    BN_STREAM_CASE(6)
-    BN_STREAM_CASE(7)
-    default:
-      kern = bulk ? gemv_stream_kernel<MT, 8, 8, NT, true> : gemv_stream_kernel<MT, 8, 8, NT, false>;
-      break;
-  }
-#undef BN_STREAM_CASE
-  if (!bulk) smem = (size_t)MT * (size_t)p.K;    // activation codes only
+constexpr int kStreamChunks = 8;               // packed chunks per lane, at most
+
+template <int MT>
+int launch_stream_mt(const LinearParams& p, int L, int warps, int grid, cudaStream_t st) {
+  void (*kern)(LinearParams, int) = gemv_stream_kernel<MT, kStreamChunks>;
+  const size_t smem = (size_t)MT * (size_t)p.K;  // activation codes
   if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
   LinearParams q = p;
   q.flags &= ~LAUNCH_PDL;
-  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(NT), smem, st, q);
+  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(32 * warps), smem, st,
+                       q, L);
 }
 
-constexpr int kStreamThreads = 256;
+constexpr int kFlatThreads = 256;
+
+template <int MT>
+int launch_flat_mt(const LinearParams& p, int R, bool bulk, cudaStream_t st) {
+  void (*kern)(LinearParams) = nullptr;
+#define BN_FLAT_CASE(RR)                                                                  \
+  case RR:                                                                                \
+    kern = bulk ? gemv_flat_kernel<MT, RR, kStreamChunks, kFlatThreads, true>             \
+                : gemv_flat_kernel<MT, RR, kStreamChunks, kFlatThreads, false>;           \
+    break;
+  switch (R) {
+    BN_FLAT_CASE(1)
+    BN_FLAT_CASE(2)
+    BN_FLAT_CASE(3)
+    BN_FLAT_CASE(4)
+    BN_FLAT_CASE(5)
+    BN_FLAT_CASE(6)
+    BN_FLAT_CASE(7)
+    default:
+      kern = bulk ? gemv_flat_kernel<MT, 8, kStreamChunks, kFlatThreads, true>
+                  : gemv_flat_kernel<MT, 8, kStreamChunks, kFlatThreads, false>;
+      break;
+  }
+#undef BN_FLAT_CASE
+  const int warps = kFlatThreads / 32;
+  const int grid = (p.N + warps * R - 1) / (warps * R);
+  // (bulk) the CTA's weight rows, then the activation codes
+  const size_t smem = (bulk ? (size_t)warps * R * p.ldw : 0) + (size_t)MT * (size_t)p.K;
+  if (int rc = set_smem_attr((const void*)kern, smem)) return rc;
+  LinearParams q = p;
+  q.flags &= ~LAUNCH_PDL;
+  return launch_pdl_if((p.flags & LAUNCH_PDL) != 0, kern, dim3(grid), dim3(kFlatThreads), smem,
+                       st, q);
+}
 
 int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
-  const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64)
-  const int warps = kStreamThreads / 32;
-  // about one CTA per SM per call (so several back-to-back calls can be
-  // resident at once): R rows per warp, at most 8 loads per lane
-  int R = (p.N + di.sms * warps - 1) / (di.sms * warps);
-  if (R > 8) R = 8;
-  while (R > 1 && R * C > 32 * 8) --R;
+  const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64), <= 256
   const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : 8;
-  if (mt == 8 && R > 4) R = 4;                   // lane r * MT + m holds (row, token): R MT <= 32
-  const int grid = (p.N + warps * R - 1) / (warps * R);
-  // the CTA's weight rows (bulk-copied by independent calls), then the
-  // activation codes
-  const size_t smem = (size_t)warps * R * p.ldw + (size_t)mt * (size_t)p.K;
-  if (mt == 1) return launch_stream_mt<1, kStreamThreads>(p, R, grid, smem, st);
-  if (mt == 2) return launch_stream_mt<2, kStreamThreads>(p, R, grid, smem, st);
-  return launch_stream_mt<8, kStreamThreads>(p, R, grid, smem, st);
+  // Independent calls (LAUNCH_PDL_INPUTS) and 3-8 tokens take the flat
+  // kernel; independent calls on 4 MB of weights or more bulk-copy their
+  // weight rows into shared memory there, so that more calls' CTAs share an
+  // SM (1.6 MB single and 2.5 MB q/k/v calls measured slower with the bulk
+  // copies, 4.4 MB ones faster).  Dependent calls take the row groups.
+  const bool independent = (p.flags & LAUNCH_PDL_INPUTS) != 0;
+  if (independent || mt == 8) {
+    // R rows per warp: about one CTA per SM per call, at most 8 chunks a lane
+    const int warps = kFlatThreads / 32;
+    int R = (p.N + di.sms * warps - 1) / (di.sms * warps);
+    if (R > 8) R = 8;
+    while (R > 1 && R * C > 32 * kStreamChunks) --R;
+    if (mt == 8 && R > 4) R = 4;                 // lane r * MT + m holds (row, token): R MT <= 32
+    const bool bulk = independent && (long long)p.N * p.ldw >= (1ll << 22);
+    if (mt == 1) return launch_flat_mt<1>(p, R, bulk, st);
+    if (mt == 2) return launch_flat_mt<2>(p, R, bulk, st);
+    return launch_flat_mt<8>(p, R, bulk, st);
+  }
+  // L lanes per row (a power of two): each lane at most kStreamChunks chunks,
+  // and on small matrices more lanes per row, so that the call still has
+  // about 256 lanes per SM (a row has C chunks: no more than C lanes)
+  int L = 1;
+  while (L * kStreamChunks < C) L *= 2;
+  while (L < 32 && L < C && (long long)p.N * L < (long long)di.sms * 256) L *= 2;
+  const int G = 32 / L;                        // rows per warp
+  // warps per CTA: about one CTA per SM per call (so several back-to-back
+  // calls can be resident at once), at most 8
+  int warps = p.N / (di.sms * G);
+  if (warps > 8) warps = 8;
+  if (warps < 1) warps = 1;
+  const int rows = warps * G;
+  const int grid = (p.N + rows - 1) / rows;
+  if (mt == 1) return launch_stream_mt<1>(p, L, warps, grid, st);
+  return launch_stream_mt<2>(p, L, warps, grid, st);
 }
 
 // Projection i of a call as a call of its own.

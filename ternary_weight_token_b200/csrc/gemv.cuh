@@ -217,28 +217,149 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(LinearParams p) {
 
 // ---------------------------------------------------------------------------
 // Streaming decode for 1..2 tokens (dp4a on the CUDA cores, no tensor memory,
-// no cluster).  A CTA owns NT / 32 * R consecutive weight rows and a warp R
-// of them, their R * C 16-byte packed chunks (C = row_bytes / 16) spread over
-// the 32 lanes, J per lane.  For a decode call the whole matrix is a few tens
-// of KB per SM, so a call is bound by load latency, and consecutive calls are
-// meant to overlap.  The weights are requested before anything waits: with
+// no cluster) in dependent calls (independent calls, and 3-8 tokens on small
+// matrices, take gemv_flat_kernel below).  A warp owns G = 32 / L consecutive
+// weight rows, L lanes per row: lane (g, sub) takes chunks sub, sub + L,
+// sub + 2L, ... (16 bytes, 64 weights each) of row g, at most J of them, all
+// loaded into registers before anything waits, so each lane adds into one
+// sum per token and a row's sum is an L-lane butterfly (no per-chunk row
+// bookkeeping: a dependent 1-token 4.4 MB call 3.34 -> 2.56 us against lanes
+// spread over several rows).  Activation codes are staged in shared memory
+// (K a multiple of 64) while the weights land; the lanes of different row
+// groups read the same chunks' codes.  The weights (and gamma) are read
+// before griddepcontrol.wait (the caller's LAUNCH_PDL statement covers them);
+// with LAUNCH_PDL_INPUTS the activations and the whole contraction also
+// precede it, and only the output stores wait.  A dependent call (LAUNCH_PDL
+// without _INPUTS) lets the next grid launch only after its own wait: in a
+// chain of dependent calls that bounds the look-ahead to one call, whose
+// weight loads then do not queue in front of the current call's;
+// LAUNCH_TRIGGER_EARLY keeps the trigger at the start.
+template <int MT, int J>
+__global__ void __launch_bounds__(256) gemv_stream_kernel(LinearParams p, int L) {
+  // shared memory: the activation codes as [MT][4][C] 16-byte units: unit u
+  // of a token row (its inputs 16u .. 16u + 15) sits in plane u % 4 at index
+  // u / 4, so lanes holding consecutive chunks read consecutive 16-byte words
+  extern __shared__ uint4 gs_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int C = p.ldw / 16;                    // packed chunks per row
+  const int G = 32 / L;                        // rows per warp
+  const int nb0 = blockIdx.x * (int)(blockDim.x >> 5) * G;
+  const int g = lane / L, sub = lane - g * L;
+  const int n = nb0 + warp * G + g;            // this lane's row
+  const bool row_ok = n < p.N;
+  uint4* s_x = gs_smem;
+  const bool inputs_ready = (p.flags & LAUNCH_PDL_INPUTS) != 0;
+  const bool trigger_early = inputs_ready || (p.flags & LAUNCH_TRIGGER_EARLY) != 0;
+  if (trigger_early) grid_launch_dependents();
+
+  // 1. the weights
+  int nl = 0, sg = 0;
+  if (row_ok) sg = segment_of(p, n, nl);
+  uint4 w[J];
+  const uint8_t* src = p.seg_W[sg] + (size_t)nl * p.ldw;
+#pragma unroll
+  for (int k = 0; k < J; ++k) {
+    const int c = sub + L * k;
+    w[k] = make_uint4(0x55555555u, 0x55555555u, 0x55555555u, 0x55555555u);   // t = 0
+    if (row_ok && c < C) w[k] = ld_stream_v4(src + 16 * c);
+  }
+  // the weight scale of this lane's row, part of the packed weights: fetched
+  // before any wait
+  const float gam = row_ok ? __ldg(p.seg_gamma[sg]) : 0.0f;
+
+  // 2. activation codes, token scales and code sums
+  if (!inputs_ready) {
+    grid_dependency_wait();
+    if (!trigger_early) grid_launch_dependents();
+  }
+  const int units = p.K / 16;
+  for (int i = threadIdx.x; i < MT * units; i += blockDim.x) {
+    const int m = i / units, u = i - m * units;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (m < p.M) v = *reinterpret_cast<const uint4*>(p.Xq + (size_t)m * p.K + 16 * u);
+    s_x[(m * 4 + (u & 3)) * C + (u >> 2)] = v;
+  }
+  float xs_m[MT];
+  int xrs_m[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    xs_m[m] = m < p.M ? p.xs[m] : 1.0f;
+    xrs_m[m] = m < p.M ? p.xrs[m] : 0;
+  }
+  __syncthreads();
+
+  // 3. unsigned codes x signed activations.  Word u of a chunk holds weight
+  // 16u + 4i + j at byte j, bits 2i; masking it with 0x03030303 << 2i (no
+  // shift) leaves 4^i times the codes of weights 16u + 4i .. 16u + 4i + 3, so
+  // the dp4a chain A_i of mask i carries a factor 4^i, removed once per
+  // chunk: A_0 + A_1 / 4 + A_2 / 16 + A_3 / 64, exact (each A_i is a multiple
+  // of 4^i; |A_i| < 2^19).
+  int acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) acc[m] = 0;
+#pragma unroll
+  for (int k = 0; k < J; ++k) {
+    const int c = sub + L * k;
+    if (row_ok && c < C) {
+      const uint4 wj = w[k];
+      const uint32_t wv[4] = {wj.x, wj.y, wj.z, wj.w};
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4* qp = s_x + m * 4 * C + c;           // 64 activation codes
+        const uint4 qv[4] = {qp[0], qp[C], qp[2 * C], qp[3 * C]};
+        int A[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t q4[4] = {qv[u].x, qv[u].y, qv[u].z, qv[u].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) A[i] = dp4a_us(wv[u] & (0x03030303u << (2 * i)), q4[i], A[i]);
+        }
+        acc[m] += A[0] + (A[1] >> 2) + (A[2] >> 4) + (A[3] >> 6);
+      }
+    }
+  }
+
+  // 4. row sums over the row's L lanes (butterfly: every lane of the group
+  // ends with them); lane sub of the group stores tokens m = sub, sub + L, ...
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+    for (int o = L >> 1; o > 0; o >>= 1) acc[m] += __shfl_xor_sync(0xffffffffu, acc[m], o);
+  if (inputs_ready) grid_dependency_wait();    // Y may still be read or written before
+  if (!row_ok) return;
+  const int Ns = p.seg_row0[sg + 1] - p.seg_row0[sg];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if (m % L != sub || m >= p.M) continue;
+    const int yint = acc[m] - xrs_m[m];
+    const size_t idx = (size_t)m * Ns + nl;
+    if (p.out_type == OUT_I32) {
+      reinterpret_cast<int32_t*>(p.seg_Y[sg])[idx] = yint;
+    } else {
+      float fh, fl;
+      dequant_factor(gam, xs_m[m], fh, fl);
+      store_value(p.seg_Y[sg], p.resid, idx, dequant_dw(yint, fh, fl), p.out_type, p.flags);
+    }
+  }
+}
+
+// Streaming decode with a warp's chunks spread flat over its rows (chunk
+// f = lane + 32 j of the warp's R rows), for independent calls
+// (LAUNCH_PDL_INPUTS) and for 3-8 tokens on small matrices; the row-group
+// kernel above takes the rest.  Measured on the 1-token shapes, this layout
+// streams independent calls faster (4.4 MB: 1.27 / 1.43 against 1.49 / 1.74
+// us; 1.6 MB: 0.87 against 1.13 us; q/k/v 2.5 MB: 1.05 against 1.67 us) and
+// the row groups serve dependent calls better (4.4 MB: 2.56 / 3.07 against
+// 3.34 / 3.28 us).  The weights are requested before anything waits: with
 // BULK (independent calls on 4 MB or more) one thread bulk-copies the CTA's
 // rows into shared memory (one copy per projection they fall in, completing
-// on an mbarrier), so no register holds a load in flight and more calls'
-// CTAs fit on an SM at once (back-to-back 1-token 4.4 MB calls: 1.62 -> 1.26
-// us); otherwise each lane loads its chunks into registers, all in flight at
-// once.  Activation codes are staged in shared memory (K a multiple of 64)
-// while the weights land.  The weights (and gamma) are read before
-// griddepcontrol.wait (the caller's LAUNCH_PDL statement covers them); with
-// LAUNCH_PDL_INPUTS the activations and the whole contraction also precede
-// it, and only the output stores wait.  A dependent call (LAUNCH_PDL without
-// _INPUTS) lets the next grid launch only after its own wait: in a chain of
-// dependent calls that bounds the look-ahead to one call, whose weight loads
-// then do not queue in front of the current call's; LAUNCH_TRIGGER_EARLY
-// keeps the trigger at the start.
-
+// on an mbarrier), so no register holds a load in flight and 5-6 calls' CTAs
+// share an SM (4.4 MB calls: 1.62 -> 1.26 us against register-held loads);
+// otherwise each lane loads its chunks into registers, all in flight at
+// once.  The contraction is the same masked dp4a form; warp sums put row r,
+// token m in lane r * MT + m, which dequantises and stores.  Everything but
+// the output stores precedes griddepcontrol.wait for LAUNCH_PDL_INPUTS.
 template <int MT, int R, int J, int NT, bool BULK>
-__global__ void __launch_bounds__(NT) gemv_stream_kernel(LinearParams p) {
+__global__ void __launch_bounds__(NT) gemv_flat_kernel(LinearParams p) {
   // shared memory: (BULK) the CTA's weight rows (NT / 32 * R rows of ldw
   // bytes, as stored), then the activation codes as [MT][4][C] 16-byte units:
   // unit u of a token row (its inputs 16u .. 16u + 15) sits in plane u % 4 at
