@@ -192,12 +192,15 @@ BITNET_API int bitnet_quant_act(const void *X, int x_dtype, int M, int K,
  *             codes c = t + 1 and subtract sum_k q).
  *   packed, gamma          outputs of bitnet_pack_weights() for [N][K].
  *   Y         out: [M][N] of the type in (epilogue & BITNET_EPI_TYPE_MASK):
- *             y = fp32( acc * gamma / s[m] ) (evaluated in fp64, rounded once),
- *             then the optional SiLU / residual add in fp32, then the cast.
+ *             y = fp32( acc * gamma / s[m] ), formed to ~2^-47 relative and
+ *             rounded once (the correctly rounded value except within ~2^-46
+ *             of an fp32 midpoint), then the optional SiLU / residual add in
+ *             fp32, then the cast.
  *   residual  [M][N] of Y's type when BITNET_EPI_RESIDUAL is set, else NULL.
- * M <= 2 (K a multiple of 64), or M <= 8 with N K <= 2^20, runs the dp4a streaming
- * GEMV, M <= 16 otherwise the cluster tensor-core GEMV (both HBM-bound), larger M
- * the tcgen05 GEMM.
+ * M <= 2 (K a multiple of 64), M <= 4 in a call without BITNET_LAUNCH_PDL_INPUTS
+ * and K <= 4096, or M <= 8 with N K <= 2^20, runs a dp4a streaming GEMV, M <= 16
+ * otherwise the cluster tensor-core GEMV (all HBM-bound), larger M the tcgen05
+ * GEMM.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
 BITNET_API int bitnet_linear(const int8_t *Xq, const float *x_scale, const int32_t *x_rowsum,
                   const uint8_t *packed, const float *gamma,

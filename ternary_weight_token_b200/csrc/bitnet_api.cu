@@ -581,23 +581,24 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
   const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64), <= 256
-  const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : 8;
+  const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
   // Independent calls (LAUNCH_PDL_INPUTS) and 3-8 tokens take the flat
   // kernel; independent calls on 4 MB of weights or more bulk-copy their
   // weight rows into shared memory there, so that more calls' CTAs share an
   // SM (1.6 MB single and 2.5 MB q/k/v calls measured slower with the bulk
   // copies, 4.4 MB ones faster).  Dependent calls take the row groups.
   const bool independent = (p.flags & LAUNCH_PDL_INPUTS) != 0;
-  if (independent || mt == 8) {
+  if (independent || mt == 8 || (mt == 4 && (long long)p.N * p.K <= (1ll << 20))) {
     // R rows per warp: about one CTA per SM per call, at most 8 chunks a lane
     const int warps = kFlatThreads / 32;
     int R = (p.N + di.sms * warps - 1) / (di.sms * warps);
     if (R > 8) R = 8;
     while (R > 1 && R * C > 32 * kStreamChunks) --R;
-    if (mt == 8 && R > 4) R = 4;                 // lane r * MT + m holds (row, token): R MT <= 32
+    const int mtf = mt == 4 ? 8 : mt;            // the flat kernel's token tiles: 1, 2, 8
+    if (mtf == 8 && R > 4) R = 4;                // lane r * MT + m holds (row, token): R MT <= 32
     const bool bulk = independent && (long long)p.N * p.ldw >= (1ll << 22);
-    if (mt == 1) return launch_flat_mt<1>(p, R, bulk, st);
-    if (mt == 2) return launch_flat_mt<2>(p, R, bulk, st);
+    if (mtf == 1) return launch_flat_mt<1>(p, R, bulk, st);
+    if (mtf == 2) return launch_flat_mt<2>(p, R, bulk, st);
     return launch_flat_mt<8>(p, R, bulk, st);
   }
   // L lanes per row (a power of two): each lane at most kStreamChunks chunks,
@@ -615,7 +616,8 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   const int rows = warps * G;
   const int grid = (p.N + rows - 1) / rows;
   if (mt == 1) return launch_stream_mt<1>(p, L, warps, grid, st);
-  return launch_stream_mt<2>(p, L, warps, grid, st);
+  if (mt == 2) return launch_stream_mt<2>(p, L, warps, grid, st);
+  return launch_stream_mt<4>(p, L, warps, grid, st);
 }
 
 // Projection i of a call as a call of its own.
@@ -648,15 +650,19 @@ bool token_tile_96(int M, int N) {
 }
 
 int launch_linear(const LinearParams& p, cudaStream_t st) {
-  // 1-2 tokens: the dp4a streaming kernel (measured faster than the cluster
-  // tensor-core path there; from 4 tokens on, its dp4a work and shared-memory
-  // reads sit on the critical path of dependent calls on the 2B shapes).  Up
-  // to 8 tokens on small weight matrices (<= 2^20 weights, e.g. 256 x 512):
-  // the streaming kernel too, whose short CTAs beat the cluster path's TMEM
-  // set-up and reduction there (6.2 -> 4.4 us per quantise + project pair).
-  // Both decode kernels run every projection of the call in one launch.
+  // 1-2 tokens: the dp4a streaming kernels (measured faster than the cluster
+  // tensor-core path there).  Up to 8 tokens on small weight matrices (<= 2^20
+  // weights, e.g. 256 x 512): the streaming kernels too, whose short CTAs beat
+  // the cluster path's TMEM set-up and reduction there (6.2 -> 4.4 us per
+  // quantise + project pair).  Every decode kernel runs all projections of
+  // the call in one launch.
   const bool stream_ok = p.K % 64 == 0 && p.ldw / 16 <= 32 * 8;
-  if (stream_ok && (p.M <= 2 || (p.M <= 8 && (long long)p.N * p.K <= (1ll << 20))))
+  // 3-4 tokens of a dependent call on rows of up to 4096 inputs: the
+  // row-group streaming kernel (dependent 3-4 token calls on 2560-input rows
+  // 4-9 % faster than the cluster tensor-core kernel; on 6912-input rows its
+  // lanes' chains are long and it was 7-11 % slower)
+  const bool dependent4 = p.M <= 4 && (p.flags & LAUNCH_PDL_INPUTS) == 0 && p.K <= 4096;
+  if (stream_ok && (p.M <= 2 || dependent4 || (p.M <= 8 && (long long)p.N * p.K <= (1ll << 20))))
     return launch_gemv_stream(p, st);
   if (p.M <= 16) {
     const int rc = launch_gemv_tc(p, st);
