@@ -433,11 +433,15 @@ __device__ __forceinline__ void grid_launch_dependents() {
 // --------------------------------------------------------------- misc ALU
 // SiLU y / (1 + e^-y) in fp32 ("bitnetv2-model" README, "Architecture
 // Overview"): CUDA's expf (the full-precision function, not the fast
-// intrinsic) and IEEE fp32 add and division, a few fp32 ulp from the exact
-// value.  One definition for every kernel that applies it, so the GEMM
-// epilogue and the quantiser prelude give the same value.
+// intrinsic), an IEEE fp32 add, and the quotient as y times the hardware
+// reciprocal (within 2 ulp; the IEEE division only for denominators beyond
+// 2^126, where the reciprocal flushes to zero): a few fp32 ulp from the
+// exact value.  One definition for every kernel that applies it, so the
+// GEMM epilogue and the quantiser prelude give the same value.
 __device__ __forceinline__ float silu_f32(float y) {
-  return __fdiv_rn(y, __fadd_rn(1.0f, expf(-y)));
+  const float d = __fadd_rn(1.0f, expf(-y));
+  if (d < 0x1p126f) return __fdividef(y, d);
+  return __fdiv_rn(y, d);
 }
 
 // Four unsigned bytes of `a` times four signed bytes of `b`, summed into c.
