@@ -46,7 +46,9 @@ PREFILL_M = 4096
 PREFILL_KN = ((2560, 6912), (6912, 2560))
 DECODE_M = (1, 4, 16)
 DECODE_KN = ((2560, 2560), (2560, 6912), (6912, 2560))
-GEMM_KERNEL_SRC = os.path.join(ROOT, "ternary_weight_token_b200", "csrc", "gemm_tc.cuh")
+# the prefill GEMM kernel and the headers whose device code it compiles in
+GEMM_KERNEL_SRCS = [os.path.join(ROOT, "ternary_weight_token_b200", "csrc", n)
+                    for n in ("gemm_tc.cuh", "gemv.cuh", "common.cuh")]
 GEMM_PROFILE = os.path.join(ROOT, "profiles", "gemm_tc_prefill_4096x2560x6912.md")
 
 
@@ -175,9 +177,14 @@ def measured_peaks():
             "source": "fallback"}
 
 
-def file_sha(path):
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def files_sha(paths):
+    """One hash over several files' names and contents."""
+    h = hashlib.sha256()
+    for path in paths:
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def nvtx_push(torch, name):
@@ -214,9 +221,9 @@ def profiled_traffic():
     if not os.path.exists(GEMM_PROFILE):
         return None
     txt = open(GEMM_PROFILE).read()
-    m_sha = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", txt)
+    m_sha = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]{16})", txt)
     m_b = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", txt)
-    if not m_sha or not m_b or m_sha.group(1) != file_sha(GEMM_KERNEL_SRC):
+    if not m_sha or not m_b or m_sha.group(1) != files_sha(GEMM_KERNEL_SRCS):
         return None
     return int(m_b.group(1))
 
