@@ -446,6 +446,7 @@ std::atomic<uint64_t> g_dec_attr_set{0};
 
 using TcPlain = TcConfig<128, 256, 4, false>;
 using TcPlain96 = TcConfig<96, 256, 4, false>;     // 96-token tiles (tile quantisation, below)
+using TcPlain64 = TcConfig<64, 256, 4, false>;     // 64-token tiles (single-wave calls, below)
 using TcSilu = TcConfig<128, 256, 4, false, true>;
 using TcGlu = TcConfig<128, 256, 4, true>;
 
@@ -635,18 +636,30 @@ LinearParams segment_params(const LinearParams& p, int i) {
 // a fixed part (converting its 128 weight rows, the epilogue's setup) plus a
 // part proportional to its tokens; timing 6912 -> 2560 at 4096 tokens with
 // 128- and 96-token tiles (5 and 6 waves: 61.8 and 68.5 us) puts the fixed
-// part at ~270 tokens' worth.  96-token tiles are taken when
-// waves x (tokens + 270) is clearly smaller: a last wave of 128-token tiles
-// that would leave most SMs idle, e.g. 2048 tokens x 2560 rows (320 tiles,
-// 3 waves; 440 tiles of 96, still 3 waves).
-bool token_tile_96(int M, int N) {
+// part at ~270 tokens' worth.  The token tile (128, 96 or 64 tokens) is the
+// one with the smallest waves x (tokens + 270), 128 unless another is clearly
+// (3 %) smaller.  96 takes a last wave of 128-token tiles that would leave
+// most SMs idle, e.g. 2048 tokens x 2560 rows (320 tiles, 3 waves; 440 tiles
+// of 96, still 3 waves); 64 wins on single-wave GEMMs with few row tiles,
+// e.g. 1024 tokens x 512 rows (64 tiles of 64 against 44 of 96: each CTA
+// multiplies and dequantises fewer tokens for the same weight stages; H-FFN
+// 25.5 -> 24.4 us).
+int token_tile(int M, int N) {
   DeviceInfo di;
-  if (device_info(di) != BITNET_OK || di.sms <= 0) return false;
+  if (device_info(di) != BITNET_OK || di.sms <= 0) return 128;
   auto cost = [&](int bn) {
     const long long tiles = (long long)((M + bn - 1) / bn) * ((N + 127) / 128);
     return ((tiles + di.sms - 1) / di.sms) * (bn + 270);
   };
-  return cost(96) * 100 < cost(128) * 97;
+  int best = 128;
+  long long best_cost = cost(128) * 97;
+  for (int bn : {96, 64}) {
+    if (cost(bn) * 100 < best_cost) {
+      best = bn;
+      best_cost = cost(bn) * 100;
+    }
+  }
+  return best;
 }
 
 int launch_linear(const LinearParams& p, cudaStream_t st) {
@@ -678,8 +691,9 @@ int launch_linear(const LinearParams& p, cudaStream_t st) {
       rc = launch_gemv(q, st);
     } else if (q.flags & EPI_SILU) {
       rc = launch_tc_cfg<TcSilu>(q, nullptr, nullptr, st);
-    } else if (token_tile_96(q.M, q.N)) {
-      rc = launch_tc_cfg<TcPlain96>(q, nullptr, nullptr, st);
+    } else if (const int bn = token_tile(q.M, q.N); bn != 128) {
+      rc = bn == 96 ? launch_tc_cfg<TcPlain96>(q, nullptr, nullptr, st)
+                    : launch_tc_cfg<TcPlain64>(q, nullptr, nullptr, st);
     } else {
       rc = launch_tc_cfg<TcPlain>(q, nullptr, nullptr, st);
     }
