@@ -480,17 +480,32 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   }
   for (int i = lp.nseg; i <= kMaxSegments; ++i) p.seg_tile0[i] = tiles;
   for (int i = lp.nseg; i < kMaxSegments; ++i) maps.w[i] = maps.w[0];
-  // The cluster size S: at least one CTA per SM.  When the activation codes
-  // come from the preceding kernel (a programmatic dependent launch without
-  // LAUNCH_PDL_INPUTS), a CTA converts at most three weight chunks (its
-  // ring of TMEM slots) before they arrive, and every further chunk costs a
-  // round trip between the MMA and the converter warps after that.  For a
-  // few tokens, where the cross-CTA reduction is cheap, S then grows until a
-  // CTA's slice fits the ring (three chunks, six 64-input units).
+  // The cluster size S grows from the smallest split until the call has at
+  // least half a CTA per SM, and for more than 8 tokens until a CTA's slice
+  // is at most ten 64-input units while the call stays within two CTAs per
+  // SM: more, shorter CTAs do not pay (2560 x 2560 with 80 CTAs of ten units
+  // against 160 of five: 3-4 % faster at 3-8 tokens, 11 % at 16; 16 tokens on
+  // 2560 x 6912 with 216 CTAs of ten units instead of 162 of fourteen: 4-5 %
+  // faster, while up to 8 tokens run best on fourteen; on 2560 x 13824 the
+  // 432 CTAs of ten units were no faster).  When the activation codes come
+  // from the preceding kernel (a programmatic dependent launch without
+  // LAUNCH_PDL_INPUTS), a CTA converts at most three weight chunks (its ring
+  // of TMEM slots) before they arrive, and every further chunk costs a round
+  // trip between the MMA and the converter warps after that; for up to 8
+  // tokens, where the cross-CTA reduction is cheap, such a call takes a CTA
+  // per SM and slices that fit the ring (three chunks, six units).
   const bool dependent = (lp.flags & LAUNCH_PDL) && !(lp.flags & LAUNCH_PDL_INPUTS);
-  const int units_fit = dependent && lp.M <= 8 ? 6 : 1 << 30;
+  const bool few = lp.M <= 8;
+  const int units_fit = dependent && few ? 6 : 1 << 30;
+  const int min_ctas = dependent && few ? di.sms : (di.sms + 1) / 2;
   int S = s_min;
-  while (S < s_max && (tiles * S < di.sms || (units + S - 1) / S > units_fit)) ++S;
+  while (S < s_max) {
+    const int slice = (units + S - 1) / S;
+    const bool grow = tiles * S < min_ctas || slice > units_fit ||
+                      (!few && slice > 10 && tiles * (S + 1) <= 2 * di.sms);
+    if (!grow) break;
+    ++S;
+  }
   CUtensorMap mx;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 kDecTokens, CU_TENSOR_MAP_SWIZZLE_128B))
