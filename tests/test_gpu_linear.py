@@ -330,15 +330,19 @@ def test_independent_multi_projection_bulk_rows(M, K, Ns):
     assert bn.bitnet_check_device_error() == bn.BITNET_OK
 
 
+@pytest.mark.parametrize("flags", [0, bn.BITNET_LAUNCH_PDL, bn.BITNET_LAUNCH_PDL_INPUTS],
+                         ids=["plain", "pdl", "pdl_inputs"])
 @pytest.mark.parametrize("K,N", [(2560, 2560), (2560, 6912), (6912, 2560)])
-def test_decode_shapes_all_m(K, N):
-    """The 2B-model decode shapes for every token count 1..16 (cluster split-K
-    tensor-core path), int32 bit-exact."""
+def test_decode_shapes_all_m(K, N, flags):
+    """The 2B-model decode shapes for every token count 1..16, int32
+    bit-exact, in each launch mode: the mode and the token count pick the
+    kernel (streaming, flat or cluster tensor-core) and the cluster split
+    (3, 4, 7 or 8 CTAs per 128-row tile on these shapes)."""
     rng_w, rng_x = synthetic.streams(K + N, 2)
     W = synthetic.weight(rng_w, N, K)
     g, T, P = oracle.quantize_weights(W)
     X = synthetic.activations(rng_x, 16, K)
     q, s, rs = oracle.quant_act(X)
-    for M in (1, 2, 3, 5, 8, 13, 16):
-        got = gpu_linear(q[:M], s[:M], rs[:M], P, g, K, N, out=torch.int32)
+    for M in (1, 2, 3, 4, 5, 8, 9, 13, 16):
+        got = gpu_linear(q[:M], s[:M], rs[:M], P, g, K, N, out=torch.int32, flags=flags)
         np.testing.assert_array_equal(got, oracle.contract(q[:M], T), err_msg=f"M={M}")
