@@ -623,10 +623,14 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   }
   // L lanes per row (a power of two): each lane at most kStreamChunks chunks,
   // and on small matrices more lanes per row, so that the call still has
-  // about 256 lanes per SM (a row has C chunks: no more than C lanes)
+  // about 256 lanes per SM, 128 for 3-4 tokens, whose longer per-lane sums
+  // pay off there (2560 x 2560, dependent: 5.05 -> 4.69 us at 4 tokens; 1-2
+  // tokens were 3-6 % slower with 128) (a row has C chunks: no more than C
+  // lanes)
+  const long long lanes_per_sm = mt == 4 ? 128 : 256;
   int L = 1;
   while (L * kStreamChunks < C) L *= 2;
-  while (L < 32 && L < C && (long long)p.N * L < (long long)di.sms * 256) L *= 2;
+  while (L < 32 && L < C && (long long)p.N * L < (long long)di.sms * lanes_per_sm) L *= 2;
   const int G = 32 / L;                        // rows per warp
   // warps per CTA: about one CTA per SM per call (so several back-to-back
   // calls can be resident at once), at most 8
