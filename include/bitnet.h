@@ -208,6 +208,28 @@ BITNET_API int bitnet_linear(const int8_t *Xq, const float *x_scale, const int32
                   void *Y, int epilogue, const void *residual,
                   bitnet_stream_t stream);
 
+/* Kernels of a launch plan (bitnet_plan_linear). */
+#define BITNET_PLAN_STREAM   1  /* row-group dp4a streaming GEMV                 */
+#define BITNET_PLAN_FLAT     2  /* flat dp4a streaming GEMV                      */
+#define BITNET_PLAN_GEMV_TC  3  /* cluster split-K tensor-core GEMV              */
+#define BITNET_PLAN_GEMV     4  /* plain dp4a GEMV (decode K the others refuse)  */
+#define BITNET_PLAN_GEMM_TC  5  /* persistent tcgen05 GEMM                       */
+
+/* The launch plan bitnet_linear() follows for one projection on a device with
+ * `sms` SMs: host logic only (no launch, no device access), for tests and
+ * tooling.  epilogue as bitnet_linear() (its flags choose the plan).
+ *   out[0]  kernel, BITNET_PLAN_*
+ *   out[1]  tokens per pass: decode kernels' token tile (1, 2, 4, 8, 16), the
+ *           GEMM's tile (128, 96 or 64 tokens)
+ *   out[2]  CTAs (the plain GEMV: before its occupancy cap)
+ *   out[3], out[4]
+ *           STREAM: lanes per row, warps per CTA; FLAT: rows per warp, bulk
+ *           weight copies (0 / 1); GEMV_TC: cluster size, 128-row tiles;
+ *           GEMM_TC: tiles, 0; GEMV: 0, 0
+ * Errors: INVALID_ARG (out NULL, M, N or sms not positive, K as for
+ * bitnet_linear()). */
+BITNET_API int bitnet_plan_linear(int M, int N, int K, int epilogue, int sms, int *out);
+
 /* Several projections of one quantised input in one call -- the q, k and v
  * projections of an attention block (2560 -> 2560 + 640 + 640 in the 2B
  * model, nnterp "bitnet", "Printout"), or gate and up -- as bitnet_linear()

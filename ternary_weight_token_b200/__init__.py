@@ -33,6 +33,11 @@ from ._binding import (  # noqa: F401
     BITNET_LAUNCH_PDL,
     BITNET_LAUNCH_PDL_INPUTS,
     BITNET_OK,
+    BITNET_PLAN_FLAT,
+    BITNET_PLAN_GEMM_TC,
+    BITNET_PLAN_GEMV,
+    BITNET_PLAN_GEMV_TC,
+    BITNET_PLAN_STREAM,
     BITNET_PRELUDE_FWHT,
     BITNET_PRELUDE_NONE,
     BITNET_PRELUDE_RMSNORM,
@@ -57,6 +62,7 @@ from ._binding import (  # noqa: F401
     bitnet_pack_weights,
     bitnet_pack_workspace_size,
     bitnet_packed_row_bytes,
+    bitnet_plan_linear,
     bitnet_quant_act,
     bitnet_release_cache,
     bitnet_version,

@@ -23,6 +23,8 @@ BITNET_LAUNCH_PDL = 0x100
 BITNET_LAUNCH_PDL_INPUTS = 0x200
 BITNET_FFN_RELU2_GLU, BITNET_FFN_HADAMARD_SILU = 0, 1
 BITNET_FFN_SINGLE_LAUNCH = 0x200
+(BITNET_PLAN_STREAM, BITNET_PLAN_FLAT, BITNET_PLAN_GEMV_TC, BITNET_PLAN_GEMV,
+ BITNET_PLAN_GEMM_TC) = 1, 2, 3, 4, 5
 
 _DTYPE_CODE = {torch.float32: BITNET_F32, torch.bfloat16: BITNET_BF16, torch.int32: BITNET_I32}
 
@@ -60,6 +62,7 @@ def library():
         "bitnet_import_tw2": (I, [P, I, I, P, P]),
         "bitnet_quant_act": (I, [P, I, I, I, I, P, F, P, P, P, P]),
         "bitnet_linear": (I, [P, P, P, P, P, I, I, I, P, I, P, P]),
+        "bitnet_plan_linear": (I, [I, I, I, I, I, P]),
         "bitnet_ffn_workspace_size": (S, [I, I, I, I]),
         "bitnet_ffn": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P, S, P]),
         "bitnet_ffn_noalloc": (I, [P, I, I, I, I, P, P, P, P, P, P, P, P, F, I, P, I, P]),
@@ -137,6 +140,15 @@ def bitnet_version():
 
 def bitnet_release_cache():
     library().bitnet_release_cache()
+
+
+def bitnet_plan_linear(M, N, K, epilogue=BITNET_BF16, sms=148):
+    """The launch plan bitnet_linear() follows for one projection on a device
+    with `sms` SMs (host logic only): a dict with the kernel (BITNET_PLAN_*),
+    its token tile, CTAs and two kernel-specific values (see the header)."""
+    out = (ctypes.c_int * 5)()
+    _check(library().bitnet_plan_linear(int(M), int(N), int(K), int(epilogue), int(sms), out))
+    return {"kernel": out[0], "tokens": out[1], "grid": out[2], "a": out[3], "b": out[4]}
 
 
 # ------------------------------------------------------------- device calls

@@ -450,17 +450,53 @@ using TcPlain64 = TcConfig<64, 256, 4, false>;     // 64-token tiles (single-wav
 using TcSilu = TcConfig<128, 256, 4, false, true>;
 using TcGlu = TcConfig<128, 256, 4, true>;
 
+// The cluster size S of the tensor-core decode GEMV for a call of `tiles`
+// 128-row weight tiles, or 0 when K does not split (K not a multiple of 64,
+// or more than 8 slices of at most 14 64-input units needed).  Pure host
+// logic, shared by the launch and bitnet_plan_linear.
+int decode_cluster_size(int M, int K, int tiles, int flags, int sms) {
+  const int units = K / 64;
+  if (K % 64 != 0 || units < 1) return 0;
+  const int s_min = (units + 13) / 14;                    // ceil(units / S) <= 14
+  const int s_max = units < kDecMaxCluster ? units : kDecMaxCluster;
+  if (s_min > s_max) return 0;
+  // The cluster size S grows from the smallest split until the call has at
+  // least half a CTA per SM, and for more than 8 tokens until a CTA's slice
+  // is at most ten 64-input units while the call stays within two CTAs per
+  // SM: more, shorter CTAs do not pay (2560 x 2560 with 80 CTAs of ten units
+  // against 160 of five: 3-4 % faster at 3-8 tokens, 11 % at 16; 16 tokens on
+  // 2560 x 6912 with 216 CTAs of ten units instead of 162 of fourteen: 4-5 %
+  // faster, while up to 8 tokens run best on fourteen; on 2560 x 13824 the
+  // 432 CTAs of ten units were no faster).  When the activation codes come
+  // from the preceding kernel (a programmatic dependent launch without
+  // LAUNCH_PDL_INPUTS), a CTA converts at most three weight chunks (its ring
+  // of TMEM slots) before they arrive, and every further chunk costs a round
+  // trip between the MMA and the converter warps after that; for up to 8
+  // tokens, where the cross-CTA reduction is cheap, such a call takes a CTA
+  // per SM and slices that fit the ring (three chunks, six units).
+  const bool dependent = (flags & LAUNCH_PDL) && !(flags & LAUNCH_PDL_INPUTS);
+  const bool few = M <= 8;
+  const int units_fit = dependent && few ? 6 : 1 << 30;
+  const int min_ctas = dependent && few ? sms : (sms + 1) / 2;
+  int S = s_min;
+  while (S < s_max) {
+    const int slice = (units + S - 1) / S;
+    const bool grow = tiles * S < min_ctas || slice > units_fit ||
+                      (!few && slice > 10 && tiles * (S + 1) <= 2 * sms);
+    if (!grow) break;
+    ++S;
+  }
+  return S;
+}
+
 // Decode on the tensor cores: 128-row weight tiles, each split over K across a
 // cluster of S CTAs (S <= 8, every slice at most 896 inputs).  Returns
 // BITNET_ERR_UNSUPPORTED when K is too long for that split.
 int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   DeviceInfo di;
   if (int rc = device_info(di)) return rc;
+  if (decode_cluster_size(lp.M, lp.K, 1, lp.flags, di.sms) == 0) return BITNET_ERR_UNSUPPORTED;
   const int units = lp.K / 64;
-  if (lp.K % 64 != 0 || units < 1) return BITNET_ERR_UNSUPPORTED;
-  const int s_min = (units + 13) / 14;                    // ceil(units / S) <= 14
-  const int s_max = units < kDecMaxCluster ? units : kDecMaxCluster;
-  if (s_min > s_max) return BITNET_ERR_UNSUPPORTED;
   // every projection of the call: its 128-row tiles and packed-weight map
   DecParams p;
   DecMaps maps;
@@ -480,32 +516,8 @@ int launch_gemv_tc(const LinearParams& lp, cudaStream_t st) {
   }
   for (int i = lp.nseg; i <= kMaxSegments; ++i) p.seg_tile0[i] = tiles;
   for (int i = lp.nseg; i < kMaxSegments; ++i) maps.w[i] = maps.w[0];
-  // The cluster size S grows from the smallest split until the call has at
-  // least half a CTA per SM, and for more than 8 tokens until a CTA's slice
-  // is at most ten 64-input units while the call stays within two CTAs per
-  // SM: more, shorter CTAs do not pay (2560 x 2560 with 80 CTAs of ten units
-  // against 160 of five: 3-4 % faster at 3-8 tokens, 11 % at 16; 16 tokens on
-  // 2560 x 6912 with 216 CTAs of ten units instead of 162 of fourteen: 4-5 %
-  // faster, while up to 8 tokens run best on fourteen; on 2560 x 13824 the
-  // 432 CTAs of ten units were no faster).  When the activation codes come
-  // from the preceding kernel (a programmatic dependent launch without
-  // LAUNCH_PDL_INPUTS), a CTA converts at most three weight chunks (its ring
-  // of TMEM slots) before they arrive, and every further chunk costs a round
-  // trip between the MMA and the converter warps after that; for up to 8
-  // tokens, where the cross-CTA reduction is cheap, such a call takes a CTA
-  // per SM and slices that fit the ring (three chunks, six units).
-  const bool dependent = (lp.flags & LAUNCH_PDL) && !(lp.flags & LAUNCH_PDL_INPUTS);
-  const bool few = lp.M <= 8;
-  const int units_fit = dependent && few ? 6 : 1 << 30;
-  const int min_ctas = dependent && few ? di.sms : (di.sms + 1) / 2;
-  int S = s_min;
-  while (S < s_max) {
-    const int slice = (units + S - 1) / S;
-    const bool grow = tiles * S < min_ctas || slice > units_fit ||
-                      (!few && slice > 10 && tiles * (S + 1) <= 2 * di.sms);
-    if (!grow) break;
-    ++S;
-  }
+  const int S = decode_cluster_size(lp.M, lp.K, tiles, lp.flags, di.sms);
+  if (S == 0) return BITNET_ERR_UNSUPPORTED;
   CUtensorMap mx;
   if (int rc = tensor_map_2d_u8(mx, lp.Xq, (uint64_t)lp.K, (uint64_t)lp.M, (uint64_t)lp.K, 128,
                                 kDecTokens, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -593,33 +605,43 @@ int launch_flat_mt(const LinearParams& p, int R, bool bulk, cudaStream_t st) {
                        st, q);
 }
 
-int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
-  DeviceInfo di;
-  if (int rc = device_info(di)) return rc;
-  const int C = p.ldw / 16;                    // 16-byte chunks per row (K / 64), <= 256
-  const int mt = p.M <= 1 ? 1 : p.M <= 2 ? 2 : p.M <= 4 ? 4 : 8;
+// Launch shape of the streaming decode kernels for a call (pure host logic,
+// shared by the launch and bitnet_plan_linear): the flat kernel (`flat`,
+// token tile mt, R rows per warp, bulk-copied rows) or the row groups (L
+// lanes per row, `warps` warps per CTA); `grid` CTAs.
+struct StreamShape {
+  bool flat = false, bulk = false;
+  int mt = 1, R = 1, L = 1, warps = 1, grid = 0;
+};
+
+StreamShape stream_shape(int M, int N, int K, int ldw, int flags, int sms) {
+  StreamShape sh;
+  const int C = ldw / 16;                      // 16-byte chunks per row (K / 64), <= 256
+  const int mt = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : 8;
   // Independent calls (LAUNCH_PDL_INPUTS) and 3-8 tokens take the flat
   // kernel; independent calls on 4 MB of weights or more bulk-copy their
   // weight rows into shared memory there, so that more calls' CTAs share an
   // SM (1.6 MB single and 2.5 MB q/k/v calls measured slower with the bulk
   // copies, 4.4 MB ones faster).  Dependent calls take the row groups.
-  const bool independent = (p.flags & LAUNCH_PDL_INPUTS) != 0;
-  if (independent || mt == 8 || (mt == 4 && (long long)p.N * p.K <= (1ll << 20))) {
+  const bool independent = (flags & LAUNCH_PDL_INPUTS) != 0;
+  if (independent || mt == 8 || (mt == 4 && (long long)N * K <= (1ll << 20))) {
     // R rows per warp: about one CTA per two SMs per call (fewer, fuller CTAs
     // let more back-to-back calls overlap: independent 1-2 token calls on
     // 2560 x 2560 0.88 -> 0.81 / 1.49 -> 1.31 us and the q/k/v step 1.15 ->
     // 1.08 us against a CTA per SM), at most 8 chunks a lane
     const int warps = kFlatThreads / 32;
-    const int half = (di.sms + 1) / 2;
-    int R = (p.N + half * warps - 1) / (half * warps);
+    const int half = (sms + 1) / 2;
+    int R = (N + half * warps - 1) / (half * warps);
     if (R > 8) R = 8;
     while (R > 1 && R * C > 32 * kStreamChunks) --R;
-    const int mtf = mt == 4 ? 8 : mt;            // the flat kernel's token tiles: 1, 2, 8
-    if (mtf == 8 && R > 4) R = 4;                // lane r * MT + m holds (row, token): R MT <= 32
-    const bool bulk = independent && (long long)p.N * p.ldw >= (1ll << 22);
-    if (mtf == 1) return launch_flat_mt<1>(p, R, bulk, st);
-    if (mtf == 2) return launch_flat_mt<2>(p, R, bulk, st);
-    return launch_flat_mt<8>(p, R, bulk, st);
+    sh.mt = mt == 4 ? 8 : mt;                  // the flat kernel's token tiles: 1, 2, 8
+    if (sh.mt == 8 && R > 4) R = 4;            // lane r * MT + m holds (row, token): R MT <= 32
+    sh.flat = true;
+    sh.R = R;
+    sh.warps = warps;
+    sh.bulk = independent && (long long)N * ldw >= (1ll << 22);
+    sh.grid = (N + warps * R - 1) / (warps * R);
+    return sh;
   }
   // L lanes per row (a power of two): each lane at most kStreamChunks chunks,
   // and on small matrices more lanes per row, so that the call still has
@@ -630,18 +652,33 @@ int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
   const long long lanes_per_sm = mt == 4 ? 128 : 256;
   int L = 1;
   while (L * kStreamChunks < C) L *= 2;
-  while (L < 32 && L < C && (long long)p.N * L < (long long)di.sms * lanes_per_sm) L *= 2;
+  while (L < 32 && L < C && (long long)N * L < (long long)sms * lanes_per_sm) L *= 2;
   const int G = 32 / L;                        // rows per warp
   // warps per CTA: about one CTA per SM per call (so several back-to-back
   // calls can be resident at once), at most 8
-  int warps = p.N / (di.sms * G);
+  int warps = N / (sms * G);
   if (warps > 8) warps = 8;
   if (warps < 1) warps = 1;
   const int rows = warps * G;
-  const int grid = (p.N + rows - 1) / rows;
-  if (mt == 1) return launch_stream_mt<1>(p, L, warps, grid, st);
-  if (mt == 2) return launch_stream_mt<2>(p, L, warps, grid, st);
-  return launch_stream_mt<4>(p, L, warps, grid, st);
+  sh.mt = mt;
+  sh.L = L;
+  sh.warps = warps;
+  sh.grid = (N + rows - 1) / rows;
+  return sh;
+}
+
+int launch_gemv_stream(const LinearParams& p, cudaStream_t st) {
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
+  const StreamShape sh = stream_shape(p.M, p.N, p.K, p.ldw, p.flags, di.sms);
+  if (sh.flat) {
+    if (sh.mt == 1) return launch_flat_mt<1>(p, sh.R, sh.bulk, st);
+    if (sh.mt == 2) return launch_flat_mt<2>(p, sh.R, sh.bulk, st);
+    return launch_flat_mt<8>(p, sh.R, sh.bulk, st);
+  }
+  if (sh.mt == 1) return launch_stream_mt<1>(p, sh.L, sh.warps, sh.grid, st);
+  if (sh.mt == 2) return launch_stream_mt<2>(p, sh.L, sh.warps, sh.grid, st);
+  return launch_stream_mt<4>(p, sh.L, sh.warps, sh.grid, st);
 }
 
 // Projection i of a call as a call of its own.
@@ -667,12 +704,11 @@ LinearParams segment_params(const LinearParams& p, int i) {
 // e.g. 1024 tokens x 512 rows (64 tiles of 64 against 44 of 96: each CTA
 // multiplies and dequantises fewer tokens for the same weight stages; H-FFN
 // 25.5 -> 24.4 us).
-int token_tile(int M, int N) {
-  DeviceInfo di;
-  if (device_info(di) != BITNET_OK || di.sms <= 0) return 128;
+int token_tile(int M, int N, int sms) {
+  if (sms <= 0) return 128;
   auto cost = [&](int bn) {
     const long long tiles = (long long)((M + bn - 1) / bn) * ((N + 127) / 128);
-    return ((tiles + di.sms - 1) / di.sms) * (bn + 270);
+    return ((tiles + sms - 1) / sms) * (bn + 270);
   };
   int best = 128;
   long long best_cost = cost(128) * 97;
@@ -685,27 +721,32 @@ int token_tile(int M, int N) {
   return best;
 }
 
+// Whether a call takes the streaming decode kernels (pure host logic).
+// 1-2 tokens: the dp4a streaming kernels (measured faster than the cluster
+// tensor-core path there).  Up to 8 tokens on small weight matrices (<= 2^20
+// weights, e.g. 256 x 512): the streaming kernels too, whose short CTAs beat
+// the cluster path's TMEM set-up and reduction there (6.2 -> 4.4 us per
+// quantise + project pair).  3-4 tokens of a dependent call on rows of up to
+// 4096 inputs: the row-group streaming kernel (dependent 3-4 token calls on
+// 2560-input rows 4-9 % faster than the cluster tensor-core kernel; on
+// 6912-input rows its lanes' chains are long and it was 7-11 % slower).
+bool takes_stream(int M, int N, int K, int ldw, int flags) {
+  const bool stream_ok = K % 64 == 0 && ldw / 16 <= 32 * 8;
+  const bool dependent4 = M <= 4 && (flags & LAUNCH_PDL_INPUTS) == 0 && K <= 4096;
+  return stream_ok && (M <= 2 || dependent4 || (M <= 8 && (long long)N * K <= (1ll << 20)));
+}
+
 int launch_linear(const LinearParams& p, cudaStream_t st) {
-  // 1-2 tokens: the dp4a streaming kernels (measured faster than the cluster
-  // tensor-core path there).  Up to 8 tokens on small weight matrices (<= 2^20
-  // weights, e.g. 256 x 512): the streaming kernels too, whose short CTAs beat
-  // the cluster path's TMEM set-up and reduction there (6.2 -> 4.4 us per
-  // quantise + project pair).  Every decode kernel runs all projections of
-  // the call in one launch.
-  const bool stream_ok = p.K % 64 == 0 && p.ldw / 16 <= 32 * 8;
-  // 3-4 tokens of a dependent call on rows of up to 4096 inputs: the
-  // row-group streaming kernel (dependent 3-4 token calls on 2560-input rows
-  // 4-9 % faster than the cluster tensor-core kernel; on 6912-input rows its
-  // lanes' chains are long and it was 7-11 % slower)
-  const bool dependent4 = p.M <= 4 && (p.flags & LAUNCH_PDL_INPUTS) == 0 && p.K <= 4096;
-  if (stream_ok && (p.M <= 2 || dependent4 || (p.M <= 8 && (long long)p.N * p.K <= (1ll << 20))))
-    return launch_gemv_stream(p, st);
+  // Every decode kernel runs all projections of the call in one launch.
+  if (takes_stream(p.M, p.N, p.K, p.ldw, p.flags)) return launch_gemv_stream(p, st);
   if (p.M <= 16) {
     const int rc = launch_gemv_tc(p, st);
     if (rc != BITNET_ERR_UNSUPPORTED) return rc;
   }
   // one launch per projection: the prefill GEMM, or decode inputs too long
   // for the cluster split (the plain dp4a kernel)
+  DeviceInfo di;
+  if (int rc = device_info(di)) return rc;
   for (int i = 0; i < p.nseg; ++i) {
     LinearParams q = segment_params(p, i);
     int rc;
@@ -714,7 +755,7 @@ int launch_linear(const LinearParams& p, cudaStream_t st) {
       rc = launch_gemv(q, st);
     } else if (q.flags & EPI_SILU) {
       rc = launch_tc_cfg<TcSilu>(q, nullptr, nullptr, st);
-    } else if (const int bn = token_tile(q.M, q.N); bn != 128) {
+    } else if (const int bn = token_tile(q.M, q.N, di.sms); bn != 128) {
       rc = bn == 96 ? launch_tc_cfg<TcPlain96>(q, nullptr, nullptr, st)
                     : launch_tc_cfg<TcPlain64>(q, nullptr, nullptr, st);
     } else {
@@ -978,6 +1019,47 @@ int bitnet_quant_act(const void* X, int x_dtype, int M, int K, int prelude,
     return fail(BITNET_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   return launch_quant(X, x_dtype == BITNET_BF16, M, K, prelude, norm_gain, eps, Xq, x_scale,
                       x_rowsum, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitnet_plan_linear(int M, int N, int K, int epilogue, int sms, int* out) {
+  g_last_error.clear();
+  if (out == nullptr) return fail(BITNET_ERR_INVALID_ARG, "out is NULL");
+  if (M <= 0 || N <= 0 || sms <= 0)
+    return fail(BITNET_ERR_INVALID_ARG, "M=%d, N=%d and sms=%d must be positive", M, N, sms);
+  if (int rc = check_k(K)) return rc;
+  const int ldw = (int)bitnet_packed_row_bytes(K);
+  const int flags = epilogue & ~BITNET_EPI_TYPE_MASK;
+  int o[5] = {0, 0, 0, 0, 0};
+  const int tiles_n = (N + 127) / 128;
+  int S = 0;
+  if (takes_stream(M, N, K, ldw, flags)) {
+    const StreamShape sh = stream_shape(M, N, K, ldw, flags, sms);
+    o[0] = sh.flat ? BITNET_PLAN_FLAT : BITNET_PLAN_STREAM;
+    o[1] = sh.mt;
+    o[2] = sh.grid;
+    o[3] = sh.flat ? sh.R : sh.L;
+    o[4] = sh.flat ? (sh.bulk ? 1 : 0) : sh.warps;
+  } else if (M <= 16 && (S = decode_cluster_size(M, K, tiles_n, flags, sms)) > 0) {
+    o[0] = BITNET_PLAN_GEMV_TC;
+    o[1] = kDecTokens;
+    o[2] = tiles_n * S;
+    o[3] = S;
+    o[4] = tiles_n;
+  } else if (M <= 16) {
+    const int rows_per_cta = (kGemvThreads / 32) * kGemvRows;
+    o[0] = BITNET_PLAN_GEMV;
+    o[1] = M <= 1 ? 1 : M <= 2 ? 2 : M <= 4 ? 4 : M <= 8 ? 8 : 16;
+    o[2] = (N + rows_per_cta - 1) / rows_per_cta;
+  } else {
+    const int bn = (flags & EPI_SILU) ? 128 : token_tile(M, N, sms);
+    const int tiles = ((M + bn - 1) / bn) * tiles_n;
+    o[0] = BITNET_PLAN_GEMM_TC;
+    o[1] = bn;
+    o[2] = tiles < sms ? tiles : sms;
+    o[3] = tiles;
+  }
+  for (int k = 0; k < 5; ++k) out[k] = o[k];
+  return BITNET_OK;
 }
 
 int bitnet_linear(const int8_t* Xq, const float* x_scale, const int32_t* x_rowsum,
